@@ -80,7 +80,7 @@ uint16_t orc_f64_to_f16(double v) {
 // Appendix E.1 (the 8-bit RTN model is the parent of every truncated width).
 // Library convention: s = fp16(range / 255) rounded to nearest even straight
 // from fp64, s := 1 if that rounds to 0, s := 65504 if it overflows;
-// z = clamp(rne(-min / s), 0, 255) stored as fp16 (exact);
+// z = clamp(rne(-min / s), 0, 255) stored as fp16 (exact, and +0 rather than -0);
 // q = clamp(rne(w / s) + z, 0, 255). Quotients are taken in fp64; for a binary32
 // numerator and a binary16 denominator the fp64 quotient never lands on, or
 // crosses, a half-integer that the exact quotient does not, so rne of it equals
@@ -108,6 +108,7 @@ int orc_rtn_quantize(const float* W, int K, int N, uint8_t* q, uint16_t* scale, 
       double z = std::nearbyint(-mn / s);
       if (z < 0.0) z = 0.0;
       if (z > 255.0) z = 255.0;
+      z = z + 0.0;   // a zero point of -0 (min = +0) is stored as +0
       scale[(size_t)k * ng + g] = sb;
       zero[(size_t)k * ng + g] = orc_f64_to_f16(z);
       for (int n = c0; n < c1; ++n) {
