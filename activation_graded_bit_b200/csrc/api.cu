@@ -1,0 +1,256 @@
+// C ABI of the GRINQH library: argument validation on the host, then launches.
+// Every check happens before anything is enqueued, so a rejected call leaves the
+// stream untouched. See include/grinqh.h for the contract of each call.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "../../include/grinqh.h"
+#include "kernels.h"
+
+using namespace grinqh;
+
+namespace {
+
+constexpr int64_t kMaxDim = int64_t(1) << 24;
+constexpr int64_t kMaxElems = int64_t(1) << 34;
+constexpr int kTileN = 512;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+grinqh_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GRINQH_OK : GRINQH_ERR_CUDA; }
+
+bool valid_classes(const uint8_t* classes, int32_t n) {
+  if (!classes || n < 1 || n > GRINQH_MAX_CLASSES) return false;
+  for (int i = 0; i < n; ++i) {
+    if (classes[i] > 8) return false;
+    if (i > 0 && classes[i] <= classes[i - 1]) return false;
+  }
+  return true;
+}
+
+bool layout_ok(const grinqh_layout* L) {
+  if (!L) return false;
+  grinqh_layout ref;
+  if (grinqh_layout_init(L->K, L->N, &ref) != GRINQH_OK) return false;
+  return std::memcmp(&ref, L, sizeof(ref)) == 0;
+}
+
+ClassTable table(const uint8_t* classes, int32_t n) {
+  ClassTable t{};
+  t.n = n;
+  for (int i = 0; i < n; ++i) t.width[i] = classes[i];
+  return t;
+}
+
+// Maximum-entropy distribution p_i ~ exp(lam * b_i) with mean target (host).
+void gibbs(const uint8_t* b, int m, double lam, double* p) {
+  const double c = lam >= 0.0 ? (double)b[m - 1] : (double)b[0];
+  double z = 0.0;
+  for (int i = 0; i < m; ++i) {
+    p[i] = std::exp(lam * ((double)b[i] - c));
+    z += p[i];
+  }
+  for (int i = 0; i < m; ++i) p[i] /= z;
+}
+
+double mean_width(const uint8_t* b, int m, const double* p) {
+  double s = 0.0;
+  for (int i = 0; i < m; ++i) s += p[i] * (double)b[i];
+  return s;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* grinqh_version(void) { return "grinqh-b200 0.1.0 (sm_100a)"; }
+
+const char* grinqh_status_string(grinqh_status s) {
+  switch (s) {
+    case GRINQH_OK: return "ok";
+    case GRINQH_ERR_INVALID_ARG: return "invalid argument";
+    case GRINQH_ERR_ALIGNMENT: return "misaligned pointer";
+    case GRINQH_ERR_UNSUPPORTED: return "unsupported";
+    case GRINQH_ERR_WORKSPACE: return "workspace missing or too small";
+    case GRINQH_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+grinqh_status grinqh_layout_init(int32_t K, int32_t N, grinqh_layout* out) {
+  if (!out) return GRINQH_ERR_INVALID_ARG;
+  if (K < 1 || N < 1 || K > kMaxDim || N > kMaxDim) return GRINQH_ERR_INVALID_ARG;
+  if ((int64_t)K * N > kMaxElems) return GRINQH_ERR_INVALID_ARG;
+  grinqh_layout L;
+  std::memset(&L, 0, sizeof(L));
+  L.K = K;
+  L.N = N;
+  L.n_groups = (N + GRINQH_GROUP - 1) / GRINQH_GROUP;
+  L.tile_n = kTileN;
+  L.n_tiles = (N + kTileN - 1) / kTileN;
+  L.meta_stride = L.n_tiles * (kTileN / GRINQH_GROUP);
+  L.planes_bytes = (int64_t)L.n_tiles * K * kTileN;
+  L.meta_bytes = (int64_t)4 * K * L.meta_stride;
+  *out = L;
+  return GRINQH_OK;
+}
+
+grinqh_status grinqh_pack(const grinqh_layout* layout, const float* W, void* planes, uint32_t* meta,
+                          void* stream) {
+  if (!layout_ok(layout) || !W || !planes || !meta) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(W, 4) || !aligned(planes, 16) || !aligned(meta, 16)) return GRINQH_ERR_ALIGNMENT;
+  const grinqh_layout& L = *layout;
+  return cuda_status(launch_pack(W, L.K, L.N, L.tile_n, L.n_tiles, L.meta_stride, L.n_groups, planes,
+                                 meta, (cudaStream_t)stream));
+}
+
+grinqh_status grinqh_unpack_codes(const grinqh_layout* layout, const void* planes, const uint8_t* bits,
+                                  uint8_t* codes, void* stream) {
+  if (!layout_ok(layout) || !planes || !codes) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(planes, 16)) return GRINQH_ERR_ALIGNMENT;
+  const grinqh_layout& L = *layout;
+  return cuda_status(launch_unpack(planes, bits, L.K, L.N, L.tile_n, L.n_tiles, codes, (cudaStream_t)stream));
+}
+
+grinqh_status grinqh_maxent_distribution(const uint8_t* classes, int32_t n_classes, double target_bits,
+                                         double* P) {
+  if (!valid_classes(classes, n_classes) || !P) return GRINQH_ERR_INVALID_ARG;
+  const double lo = classes[0], hi = classes[n_classes - 1];
+  if (!(target_bits >= lo && target_bits <= hi)) return GRINQH_ERR_INVALID_ARG;
+  for (int i = 0; i < n_classes; ++i) P[i] = 0.0;
+  if (target_bits == hi) { P[n_classes - 1] = 1.0; return GRINQH_OK; }
+  if (target_bits == lo) { P[0] = 1.0; return GRINQH_OK; }
+  double p[GRINQH_MAX_CLASSES];
+  // bracket lambda: mean(L) > target > mean(-L)
+  double Lb = 1.0;
+  for (int it = 0; it < 64; ++it) {
+    gibbs(classes, n_classes, Lb, p);
+    const double up = mean_width(classes, n_classes, p);
+    gibbs(classes, n_classes, -Lb, p);
+    const double dn = mean_width(classes, n_classes, p);
+    if (up > target_bits && dn < target_bits) break;
+    Lb *= 2.0;
+  }
+  double a = -Lb, c = Lb;
+  for (int it = 0; it < 200; ++it) {
+    const double mid = 0.5 * (a + c);
+    if (mid == a || mid == c) break;
+    gibbs(classes, n_classes, mid, p);
+    if (mean_width(classes, n_classes, p) < target_bits) a = mid; else c = mid;
+  }
+  gibbs(classes, n_classes, 0.5 * (a + c), P);
+  return GRINQH_OK;
+}
+
+grinqh_status grinqh_calibrate_workspace_bytes(int32_t S, int32_t n_classes, size_t* bytes) {
+  if (!bytes || S < 1 || S > 65535 || n_classes < 1 || n_classes > GRINQH_MAX_CLASSES)
+    return GRINQH_ERR_INVALID_ARG;
+  *bytes = calibrate_workspace_bytes(S, n_classes - 1);
+  return GRINQH_OK;
+}
+
+grinqh_status grinqh_calibrate(const uint16_t* X, int32_t S, int32_t K, const uint8_t* classes,
+                               int32_t n_classes, const double* P, double target_bits, float* thresholds,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
+  if (S < 1 || S > 65535 || K < 1 || K > kMaxDim) return GRINQH_ERR_INVALID_ARG;
+  const int n = n_classes - 1;
+  if (n > 0 && (!X || !thresholds)) return GRINQH_ERR_INVALID_ARG;
+  double Pv[GRINQH_MAX_CLASSES];
+  if (P) {
+    double tot = 0.0;
+    for (int i = 0; i < n_classes; ++i) {
+      if (!(P[i] >= 0.0)) return GRINQH_ERR_INVALID_ARG;
+      Pv[i] = P[i];
+      tot += P[i];
+    }
+    if (std::fabs(tot - 1.0) > 1e-9) return GRINQH_ERR_INVALID_ARG;
+  } else {
+    const grinqh_status st = grinqh_maxent_distribution(classes, n_classes, target_bits, Pv);
+    if (st != GRINQH_OK) return st;
+  }
+  if (n == 0) return GRINQH_OK;
+  if (!aligned(X, 2) || !aligned(thresholds, 4) || !aligned(workspace, 16)) return GRINQH_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < calibrate_workspace_bytes(S, n)) return GRINQH_ERR_WORKSPACE;
+
+  CalibArgs a{};
+  a.X = X;
+  a.S = S;
+  a.K = K;
+  a.n = n;
+  a.per_sample = (double*)workspace;
+  a.thresholds = thresholds;
+  double q = 0.0;
+  for (int j = 1; j <= n; ++j) {
+    q += Pv[j - 1];   // q_j = p_0 + ... + p_{j-1}, summed in ascending order
+    bool tail_empty = true;
+    for (int i = j; i < n_classes; ++i)
+      if (Pv[i] != 0.0) tail_empty = false;
+    const int jj = j - 1;
+    if (tail_empty) { a.mode[jj] = 2; continue; }
+    if (q == 0.0) { a.mode[jj] = 1; continue; }
+    a.mode[jj] = 0;
+    const double pos = q * (double)(K - 1);
+    if (pos >= (double)(K - 1)) {
+      a.lo[jj] = a.hi[jj] = K - 1;
+      a.frac[jj] = 0.0;
+    } else {
+      const double fl = std::floor(pos);
+      a.lo[jj] = (int)fl;
+      a.hi[jj] = (a.lo[jj] + 1 < K) ? a.lo[jj] + 1 : K - 1;
+      a.frac[jj] = pos - fl;
+    }
+  }
+  return cuda_status(launch_calibrate(a, (cudaStream_t)stream));
+}
+
+grinqh_status grinqh_select(const uint16_t* x, int32_t K, const float* thresholds, const uint8_t* classes,
+                            int32_t n_classes, uint8_t* bits, int32_t* idx, int32_t* offsets, void* stream) {
+  if (!valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
+  if (K < 1 || K > kMaxDim) return GRINQH_ERR_INVALID_ARG;
+  if (!x || !bits || !idx || !offsets || (n_classes > 1 && !thresholds)) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(x, 2) || !aligned(idx, 4) || !aligned(offsets, 4) || (thresholds && !aligned(thresholds, 4)))
+    return GRINQH_ERR_ALIGNMENT;
+  return cuda_status(launch_select(x, K, thresholds, table(classes, n_classes), bits, idx, offsets,
+                                   (cudaStream_t)stream));
+}
+
+grinqh_status grinqh_vmm_workspace_bytes(const grinqh_layout* layout, size_t* bytes) {
+  if (!layout_ok(layout) || !bytes) return GRINQH_ERR_INVALID_ARG;
+  *bytes = vmm_workspace_bytes(layout->n_tiles, layout->tile_n);
+  return GRINQH_OK;
+}
+
+grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* planes, const uint32_t* meta,
+                         const uint16_t* x, const int32_t* idx, const int32_t* offsets, const uint8_t* classes,
+                         int32_t n_classes, float* y, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!layout_ok(layout) || !valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
+  if (!planes || !meta || !x || !idx || !offsets || !y) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(planes, 16) || !aligned(meta, 16) || !aligned(x, 2) || !aligned(idx, 4) ||
+      !aligned(offsets, 4) || !aligned(y, 4))
+    return GRINQH_ERR_ALIGNMENT;
+  const grinqh_layout& L = *layout;
+  const size_t need = vmm_workspace_bytes(L.n_tiles, L.tile_n);
+  if (!workspace || workspace_bytes < need) return GRINQH_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return GRINQH_ERR_ALIGNMENT;
+  VmmArgs a{};
+  a.K = L.K;
+  a.N = L.N;
+  a.tile_n = L.tile_n;
+  a.n_tiles = L.n_tiles;
+  a.meta_stride = L.meta_stride;
+  a.planes = (const uint32_t*)planes;
+  a.meta = meta;
+  a.x = x;
+  a.idx = idx;
+  a.offsets = offsets;
+  a.y = y;
+  a.accum = (float*)workspace;
+  a.counters = (uint32_t*)((char*)workspace + (size_t)L.n_tiles * L.tile_n * sizeof(float));
+  a.ct = table(classes, n_classes);
+  return cuda_status(launch_vmm(a, (cudaStream_t)stream));
+}
+
+}  // extern "C"

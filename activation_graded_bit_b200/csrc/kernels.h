@@ -1,0 +1,53 @@
+// Internal launchers of the GRINQH kernels; called by the C ABI in api.cu after
+// it has validated every argument. Not part of the public interface.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace grinqh {
+
+cudaError_t launch_pack(const float* W, int K, int N, int tile_n, int n_tiles, int meta_stride,
+                        int n_groups, void* planes, uint32_t* meta, cudaStream_t st);
+
+cudaError_t launch_unpack(const void* planes, const uint8_t* bits, int K, int N, int tile_n,
+                          int n_tiles, uint8_t* codes, cudaStream_t st);
+
+struct ClassTable {
+  int n;              // number of classes (1..9)
+  uint8_t width[9];   // bit width of class j
+};
+
+cudaError_t launch_select(const uint16_t* x, int K, const float* thresholds, const ClassTable& ct,
+                          uint8_t* bits, int32_t* idx, int32_t* offsets, cudaStream_t st);
+
+struct VmmArgs {
+  int K, N, tile_n, n_tiles, meta_stride;
+  const uint32_t* planes;
+  const uint32_t* meta;
+  const uint16_t* x;
+  const int32_t* idx;
+  const int32_t* offsets;
+  float* y;
+  float* accum;         // workspace: n_tiles * tile_n floats, zero between calls
+  uint32_t* counters;   // workspace: n_tiles tickets, zero between calls
+  ClassTable ct;
+};
+
+size_t vmm_workspace_bytes(int n_tiles, int tile_n);
+cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st);
+
+// Calibration: per-sample order statistics, then the fixed-order mean.
+struct CalibArgs {
+  const uint16_t* X;
+  int S, K, n;          // n = number of thresholds
+  int lo[8], hi[8];     // ranks of the two order statistics around q_j (K-1)
+  double frac[8];       // interpolation weight
+  int mode[8];          // 0: interpolate, 1: theta = 0, 2: theta = +inf
+  double* per_sample;   // workspace [S][n]
+  float* thresholds;
+};
+size_t calibrate_workspace_bytes(int S, int n);
+cudaError_t launch_calibrate(const CalibArgs& a, cudaStream_t st);
+
+}  // namespace grinqh

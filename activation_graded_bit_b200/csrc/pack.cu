@@ -1,0 +1,153 @@
+// Offline packing: 8-bit RTN per (row, 128-column group) + MSB-first bit planes,
+// and the test-only decoder of the packed format.
+//
+// Paper: "GRINQH" Section 3.3 (uniform b_max-bit codes split into significance
+// slices, input-major storage), Section 4 (RTN with group size 128) and
+// Appendix C.1 (same-significance bits of neighbouring weights in one 32-bit
+// word, grouped offline so the kernel rebuilds codes with OR/SHIFT).
+#include <cstdint>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace grinqh {
+
+// fp64 -> binary16, round to nearest even, in one conversion (no fp32 detour).
+__device__ __forceinline__ uint16_t f64_to_f16_rn(double v) {
+  unsigned short h;
+  asm("cvt.rn.f16.f64 %0, %1;" : "=h"(h) : "d"(v));
+  return h;
+}
+
+__device__ __forceinline__ double f16_to_f64(uint16_t h) {
+  return (double)__half2float(__ushort_as_half(h));
+}
+
+// One CTA per (tile t, row k): 4 warps, warp g handles the tile's group g.
+// 128 threads then build the 8 x 16 plane words of the record.
+__global__ void __launch_bounds__(128) pack_kernel(const float* __restrict__ W, int K, int N,
+                                                   int tile_n, int meta_stride, int n_groups,
+                                                   uint32_t* __restrict__ planes,
+                                                   uint32_t* __restrict__ meta) {
+  __shared__ uint8_t codes[512];
+  const int k = blockIdx.x, t = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gl = t * (tile_n / kGroup) + warp;     // global group index
+  const int c0 = gl * kGroup;                      // first column of the group
+  const float* row = W + (size_t)k * N;
+
+  float v[4];
+  float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int n = c0 + lane + 32 * e;
+    v[e] = (n < N) ? row[n] : 0.0f;
+    if (n < N) { mn = fminf(mn, v[e]); mx = fmaxf(mx, v[e]); }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const bool live = gl < n_groups;
+  double s = 1.0, z = 0.0;
+  uint16_t sb = 0, zb = 0;
+  if (live) {
+    const double range = __dsub_rn((double)mx, (double)mn);
+    sb = f64_to_f16_rn(__ddiv_rn(range, 255.0));
+    s = f16_to_f64(sb);
+    if (s == 0.0) { sb = 0x3C00; s = 1.0; }
+    if (isinf(s)) { sb = 0x7BFF; s = 65504.0; }
+    z = rint(__ddiv_rn(-(double)mn, s));
+    z = __dadd_rn(fmin(fmax(z, 0.0), 255.0), 0.0);   // -0 -> +0
+    zb = f64_to_f16_rn(z);
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int n = c0 + lane + 32 * e;
+    uint8_t q = 0;
+    if (live && n < N) {
+      double qv = __dadd_rn(rint(__ddiv_rn((double)v[e], s)), z);
+      qv = fmin(fmax(qv, 0.0), 255.0);
+      q = (uint8_t)qv;
+    }
+    codes[warp * kGroup + lane + 32 * e] = q;
+  }
+  if (lane == 0) meta[(size_t)k * meta_stride + gl] = live ? ((uint32_t)sb | ((uint32_t)zb << 16)) : 0u;
+  __syncthreads();
+
+  // thread -> (plane p, word w): 8 planes x 16 words for a 512-column tile
+  const int p = threadIdx.x >> 4, w = threadIdx.x & 15;
+  uint32_t word = 0;
+#pragma unroll 8
+  for (int L = 0; L < 32; ++L) {
+    const int c = 32 * w + col_at(p, L);
+    word |= (uint32_t)((codes[c] >> (7 - p)) & 1u) << L;
+  }
+  uint32_t* rec = planes + ((size_t)t * K + k) * (tile_n / 4);
+  rec[p * (tile_n / 32) + w] = word;
+}
+
+// Decoder: 16 threads per (tile, row) record, 8 records per CTA.
+template <int B>
+__device__ __forceinline__ void decode_word(const uint32_t* plane_w, int stride_words, uint32_t (&R)[8]) {
+  uint32_t P[8];
+#pragma unroll
+  for (int p = 0; p < 8; ++p) P[p] = (p < B) ? plane_w[p * stride_words] : 0u;
+  assemble<B>(P, R);
+  const uint32_t mid = midpoint_bytes(B);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) R[j] |= mid;
+}
+
+__global__ void __launch_bounds__(128) unpack_kernel(const uint32_t* __restrict__ planes,
+                                                     const uint8_t* __restrict__ bits, int K, int N,
+                                                     int tile_n, uint8_t* __restrict__ codes) {
+  const int t = blockIdx.y;
+  const int k = blockIdx.x * 8 + (threadIdx.x >> 4);
+  const int w = threadIdx.x & 15;
+  if (k >= K) return;
+  const int b = bits ? bits[k] : 8;
+  const uint32_t* rec = planes + ((size_t)t * K + k) * (tile_n / 4) + w;
+  const int sw = tile_n / 32;
+  uint32_t R[8];
+  switch (b) {
+    case 1: decode_word<1>(rec, sw, R); break;
+    case 2: decode_word<2>(rec, sw, R); break;
+    case 3: decode_word<3>(rec, sw, R); break;
+    case 4: decode_word<4>(rec, sw, R); break;
+    case 5: decode_word<5>(rec, sw, R); break;
+    case 6: decode_word<6>(rec, sw, R); break;
+    case 7: decode_word<7>(rec, sw, R); break;
+    case 8: decode_word<8>(rec, sw, R); break;
+    default:
+#pragma unroll
+      for (int j = 0; j < 8; ++j) R[j] = 0u;
+  }
+  const int n0 = t * tile_n + 32 * w;
+  uint8_t* out = codes + (size_t)k * N;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int n = n0 + 4 * j + i;
+      if (n < N) out[n] = (uint8_t)(R[j] >> (8 * i));
+    }
+}
+
+cudaError_t launch_pack(const float* W, int K, int N, int tile_n, int n_tiles, int meta_stride,
+                        int n_groups, void* planes, uint32_t* meta, cudaStream_t st) {
+  dim3 grid(K, n_tiles);
+  pack_kernel<<<grid, 128, 0, st>>>(W, K, N, tile_n, meta_stride, n_groups, (uint32_t*)planes, meta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack(const void* planes, const uint8_t* bits, int K, int N, int tile_n,
+                          int n_tiles, uint8_t* codes, cudaStream_t st) {
+  dim3 grid((K + 7) / 8, n_tiles);
+  unpack_kernel<<<grid, 128, 0, st>>>((const uint32_t*)planes, bits, K, N, tile_n, codes);
+  return cudaGetLastError();
+}
+
+}  // namespace grinqh

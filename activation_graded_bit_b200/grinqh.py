@@ -1,0 +1,221 @@
+"""Thin ctypes binding over libgrinqh.so (the C ABI in include/grinqh.h).
+
+Argument marshalling only: every step of the graded VMM runs in the library's
+CUDA kernels. torch is used for device memory and streams: tensors are passed as
+raw device pointers and the current torch stream as the cudaStream_t. There is
+no fallback: if the shared library is missing, importing this module fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgrinqh.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "libgrinqh.so is not built (expected at %s); run `python -m activation_graded_bit_b200.build` "
+        "or __graft_entry__.build()" % LIB_PATH)
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK = 0
+STATUS = {0: "ok", 1: "invalid argument", 2: "misaligned pointer", 3: "unsupported",
+          4: "workspace missing or too small", 5: "CUDA error"}
+
+
+class GrinqhError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__("%s failed: %s (%d)" % (where, STATUS.get(code, "?"), code))
+        self.code = code
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [("K", ctypes.c_int32), ("N", ctypes.c_int32), ("n_groups", ctypes.c_int32),
+                ("tile_n", ctypes.c_int32), ("n_tiles", ctypes.c_int32), ("meta_stride", ctypes.c_int32),
+                ("planes_bytes", ctypes.c_int64), ("meta_bytes", ctypes.c_int64)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_LP = ctypes.POINTER(Layout)
+
+
+def _sig(name, args, res=ctypes.c_int):
+    f = getattr(_lib, name)
+    f.argtypes = args
+    f.restype = res
+    return f
+
+
+_version = _sig("grinqh_version", [], ctypes.c_char_p)
+_status_string = _sig("grinqh_status_string", [ctypes.c_int], ctypes.c_char_p)
+_layout_init = _sig("grinqh_layout_init", [_I, _I, _LP])
+_pack = _sig("grinqh_pack", [_LP, _P, _P, _P, _P])
+_unpack = _sig("grinqh_unpack_codes", [_LP, _P, _P, _P, _P])
+_maxent = _sig("grinqh_maxent_distribution", [_P, _I, ctypes.c_double, _P])
+_cal_ws = _sig("grinqh_calibrate_workspace_bytes", [_I, _I, ctypes.POINTER(ctypes.c_size_t)])
+_calibrate = _sig("grinqh_calibrate", [_P, _I, _I, _P, _I, _P, ctypes.c_double, _P, _P, ctypes.c_size_t, _P])
+_select = _sig("grinqh_select", [_P, _I, _P, _P, _I, _P, _P, _P, _P])
+_vmm_ws = _sig("grinqh_vmm_workspace_bytes", [_LP, ctypes.POINTER(ctypes.c_size_t)])
+_vmm = _sig("grinqh_vmm", [_LP, _P, _P, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
+
+# Every exported symbol of the C ABI, for the export check in the tests.
+EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grinqh_pack",
+           "grinqh_unpack_codes", "grinqh_maxent_distribution", "grinqh_calibrate_workspace_bytes",
+           "grinqh_calibrate", "grinqh_select", "grinqh_vmm_workspace_bytes", "grinqh_vmm")
+
+
+def version() -> str:
+    return _version().decode()
+
+
+def _check(rc: int, where: str):
+    if rc != OK:
+        raise GrinqhError(rc, where)
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _classes_buf(classes: Sequence[int]):
+    arr = (ctypes.c_uint8 * len(classes))(*[int(c) for c in classes])
+    return arr, len(classes)
+
+
+def layout(K: int, N: int) -> Layout:
+    L = Layout()
+    _check(_layout_init(int(K), int(N), ctypes.byref(L)), "grinqh_layout_init")
+    return L
+
+
+@dataclass
+class PackedLayer:
+    """Bit-plane packed K x N layer: planes (uint8 bytes) and meta (int32 words)."""
+    layout: Layout
+    planes: torch.Tensor
+    meta: torch.Tensor
+
+    @property
+    def K(self):
+        return self.layout.K
+
+    @property
+    def N(self):
+        return self.layout.N
+
+
+def empty_packed(K: int, N: int, device="cuda") -> PackedLayer:
+    L = layout(K, N)
+    planes = torch.empty(int(L.planes_bytes), dtype=torch.uint8, device=device)
+    meta = torch.empty(int(L.meta_bytes) // 4, dtype=torch.int32, device=device)
+    return PackedLayer(L, planes, meta)
+
+
+def pack(W: torch.Tensor, out: Optional[PackedLayer] = None, stream=None) -> PackedLayer:
+    """grinqh_pack: W is a contiguous fp32 [K, N] CUDA tensor."""
+    assert W.dtype == torch.float32 and W.is_cuda and W.is_contiguous() and W.dim() == 2
+    K, N = W.shape
+    p = out if out is not None else empty_packed(K, N, W.device)
+    _check(_pack(ctypes.byref(p.layout), _ptr(W), _ptr(p.planes), _ptr(p.meta), _stream(stream)), "grinqh_pack")
+    return p
+
+
+def unpack_codes(p: PackedLayer, bits: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    codes = torch.empty((p.K, p.N), dtype=torch.uint8, device=p.planes.device)
+    _check(_unpack(ctypes.byref(p.layout), _ptr(p.planes), _ptr(bits), _ptr(codes), _stream(stream)),
+           "grinqh_unpack_codes")
+    return codes
+
+
+def maxent_distribution(classes: Sequence[int], target_bits: float):
+    cb, n = _classes_buf(classes)
+    P = (ctypes.c_double * n)()
+    _check(_maxent(ctypes.addressof(cb), n, float(target_bits), ctypes.addressof(P)), "grinqh_maxent_distribution")
+    return [P[i] for i in range(n)]
+
+
+def calibrate_workspace_bytes(S: int, n_classes: int) -> int:
+    v = ctypes.c_size_t()
+    _check(_cal_ws(int(S), int(n_classes), ctypes.byref(v)), "grinqh_calibrate_workspace_bytes")
+    return v.value
+
+
+def calibrate(X: torch.Tensor, classes: Sequence[int], P: Optional[Sequence[float]] = None,
+              target_bits: float = 0.0, out: Optional[torch.Tensor] = None,
+              workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """grinqh_calibrate: X is a [S, K] CUDA tensor of fp16 (or its int16/uint16 bit view)."""
+    assert X.is_cuda and X.dim() == 2 and X.is_contiguous() and X.element_size() == 2
+    S, K = X.shape
+    cb, n = _classes_buf(classes)
+    th = out if out is not None else torch.empty(max(n - 1, 1), dtype=torch.float32, device=X.device)
+    ws_bytes = calibrate_workspace_bytes(S, n)
+    ws = workspace if workspace is not None else torch.empty(ws_bytes, dtype=torch.uint8, device=X.device)
+    Pbuf = None
+    if P is not None:
+        Pbuf = (ctypes.c_double * n)(*[float(v) for v in P])
+    _check(_calibrate(_ptr(X), S, K, ctypes.addressof(cb), n,
+                      ctypes.addressof(Pbuf) if Pbuf is not None else None, float(target_bits),
+                      _ptr(th), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "grinqh_calibrate")
+    return th[: n - 1]
+
+
+@dataclass
+class Selection:
+    bits: torch.Tensor      # uint8 [K]
+    idx: torch.Tensor       # int32 [K]
+    offsets: torch.Tensor   # int32 [n_classes + 1]
+    classes: tuple
+
+
+def empty_selection(K: int, classes: Sequence[int], device="cuda") -> Selection:
+    return Selection(torch.empty(K, dtype=torch.uint8, device=device),
+                     torch.empty(K, dtype=torch.int32, device=device),
+                     torch.empty(len(classes) + 1, dtype=torch.int32, device=device), tuple(classes))
+
+
+def select(x: torch.Tensor, thresholds: torch.Tensor, classes: Sequence[int],
+           out: Optional[Selection] = None, stream=None) -> Selection:
+    """grinqh_select: x is a [K] CUDA tensor of fp16 (or its 16-bit bit view)."""
+    assert x.is_cuda and x.dim() == 1 and x.is_contiguous() and x.element_size() == 2
+    K = x.shape[0]
+    sel = out if out is not None else empty_selection(K, classes, x.device)
+    cb, n = _classes_buf(classes)
+    _check(_select(_ptr(x), K, _ptr(thresholds), ctypes.addressof(cb), n, _ptr(sel.bits), _ptr(sel.idx),
+                   _ptr(sel.offsets), _stream(stream)), "grinqh_select")
+    return sel
+
+
+def vmm_workspace_bytes(L: Layout) -> int:
+    v = ctypes.c_size_t()
+    _check(_vmm_ws(ctypes.byref(L), ctypes.byref(v)), "grinqh_vmm_workspace_bytes")
+    return v.value
+
+
+def vmm_workspace(L: Layout, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace for grinqh_vmm (reusable across calls on one stream)."""
+    return torch.zeros(vmm_workspace_bytes(L), dtype=torch.uint8, device=device)
+
+
+def vmm(p: PackedLayer, x: torch.Tensor, sel: Selection, workspace: torch.Tensor,
+        y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """grinqh_vmm: y[N] fp32 = x . W_hat over the graded bit planes."""
+    if y is None:
+        y = torch.empty(p.N, dtype=torch.float32, device=p.planes.device)
+    cb, n = _classes_buf(sel.classes)
+    _check(_vmm(ctypes.byref(p.layout), _ptr(p.planes), _ptr(p.meta), _ptr(x), _ptr(sel.idx), _ptr(sel.offsets),
+                ctypes.addressof(cb), n, _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                _stream(stream)), "grinqh_vmm")
+    return y

@@ -1,0 +1,394 @@
+"""Benchmark of the graded bit-plane VMM (GRINQH decode hot path) on B200.
+
+Workload (default): the seven decode linears of a Llama3-8B-shaped layer
+(q/o 4096x4096, k/v 4096x1024, gate/up 4096x14336, down 14336x4096), batch 1,
+weights ~N(0, 0.02) RTN-8 packed as bit planes, fp16 activations ~N(0,1) with a
+fixed 1% of channels scaled x20, thresholds calibrated (128 vectors, classes
+{0,2,3,4,8}, maximum-entropy P) for average widths 4, 3 and 2 bits.
+
+One step = grinqh_select + grinqh_vmm for each of the 7 linears at each of the 3
+widths (21 pairs), every pair on its own packed copy of its layer (6 copies of
+the layer in HBM, ~1.3 GB, far above the 126 MB L2), replayed from a CUDA graph.
+value = microseconds per select+VMM pair (lower is better).
+
+The roofline entry is for grinqh_vmm alone, timed by a graph of the 21 VMMs with
+CUDA events on the launching stream; achieved GB/s counts the algorithmic bytes
+of each call: planes sum_k b_k N/8, scale/zero 4 bytes per (active row, 128
+columns), x (2K), the channel list (4 per active row) and y (4N).
+
+`--impl reference` times the fp64 CPU oracle (the only reference there is) on a
+bounded sample of the same workload on the host cores.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "µs per batch-1 VMM and effective HBM GB/s (% of peak) vs average bits"
+UNIT = "µs"
+TARGETS = (4.0, 3.0, 2.0)
+WORKLOAD = "llama3-8b decode linears (q,k,v,o,gate,up,down), batch 1, avg bits 4/3/2"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                v = [t.strip() for t in line.split(",")]
+                if len(v) >= 9:
+                    rows.append(v)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def build_workload(g, wl, torch, dev, copies=2):
+    """Pack `copies` x 3 (one per width) copies of the 7 linears, calibrate per
+    linear and width, and draw one input vector per pair."""
+    classes = wl.CLASSES
+    pairs = []
+    gen = torch.Generator(device=dev)
+    for li, (name, K, N) in enumerate(wl.LLAMA3_8B):
+        Xc = wl.activations_outlier(K, 128, key=(1, 0, li, 1), chan_key=(1, 0, li))
+        Xc_d = torch.from_numpy(Xc.view(np.int16)).to(dev)
+        th = {}
+        for t in TARGETS:
+            th[t] = g.calibrate(Xc_d, classes, P=None, target_bits=t)
+        for c in range(copies):
+            for ti, t in enumerate(TARGETS):
+                gen.manual_seed(1_000_003 * (li + 1) + 7919 * c + 31 * ti)
+                W = torch.randn(K, N, generator=gen, device=dev, dtype=torch.float32) * 0.02
+                p = g.pack(W)
+                del W
+                x = wl.activations_outlier(K, 1, key=(1, c, li, 2 + ti), chan_key=(1, 0, li))[0]
+                x_d = torch.from_numpy(x.view(np.int16)).to(dev)
+                sel = g.select(x_d, th[t], classes)
+                pairs.append(dict(name=name, K=K, N=N, target=t, copy=c, packed=p, x=x_d, x_host=x,
+                                  th=th[t], sel=sel, ws=g.vmm_workspace(p.layout, dev),
+                                  y=torch.empty(N, dtype=torch.float32, device=dev)))
+    torch.cuda.synchronize()
+    return pairs
+
+
+def algorithmic_bytes(pair):
+    bits = pair["sel"].bits.cpu().numpy().astype(np.int64)
+    K, N = pair["K"], pair["N"]
+    active = int((bits > 0).sum())
+    ng = (N + 127) // 128
+    planes = int(bits.sum()) * N / 8.0
+    meta = 4.0 * ng * active
+    total = planes + meta + 2.0 * K + 4.0 * active + 4.0 * N
+    return planes, total, float(bits.mean()), active / K
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    from activation_graded_bit_b200 import grinqh as g
+    from activation_graded_bit_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    pairs = build_workload(g, wl, torch, dev, copies=args.copies)
+    groups = {}
+    for pr in pairs:
+        groups.setdefault(pr["copy"], []).append(pr)
+    copies = sorted(groups)
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step_pairs(c):
+        for pr in groups[c]:
+            g.select(pr["x"], pr["th"], wl.CLASSES, out=pr["sel"], stream=stream)
+            g.vmm(pr["packed"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
+
+    def vmm_only(c):
+        for pr in groups[c]:
+            g.vmm(pr["packed"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
+
+    # e2e: pinned host x in, host y out, per pair
+    for pr in pairs:
+        pr["x_pin"] = torch.from_numpy(pr["x_host"].view(np.int16).copy()).pin_memory()
+        pr["y_pin"] = torch.empty(pr["N"], dtype=torch.float32).pin_memory()
+
+    def e2e_pairs(c):
+        for pr in groups[c]:
+            pr["x"].copy_(pr["x_pin"], non_blocking=True)
+            g.select(pr["x"], pr["th"], wl.CLASSES, out=pr["sel"], stream=stream)
+            g.vmm(pr["packed"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
+            pr["y_pin"].copy_(pr["y"], non_blocking=True)
+
+    def capture(fn):
+        graphs = {}
+        with torch.cuda.stream(stream):
+            for c in copies:
+                fn(c)  # eager warm-up outside capture
+            torch.cuda.synchronize()
+            for c in copies:
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=stream):
+                    fn(c)
+                graphs[c] = gr
+        torch.cuda.synchronize()
+        return graphs
+
+    g_step = capture(step_pairs)
+    g_vmm = capture(vmm_only)
+    g_e2e = capture(e2e_pairs)
+
+    def timed(graphs, steps, warmup):
+        with torch.cuda.stream(stream):
+            for i in range(warmup):
+                graphs[copies[i % len(copies)]].replay()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(steps):
+                graphs[copies[i % len(copies)]].replay()
+            e1.record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+            dist.barrier()
+        return ms
+
+    n_pairs = len(groups[copies[0]])
+    with ClockSampler(local) as clk:
+        ms_step = timed(g_step, args.steps, args.warmup)
+    clocks = clk.summary()
+    ms_vmm = timed(g_vmm, args.steps, args.warmup)
+    ms_e2e = timed(g_e2e, args.steps, args.warmup)
+
+    # correctness spot check of the timed path (one pair) before reporting
+    torch.cuda.synchronize()
+    y0 = pairs[0]["y"]
+    assert bool(torch.isfinite(y0).all()), "non-finite y"
+
+    points = []
+    tot_alg = 0.0
+    tot_planes = 0.0
+    for pr in groups[copies[0]]:
+        planes, total, mean_bits, active = algorithmic_bytes(pr)
+        tot_alg += total
+        tot_planes += planes
+        points.append(dict(linear=pr["name"], K=pr["K"], N=pr["N"], target_bits=pr["target"],
+                           mean_bits=round(mean_bits, 4), active_frac=round(active, 4),
+                           planes_bytes=int(planes), alg_bytes=int(total)))
+    peak, peak_kind = _peaks()
+    us_pair = ms_step * 1e3 / (args.steps * n_pairs)
+    us_vmm = ms_vmm * 1e3 / (args.steps * n_pairs)
+    achieved = tot_alg * args.steps / (ms_vmm * 1e-3) / 1e9
+    value = ms_step * 1e3 / (args.steps * n_pairs * world)
+    e2e_us = ms_e2e * 1e3 / (args.steps * n_pairs * world)
+    h2d = sum(2 * pr["K"] for pr in groups[copies[0]])
+    d2h = sum(4 * pr["N"] for pr in groups[copies[0]])
+
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "vmm_traffic.json")
+    if os.path.exists(tpath):
+        try:
+            traffic = json.load(open(tpath)).get("bytes_per_launch_scaled")
+        except Exception:
+            traffic = None
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(args)
+        out = {
+            "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step / args.steps, 6), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u8 planes, fp32 accumulate", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "pairs_per_step": n_pairs, "classes": list(wl.CLASSES),
+                       "l2": "inputs larger than L2: every pair of a step reads its own packed copy; "
+                             "%d copies of the layer set (%.2f GB) rotate" % (
+                                 len(pairs), sum(pr["packed"].planes.numel() for pr in pairs) / 1e9),
+                       "parallelism": "replicas only" if world > 1 else "single GPU"},
+            "vmm_us": round(us_vmm, 4), "select_plus_vmm_us": round(us_pair, 4),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
+                         "kernel": "grinqh vmm_kernel"},
+            "points": points,
+            "e2e": {"value": round(e2e_us, 4), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 2 * n_pairs * args.steps,
+            "clocks": clocks,
+        }
+        if cpu is not None:
+            out["cpu_baseline"] = cpu
+        print(json.dumps(out))
+    # release graphs before tearing down the process group
+    del g_step, g_vmm, g_e2e
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (host cores)
+# ---------------------------------------------------------------------------
+def _oracle_sample(budget_s, nthreads):
+    """Time oracle select + vmm on a bounded sample of the workload's pairs."""
+    import oracle
+    from activation_graded_bit_b200 import workloads as wl
+    classes = np.array(wl.CLASSES, np.uint8)
+    done = 0
+    secs = 0.0
+    names = []
+    t_start = time.time()
+    for li, (name, K, N) in enumerate(wl.LLAMA3_8B):
+        if time.time() - t_start > budget_s:
+            break
+        # untimed setup: weights, RTN codes, thresholds of this linear
+        W = wl.weights_gaussian(K, N, key=(1, 9, li, 0))
+        q, s, z = oracle.rtn_quantize(W)
+        del W
+        Xc = wl.activations_outlier(K, 32, key=(1, 0, li, 1), chan_key=(1, 0, li))
+        for ti, t in enumerate(TARGETS):
+            th = oracle.thresholds(Xc, oracle.maxent_distribution(classes, t))
+            x = wl.activations_outlier(K, 1, key=(1, 0, li, 2 + ti), chan_key=(1, 0, li))[0]
+            t0 = time.perf_counter()
+            bits, idx, off = oracle.select(x, th, classes)
+            oracle.vmm(x, q, s, z, bits, nthreads=nthreads)
+            secs += time.perf_counter() - t0
+            done += 1
+            names.append("%s@%g" % (name, t))
+            if time.time() - t_start > budget_s:
+                break
+    return done, secs, names
+
+
+def cpu_baseline(args):
+    nthreads = os.cpu_count() or 1
+    done, secs, names = _oracle_sample(args.cpu_budget, nthreads)
+    return {"value": round(secs * 1e6 / max(done, 1), 1), "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": "fp64 oracle select+vmm on %d of the 21 (linear, width) pairs: %s" % (done, ", ".join(names))}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    nthreads = os.cpu_count() or 1
+    per = []
+    total_done = 0
+    for i in range(args.warmup + args.steps):
+        done, secs, names = _oracle_sample(args.cpu_budget / max(args.steps + args.warmup, 1), nthreads)
+        if i >= args.warmup:
+            per.append(secs / max(done, 1))
+            total_done += done
+    v = statistics.mean(per) * 1e6
+    out = {"impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": 0,
+           "steps": args.steps, "warmup": args.warmup, "higher_is_better": False, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": WORKLOAD, "parallelism": "host cores"},
+           "cpu_baseline": {"value": round(v, 1), "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                            "sample": "fp64 oracle select+vmm, %d pairs over %d steps" % (total_done, args.steps)},
+           "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--copies", type=int, default=2)
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,221 @@
+/*
+ * grinqh.h - C ABI of the GRINQH graded bit-plane VMM library (sm_100a).
+ *
+ * GRINQH ("GRINQH: Graded Input-based Quantization Hierarchy for Efficient LLM
+ * Generation", arXiv 2606.23419) speeds up batch-1 decoding by reading, for each
+ * input channel k of a linear layer, only the b_k most significant bits of that
+ * channel's 8-bit weights, where b_k is chosen per token from |x_k| against
+ * calibrated thresholds (Section 3.1), and b_k = 0 skips the channel entirely.
+ * The weights are stored once, as MSB-first bit planes, so every narrower width
+ * is a prefix of the wider one (Section 3.3, "Storage Layout and Weight
+ * Loading").
+ *
+ * Calls, in the order a user makes them:
+ *   grinqh_layout_init       sizes of the packed buffers for a K x N layer
+ *   grinqh_pack              offline 8-bit RTN + bit-plane packing
+ *   grinqh_maxent_distribution / grinqh_calibrate   thresholds for a target width
+ *   grinqh_select            per-token grading + per-class channel lists
+ *   grinqh_vmm               y = x . W_hat over the graded bit planes
+ *
+ * Conventions for every call:
+ *   - W is K x N: K input channels (rows), N output channels (columns).
+ *   - fp16 values are IEEE binary16 bit patterns passed as uint16_t.
+ *   - "device" pointers are CUDA global-memory addresses of the current device;
+ *     "host" pointers are ordinary CPU memory. The caller allocates and owns
+ *     every buffer; the library never allocates, frees or synchronises.
+ *   - stream is a cudaStream_t passed as void*; NULL means the legacy default
+ *     stream. Every device call is asynchronous on that stream.
+ *   - Arguments are checked on the host before anything is launched; a failed
+ *     check returns an error code and launches nothing. A CUDA launch error is
+ *     returned as GRINQH_ERR_CUDA. Nothing traps on the device.
+ *   - Sizes: 1 <= K, N <= 2^24, K * N <= 2^34. Classes: 1..9 bit widths, strictly
+ *     increasing, each in 0..8.
+ */
+#ifndef GRINQH_H_
+#define GRINQH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GRINQH_GROUP 128       /* columns per (row, group) scale/zero pair */
+#define GRINQH_MAX_CLASSES 9   /* widths 0..8 */
+#define GRINQH_PLANES 8        /* b_max = 8 */
+
+typedef enum {
+  GRINQH_OK = 0,
+  GRINQH_ERR_INVALID_ARG = 1,   /* a size, a pointer or a class set is invalid */
+  GRINQH_ERR_ALIGNMENT = 2,     /* a pointer is not aligned as documented */
+  GRINQH_ERR_UNSUPPORTED = 3,   /* valid, but outside what this build handles */
+  GRINQH_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+  GRINQH_ERR_CUDA = 5           /* a CUDA runtime call failed */
+} grinqh_status;
+
+/*
+ * Physical layout of a packed K x N layer. Filled by grinqh_layout_init; treat
+ * as read-only. Two buffers hold the layer:
+ *
+ *  planes  (device, planes_bytes, 16-byte aligned): n_tiles column tiles of
+ *          tile_n columns. Tile t, row k is one record of tile_n bytes at byte
+ *          offset (t*K + k)*tile_n, holding the 8 planes MSB first: plane p
+ *          (p = 0 is bit 7 of the code, p = 7 is bit 0) fills bytes
+ *          [p*tile_n/8, (p+1)*tile_n/8) of the record, so the top b planes of a
+ *          row are one contiguous run of b*tile_n/8 bytes. Inside a plane, 32-bit
+ *          word w holds local columns 32w..32w+31; local column 32w + 4j + i
+ *          (j in 0..7, i in 0..3) sits at bit (8i + j + 7 - p) mod 32 of the
+ *          word. Columns >= N are zero bits.
+ *  meta    (device, meta_bytes, 16-byte aligned): uint32 [K][meta_stride];
+ *          entry g of row k is scale_fp16 | (zero_fp16 << 16) for columns
+ *          [128g, 128g+128). Entries g >= n_groups are zero.
+ */
+typedef struct {
+  int32_t K;             /* input channels (rows) */
+  int32_t N;             /* output channels (columns) */
+  int32_t n_groups;      /* ceil(N / 128) */
+  int32_t tile_n;        /* columns per tile (multiple of 128) */
+  int32_t n_tiles;       /* ceil(N / tile_n) */
+  int32_t meta_stride;   /* uint32 entries per row of meta = n_tiles*tile_n/128 */
+  int64_t planes_bytes;  /* n_tiles * K * tile_n */
+  int64_t meta_bytes;    /* 4 * K * meta_stride */
+} grinqh_layout;
+
+/* Library version string (static storage). */
+const char* grinqh_version(void);
+
+/* Human-readable name of a status code (static storage). */
+const char* grinqh_status_string(grinqh_status s);
+
+/*
+ * Fill *out with the packed layout of a K x N layer. Host only.
+ * Errors: INVALID_ARG for out == NULL or sizes outside the limits above.
+ */
+grinqh_status grinqh_layout_init(int32_t K, int32_t N, grinqh_layout* out);
+
+/*
+ * Offline 8-bit RTN quantisation and bit-plane packing.
+ * Paper: Section 3.3 (uniform b_max-bit quantisation, nested slices, input-major
+ * storage), Section 4 (RTN, group size G = 128), Appendix C.1 (same-significance
+ * bits of neighbouring weights packed into 32-bit words).
+ * Per (row k, group g): s = fp16_rne((max - min) / 255) computed in fp64 and
+ * rounded straight to fp16 (s := 1 if it rounds to 0, s := 65504 if it
+ * overflows); z = clamp(rne(-min / s), 0, 255); q = clamp(rne(w / s) + z, 0, 255),
+ * quotients in fp64, ties to even.
+ *   W       device, fp32 [K][N] row-major, finite values (non-finite input
+ *           gives unspecified codes), 4-byte aligned.
+ *   planes  device, layout->planes_bytes, 16-byte aligned; fully overwritten.
+ *   meta    device, layout->meta_bytes, 16-byte aligned; fully overwritten.
+ * Errors: INVALID_ARG (NULL pointers, layout inconsistent), ALIGNMENT, CUDA.
+ */
+grinqh_status grinqh_pack(const grinqh_layout* layout, const float* W, void* planes,
+                          uint32_t* meta, void* stream);
+
+/*
+ * Decode the codes the VMM uses, for testing the packed format. For each row k
+ * with width b = bits[k] (8 for every row when bits == NULL):
+ *   b = 0: code 0 (the row is never read by grinqh_vmm);
+ *   1 <= b <= 7: c_b * 2^(8-b) + 2^(7-b), c_b = top b bits of q (Section 3.3
+ *     reconstruction with its midpoint term);
+ *   b = 8: q.
+ *   planes  device, as written by grinqh_pack for the same layout.
+ *   bits    device uint8 [K] of widths 0..8, or NULL.
+ *   codes   device uint8 [K][N] row-major; fully overwritten.
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ */
+grinqh_status grinqh_unpack_codes(const grinqh_layout* layout, const void* planes,
+                                  const uint8_t* bits, uint8_t* codes, void* stream);
+
+/*
+ * Maximum-entropy precision distribution P over a class set for a requested
+ * mean width target_bits (host only, no CUDA). Paper: Appendix A.1 eq. (1)
+ * constrains P to the simplex with sum_i p_i b_i = b*; the objective there is a
+ * model-quality metric, which needs trained models. This library takes the
+ * distribution of maximum entropy, p_i proportional to exp(lambda * b_i), with
+ * lambda found by fp64 bisection. target_bits equal to the smallest or largest
+ * class gives the one-hot distribution of that class.
+ *   classes  host uint8 [n_classes], strictly increasing widths in 0..8.
+ *   P        host double [n_classes], output.
+ * Errors: INVALID_ARG (bad class set, target outside [classes[0],
+ * classes[n_classes-1]], NULL pointers).
+ */
+grinqh_status grinqh_maxent_distribution(const uint8_t* classes, int32_t n_classes,
+                                         double target_bits, double* P);
+
+/* Workspace bytes grinqh_calibrate needs for S samples and n_classes classes. */
+grinqh_status grinqh_calibrate_workspace_bytes(int32_t S, int32_t n_classes, size_t* bytes);
+
+/*
+ * Threshold calibration by percentile mapping. Paper: Section 3.2 and Appendix
+ * A.1 eq. (2): for every calibration sample, theta_j is the
+ * (p_0 + ... + p_{j-1})-quantile of |x|; the per-sample values are averaged.
+ * Readings used here: n_classes - 1 thresholds; quantile = linear interpolation
+ * at position q_j*(K-1) of the ascending magnitudes (fp64); mean over samples
+ * summed in ascending sample order in fp64, then rounded to fp32; theta_j = 0
+ * when q_j == 0 exactly; theta_j = +inf when p_j..p_n are all zero.
+ *   X           device, fp16 [S][K] calibration vectors, finite, 2-byte aligned.
+ *   classes     host uint8 [n_classes].
+ *   P           host double [n_classes] (each >= 0, sum 1 within 1e-9), or NULL
+ *               to use grinqh_maxent_distribution(classes, target_bits).
+ *   thresholds  device fp32 [n_classes - 1], output, 4-byte aligned.
+ *   workspace   device, >= grinqh_calibrate_workspace_bytes, 16-byte aligned.
+ * Limits: 1 <= S <= 65535, 1 <= K <= 2^24.
+ * Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, CUDA.
+ */
+grinqh_status grinqh_calibrate(const uint16_t* X, int32_t S, int32_t K, const uint8_t* classes,
+                               int32_t n_classes, const double* P, double target_bits,
+                               float* thresholds, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/*
+ * Per-token grading and stable per-class compaction.
+ * Paper: Section 3.1: channel k gets class j = #{ i : |x_k| >= theta_i } (the
+ * interval rule [theta_j, theta_{j+1}) with theta_0 = 0, theta_{n+1} = inf,
+ * written as a count so that ties go to the upper class); NaN goes to class 0.
+ *   x          device fp16 [K].
+ *   thresholds device fp32 [n_classes - 1].
+ *   classes    host uint8 [n_classes].
+ *   bits       device uint8 [K], output: classes[j_k].
+ *   idx        device int32 [K], output: channel indices, class-major, ascending
+ *              k inside each class.
+ *   offsets    device int32 [n_classes + 1], output: offsets[j] = first position
+ *              of class j in idx, offsets[n_classes] = K.
+ * All device pointers 4-byte aligned except x (2) and bits (1).
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ */
+grinqh_status grinqh_select(const uint16_t* x, int32_t K, const float* thresholds,
+                            const uint8_t* classes, int32_t n_classes, uint8_t* bits,
+                            int32_t* idx, int32_t* offsets, void* stream);
+
+/* Workspace bytes grinqh_vmm needs for a layout. */
+grinqh_status grinqh_vmm_workspace_bytes(const grinqh_layout* layout, size_t* bytes);
+
+/*
+ * The graded vector-matrix product (the decode hot path).
+ * Paper: Fig. 2 and Section 3.3: for every channel k with b_k > 0, only planes
+ * 0..b_k-1 of row k (and its scale/zero pairs) are read; the row is rebuilt as
+ * w_hat = s * (code - z) with code = c_b * 2^(8-b) + 2^(7-b) for b < 8 and q for
+ * b = 8; channels with b_k = 0 are never read and add nothing.
+ *   y[n] = sum_k x_k * w_hat[k][n], accumulated in fp32 (order unspecified).
+ *   planes, meta  device, from grinqh_pack with this layout.
+ *   x             device fp16 [K] (the same vector grinqh_select graded).
+ *   idx, offsets  device, from grinqh_select with the same classes.
+ *   classes       host uint8 [n_classes].
+ *   y             device fp32 [N], output (overwritten), 4-byte aligned.
+ *   workspace     device, >= grinqh_vmm_workspace_bytes(layout), 16-byte
+ *                 aligned. It must be zero-filled once before its first use;
+ *                 every call leaves it zero-filled again. Calls that share one
+ *                 workspace must not overlap in time (use one stream).
+ * Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, CUDA.
+ */
+grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* planes, const uint32_t* meta,
+                         const uint16_t* x, const int32_t* idx, const int32_t* offsets,
+                         const uint8_t* classes, int32_t n_classes, float* y, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GRINQH_H_ */

@@ -1,0 +1,119 @@
+"""The C ABI library loads, exports every call include/grinqh.h declares, and
+rejects bad arguments on the host before anything reaches a GPU. No test here
+passes a pointer that could be launched on: every call fails validation first."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HDR = os.path.join(ROOT, "include", "grinqh.h")
+
+
+@pytest.fixture(scope="module")
+def g():
+    from activation_graded_bit_b200 import build
+    build.build()
+    from activation_graded_bit_b200 import grinqh
+    return grinqh
+
+
+def _declared():
+    txt = open(HDR).read()
+    return sorted(set(re.findall(r"\b(grinqh_[a-z_]+)\s*\(", txt)))
+
+
+def test_every_declared_symbol_is_exported(g):
+    names = _declared()
+    assert len(names) >= 11
+    lib = ctypes.CDLL(g.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(g.EXPORTS) == names
+
+
+def test_version_and_status_strings(g):
+    assert "sm_100a" in g.version()
+    for c in range(6):
+        assert g._status_string(c).decode() == g.STATUS[c]
+
+
+def test_layout(g):
+    L = g.layout(4096, 14336)
+    assert (L.K, L.N, L.n_groups, L.tile_n, L.n_tiles) == (4096, 14336, 112, 512, 28)
+    assert L.meta_stride == 28 * 4
+    assert L.planes_bytes == 28 * 4096 * 512 and L.meta_bytes == 4 * 4096 * 112
+    L = g.layout(4, 4)
+    assert (L.n_groups, L.n_tiles, L.meta_stride) == (1, 1, 4)
+    for K, N in ((0, 4), (4, 0), (-1, 5), (1 << 24 + 1, 1), (1 << 24, 1 << 24)):
+        with pytest.raises(g.GrinqhError) as e:
+            g.layout(K, N)
+        assert e.value.code == 1
+
+
+def test_maxent_matches_oracle(g, orc):
+    for classes in ((0, 2, 3, 4, 8), (0, 2, 4, 6, 8), (1, 8), (3,)):
+        lo, hi = classes[0], classes[-1]
+        for t in np.linspace(lo, hi, 7):
+            got = np.array(g.maxent_distribution(classes, t))
+            ref = orc.maxent_distribution(np.array(classes, np.uint8), t)
+            assert np.allclose(got, ref, rtol=0, atol=1e-12)
+    with pytest.raises(g.GrinqhError):
+        g.maxent_distribution((0, 2, 3, 4, 8), 8.5)
+    with pytest.raises(g.GrinqhError):
+        g.maxent_distribution((0, 3, 2), 2.0)
+    with pytest.raises(g.GrinqhError):
+        g.maxent_distribution((0, 2, 9), 2.0)
+
+
+def _L(g, K, N):
+    return ctypes.byref(g.layout(K, N))
+
+
+def test_host_validation_rejects_before_launch(g):
+    P = ctypes.c_void_p
+    cl = (ctypes.c_uint8 * 5)(0, 2, 3, 4, 8)
+    bad_cl = (ctypes.c_uint8 * 3)(0, 4, 4)
+    ws = ctypes.c_size_t()
+    # NULL layout / NULL pointers
+    assert g._pack(None, P(0x1000), P(0x1000), P(0x1000), None) == 1
+    assert g._pack(_L(g, 8, 8), None, P(0x1000), P(0x1000), None) == 1
+    # layout that grinqh_layout_init would not produce
+    L = g.layout(8, 8)
+    L.tile_n = 256
+    assert g._pack(ctypes.byref(L), P(0x1000), P(0x1000), P(0x1000), None) == 1
+    # misaligned planes (alignment checked before launch)
+    assert g._pack(_L(g, 8, 8), P(0x1000), P(0x1008), P(0x1000), None) == 2
+    # select: bad class sets, bad K, misaligned idx
+    assert g._select(P(0x1000), 8, P(0x1000), ctypes.addressof(bad_cl), 3, P(0x1000), P(0x1000), P(0x1000), None) == 1
+    assert g._select(P(0x1000), 8, P(0x1000), ctypes.addressof(cl), 10, P(0x1000), P(0x1000), P(0x1000), None) == 1
+    assert g._select(P(0x1000), 0, P(0x1000), ctypes.addressof(cl), 5, P(0x1000), P(0x1000), P(0x1000), None) == 1
+    assert g._select(P(0x1000), 8, P(0x1000), ctypes.addressof(cl), 5, P(0x1000), P(0x1002), P(0x1000), None) == 2
+    assert g._select(None, 8, P(0x1000), ctypes.addressof(cl), 5, P(0x1000), P(0x1000), P(0x1000), None) == 1
+    # vmm: workspace too small / missing, misaligned y
+    L = g.layout(64, 1024)
+    need = g.vmm_workspace_bytes(L)
+    args = [ctypes.byref(L), P(0x1000), P(0x1000), P(0x1000), P(0x1000), P(0x1000), ctypes.addressof(cl), 5,
+            P(0x1000)]
+    assert g._vmm(*args, None, need, None) == 4
+    assert g._vmm(*args, P(0x1000), need - 1, None) == 4
+    a2 = list(args)
+    a2[8] = P(0x1002)
+    assert g._vmm(*a2, P(0x1000), need, None) == 2
+    assert g._vmm(*args[:6], ctypes.addressof(bad_cl), 3, P(0x1000), P(0x1000), need, None) == 1
+    # calibrate: bad P, missing workspace
+    Pbad = (ctypes.c_double * 5)(0.5, 0.5, 0.5, 0.0, 0.0)
+    assert g._calibrate(P(0x1000), 4, 16, ctypes.addressof(cl), 5, ctypes.addressof(Pbad), 0.0, P(0x1000),
+                        P(0x1000), 1 << 20, None) == 1
+    Pneg = (ctypes.c_double * 5)(-0.5, 0.5, 0.5, 0.5, 0.0)
+    assert g._calibrate(P(0x1000), 4, 16, ctypes.addressof(cl), 5, ctypes.addressof(Pneg), 0.0, P(0x1000),
+                        P(0x1000), 1 << 20, None) == 1
+    assert g._calibrate(P(0x1000), 4, 16, ctypes.addressof(cl), 5, None, 9.0, P(0x1000), P(0x1000), 1 << 20,
+                        None) == 1
+    assert g._calibrate(P(0x1000), 4, 16, ctypes.addressof(cl), 5, None, 3.0, P(0x1000), None, 0, None) == 4
+    assert g._calibrate(P(0x1000), 0, 16, ctypes.addressof(cl), 5, None, 3.0, P(0x1000), P(0x1000), 1 << 20,
+                        None) == 1
+    assert g._cal_ws(70000, 5, ctypes.byref(ws)) == 1
+    assert g._cal_ws(128, 5, ctypes.byref(ws)) == 0 and ws.value >= 128 * 4 * 8
