@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/grinqh.h"
+#include "common.cuh"
 #include "kernels.h"
 
 using namespace grinqh;
@@ -15,7 +16,6 @@ namespace {
 
 constexpr int64_t kMaxDim = int64_t(1) << 24;
 constexpr int64_t kMaxElems = int64_t(1) << 34;
-constexpr int kTileN = 512;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -90,28 +90,25 @@ grinqh_status grinqh_layout_init(int32_t K, int32_t N, grinqh_layout* out) {
   L.n_groups = (N + GRINQH_GROUP - 1) / GRINQH_GROUP;
   L.tile_n = kTileN;
   L.n_tiles = (N + kTileN - 1) / kTileN;
-  L.meta_stride = L.n_tiles * (kTileN / GRINQH_GROUP);
-  L.planes_bytes = (int64_t)L.n_tiles * K * kTileN;
-  L.meta_bytes = (int64_t)4 * K * L.meta_stride;
+  L.record_bytes = kRecordBytes;
+  L.packed_bytes = (int64_t)K * L.n_tiles * kRecordBytes;
   *out = L;
   return GRINQH_OK;
 }
 
-grinqh_status grinqh_pack(const grinqh_layout* layout, const float* W, void* planes, uint32_t* meta,
-                          void* stream) {
-  if (!layout_ok(layout) || !W || !planes || !meta) return GRINQH_ERR_INVALID_ARG;
-  if (!aligned(W, 4) || !aligned(planes, 16) || !aligned(meta, 16)) return GRINQH_ERR_ALIGNMENT;
+grinqh_status grinqh_pack(const grinqh_layout* layout, const float* W, void* packed, void* stream) {
+  if (!layout_ok(layout) || !W || !packed) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(W, 4) || !aligned(packed, 16)) return GRINQH_ERR_ALIGNMENT;
   const grinqh_layout& L = *layout;
-  return cuda_status(launch_pack(W, L.K, L.N, L.tile_n, L.n_tiles, L.meta_stride, L.n_groups, planes,
-                                 meta, (cudaStream_t)stream));
+  return cuda_status(launch_pack(W, L.K, L.N, L.n_tiles, L.n_groups, packed, (cudaStream_t)stream));
 }
 
-grinqh_status grinqh_unpack_codes(const grinqh_layout* layout, const void* planes, const uint8_t* bits,
+grinqh_status grinqh_unpack_codes(const grinqh_layout* layout, const void* packed, const uint8_t* bits,
                                   uint8_t* codes, void* stream) {
-  if (!layout_ok(layout) || !planes || !codes) return GRINQH_ERR_INVALID_ARG;
-  if (!aligned(planes, 16)) return GRINQH_ERR_ALIGNMENT;
+  if (!layout_ok(layout) || !packed || !codes) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(packed, 16)) return GRINQH_ERR_ALIGNMENT;
   const grinqh_layout& L = *layout;
-  return cuda_status(launch_unpack(planes, bits, L.K, L.N, L.tile_n, L.n_tiles, codes, (cudaStream_t)stream));
+  return cuda_status(launch_unpack(packed, bits, L.K, L.N, L.n_tiles, codes, (cudaStream_t)stream));
 }
 
 grinqh_status grinqh_maxent_distribution(const uint8_t* classes, int32_t n_classes, double target_bits,
@@ -223,13 +220,12 @@ grinqh_status grinqh_vmm_workspace_bytes(const grinqh_layout* layout, size_t* by
   return GRINQH_OK;
 }
 
-grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* planes, const uint32_t* meta,
-                         const uint16_t* x, const int32_t* idx, const int32_t* offsets, const uint8_t* classes,
-                         int32_t n_classes, float* y, void* workspace, size_t workspace_bytes, void* stream) {
+grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* packed, const uint16_t* x, const int32_t* idx,
+                         const int32_t* offsets, const uint8_t* classes, int32_t n_classes, float* y,
+                         void* workspace, size_t workspace_bytes, void* stream) {
   if (!layout_ok(layout) || !valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
-  if (!planes || !meta || !x || !idx || !offsets || !y) return GRINQH_ERR_INVALID_ARG;
-  if (!aligned(planes, 16) || !aligned(meta, 16) || !aligned(x, 2) || !aligned(idx, 4) ||
-      !aligned(offsets, 4) || !aligned(y, 4))
+  if (!packed || !x || !idx || !offsets || !y) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(x, 2) || !aligned(idx, 4) || !aligned(offsets, 4) || !aligned(y, 4))
     return GRINQH_ERR_ALIGNMENT;
   const grinqh_layout& L = *layout;
   const size_t need = vmm_workspace_bytes(L.n_tiles, L.tile_n);
@@ -238,17 +234,14 @@ grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* planes, const 
   VmmArgs a{};
   a.K = L.K;
   a.N = L.N;
-  a.tile_n = L.tile_n;
   a.n_tiles = L.n_tiles;
-  a.meta_stride = L.meta_stride;
-  a.planes = (const uint32_t*)planes;
-  a.meta = meta;
+  a.packed = (const uint8_t*)packed;
   a.x = x;
   a.idx = idx;
   a.offsets = offsets;
   a.y = y;
-  a.accum = (float*)workspace;
-  a.counters = (uint32_t*)((char*)workspace + (size_t)L.n_tiles * L.tile_n * sizeof(float));
+  a.status = (uint32_t*)workspace;
+  a.partial = (float*)((char*)workspace + 16);
   a.ct = table(classes, n_classes);
   return cuda_status(launch_vmm(a, (cudaStream_t)stream));
 }

@@ -19,6 +19,10 @@ namespace grinqh {
 
 constexpr int kPlanes = 8;
 constexpr int kGroup = 128;
+constexpr int kTileN = 1024;                          // columns per tile
+constexpr int kMetaBytes = 4 * (kTileN / kGroup);     // scale/zero words at the head of a record
+constexpr int kPlaneBytes = kTileN / 8;               // one plane of one tile row
+constexpr int kRecordBytes = kMetaBytes + kPlanes * kPlaneBytes;   // 1056 = 33 sectors of 32 B
 
 // Bit position of local column c (0..31 inside its word) in plane p's word.
 __host__ __device__ __forceinline__ int bit_pos(int p, int c) {

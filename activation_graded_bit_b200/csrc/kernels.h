@@ -7,11 +7,10 @@
 
 namespace grinqh {
 
-cudaError_t launch_pack(const float* W, int K, int N, int tile_n, int n_tiles, int meta_stride,
-                        int n_groups, void* planes, uint32_t* meta, cudaStream_t st);
+cudaError_t launch_pack(const float* W, int K, int N, int n_tiles, int n_groups, void* packed, cudaStream_t st);
 
-cudaError_t launch_unpack(const void* planes, const uint8_t* bits, int K, int N, int tile_n,
-                          int n_tiles, uint8_t* codes, cudaStream_t st);
+cudaError_t launch_unpack(const void* packed, const uint8_t* bits, int K, int N, int n_tiles, uint8_t* codes,
+                          cudaStream_t st);
 
 struct ClassTable {
   int n;              // number of classes (1..9)
@@ -22,15 +21,14 @@ cudaError_t launch_select(const uint16_t* x, int K, const float* thresholds, con
                           uint8_t* bits, int32_t* idx, int32_t* offsets, cudaStream_t st);
 
 struct VmmArgs {
-  int K, N, tile_n, n_tiles, meta_stride;
-  const uint32_t* planes;
-  const uint32_t* meta;
+  int K, N, n_tiles;
+  const uint8_t* packed;
   const uint16_t* x;
   const int32_t* idx;
   const int32_t* offsets;
   float* y;
-  float* accum;         // workspace: n_tiles * tile_n floats, zero between calls
-  uint32_t* counters;   // workspace: n_tiles tickets, zero between calls
+  uint32_t* status;     // workspace: sticky error word (bit 0: a bounded wait timed out)
+  float* partial;       // workspace: per-row-split partial sums [R][n_tiles * 1024]
   ClassTable ct;
 };
 

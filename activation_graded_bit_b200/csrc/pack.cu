@@ -24,18 +24,17 @@ __device__ __forceinline__ double f16_to_f64(uint16_t h) {
   return (double)__half2float(__ushort_as_half(h));
 }
 
-// One CTA per (tile t, row k): 4 warps, warp g handles the tile's group g.
-// 128 threads then build the 8 x 16 plane words of the record.
-__global__ void __launch_bounds__(128) pack_kernel(const float* __restrict__ W, int K, int N,
-                                                   int tile_n, int meta_stride, int n_groups,
-                                                   uint32_t* __restrict__ planes,
-                                                   uint32_t* __restrict__ meta) {
-  __shared__ uint8_t codes[512];
+// One CTA per (row k, tile t): 8 warps, warp g handles the tile's group g
+// (128 columns), then 256 threads build the 8 x 32 plane words of the record.
+__global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ W, int K, int N, int n_tiles,
+                                                   int n_groups, uint8_t* __restrict__ packed) {
+  __shared__ uint8_t codes[kTileN];
   const int k = blockIdx.x, t = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gl = t * (tile_n / kGroup) + warp;     // global group index
+  const int gl = t * (kTileN / kGroup) + warp;     // global group index
   const int c0 = gl * kGroup;                      // first column of the group
   const float* row = W + (size_t)k * N;
+  uint8_t* rec = packed + ((size_t)k * n_tiles + t) * kRecordBytes;
 
   float v[4];
   float mn = INFINITY, mx = -INFINITY;
@@ -74,58 +73,58 @@ __global__ void __launch_bounds__(128) pack_kernel(const float* __restrict__ W, 
     }
     codes[warp * kGroup + lane + 32 * e] = q;
   }
-  if (lane == 0) meta[(size_t)k * meta_stride + gl] = live ? ((uint32_t)sb | ((uint32_t)zb << 16)) : 0u;
+  if (lane == 0)
+    reinterpret_cast<uint32_t*>(rec)[warp] = live ? ((uint32_t)sb | ((uint32_t)zb << 16)) : 0u;
   __syncthreads();
 
-  // thread -> (plane p, word w): 8 planes x 16 words for a 512-column tile
-  const int p = threadIdx.x >> 4, w = threadIdx.x & 15;
+  // thread -> (plane p, word w): 8 planes x 32 words for a 1024-column tile
+  const int p = threadIdx.x >> 5, w = threadIdx.x & 31;
   uint32_t word = 0;
 #pragma unroll 8
   for (int L = 0; L < 32; ++L) {
     const int c = 32 * w + col_at(p, L);
     word |= (uint32_t)((codes[c] >> (7 - p)) & 1u) << L;
   }
-  uint32_t* rec = planes + ((size_t)t * K + k) * (tile_n / 4);
-  rec[p * (tile_n / 32) + w] = word;
+  reinterpret_cast<uint32_t*>(rec + kMetaBytes + p * kPlaneBytes)[w] = word;
 }
 
-// Decoder: 16 threads per (tile, row) record, 8 records per CTA.
+// Decoder: one warp per (row, tile) record, 8 records per CTA.
 template <int B>
-__device__ __forceinline__ void decode_word(const uint32_t* plane_w, int stride_words, uint32_t (&R)[8]) {
+__device__ __forceinline__ void decode_word(const uint8_t* rec, int w, uint32_t (&R)[8]) {
   uint32_t P[8];
 #pragma unroll
-  for (int p = 0; p < 8; ++p) P[p] = (p < B) ? plane_w[p * stride_words] : 0u;
+  for (int p = 0; p < 8; ++p)
+    P[p] = (p < B) ? reinterpret_cast<const uint32_t*>(rec + kMetaBytes + p * kPlaneBytes)[w] : 0u;
   assemble<B>(P, R);
   const uint32_t mid = midpoint_bytes(B);
 #pragma unroll
   for (int j = 0; j < 8; ++j) R[j] |= mid;
 }
 
-__global__ void __launch_bounds__(128) unpack_kernel(const uint32_t* __restrict__ planes,
+__global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__ packed,
                                                      const uint8_t* __restrict__ bits, int K, int N,
-                                                     int tile_n, uint8_t* __restrict__ codes) {
+                                                     int n_tiles, uint8_t* __restrict__ codes) {
   const int t = blockIdx.y;
-  const int k = blockIdx.x * 8 + (threadIdx.x >> 4);
-  const int w = threadIdx.x & 15;
+  const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int w = threadIdx.x & 31;
   if (k >= K) return;
   const int b = bits ? bits[k] : 8;
-  const uint32_t* rec = planes + ((size_t)t * K + k) * (tile_n / 4) + w;
-  const int sw = tile_n / 32;
+  const uint8_t* rec = packed + ((size_t)k * n_tiles + t) * kRecordBytes;
   uint32_t R[8];
   switch (b) {
-    case 1: decode_word<1>(rec, sw, R); break;
-    case 2: decode_word<2>(rec, sw, R); break;
-    case 3: decode_word<3>(rec, sw, R); break;
-    case 4: decode_word<4>(rec, sw, R); break;
-    case 5: decode_word<5>(rec, sw, R); break;
-    case 6: decode_word<6>(rec, sw, R); break;
-    case 7: decode_word<7>(rec, sw, R); break;
-    case 8: decode_word<8>(rec, sw, R); break;
+    case 1: decode_word<1>(rec, w, R); break;
+    case 2: decode_word<2>(rec, w, R); break;
+    case 3: decode_word<3>(rec, w, R); break;
+    case 4: decode_word<4>(rec, w, R); break;
+    case 5: decode_word<5>(rec, w, R); break;
+    case 6: decode_word<6>(rec, w, R); break;
+    case 7: decode_word<7>(rec, w, R); break;
+    case 8: decode_word<8>(rec, w, R); break;
     default:
 #pragma unroll
       for (int j = 0; j < 8; ++j) R[j] = 0u;
   }
-  const int n0 = t * tile_n + 32 * w;
+  const int n0 = t * kTileN + 32 * w;
   uint8_t* out = codes + (size_t)k * N;
 #pragma unroll
   for (int j = 0; j < 8; ++j)
@@ -136,17 +135,16 @@ __global__ void __launch_bounds__(128) unpack_kernel(const uint32_t* __restrict_
     }
 }
 
-cudaError_t launch_pack(const float* W, int K, int N, int tile_n, int n_tiles, int meta_stride,
-                        int n_groups, void* planes, uint32_t* meta, cudaStream_t st) {
+cudaError_t launch_pack(const float* W, int K, int N, int n_tiles, int n_groups, void* packed, cudaStream_t st) {
   dim3 grid(K, n_tiles);
-  pack_kernel<<<grid, 128, 0, st>>>(W, K, N, tile_n, meta_stride, n_groups, (uint32_t*)planes, meta);
+  pack_kernel<<<grid, 256, 0, st>>>(W, K, N, n_tiles, n_groups, (uint8_t*)packed);
   return cudaGetLastError();
 }
 
-cudaError_t launch_unpack(const void* planes, const uint8_t* bits, int K, int N, int tile_n,
-                          int n_tiles, uint8_t* codes, cudaStream_t st) {
+cudaError_t launch_unpack(const void* packed, const uint8_t* bits, int K, int N, int n_tiles, uint8_t* codes,
+                          cudaStream_t st) {
   dim3 grid((K + 7) / 8, n_tiles);
-  unpack_kernel<<<grid, 128, 0, st>>>((const uint32_t*)planes, bits, K, N, tile_n, codes);
+  unpack_kernel<<<grid, 256, 0, st>>>((const uint8_t*)packed, bits, K, N, n_tiles, codes);
   return cudaGetLastError();
 }
 

@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <cuda_fp16.h>
 
+#include "async.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -39,11 +40,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __r
   __shared__ float s_thr[8];
   __shared__ int s_tot[9];
   __shared__ int s_off[10];
+  __shared__ uint8_t s_width[9];
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int n = ct.n - 1;
+#pragma unroll
+  for (int c = 0; c < 9; ++c)
+    if (tid == c && c < ct.n) s_width[c] = ct.width[c];
+  pdl_wait();   // x and the thresholds may come from the kernel just before
   if (tid < n) s_thr[tid] = thresholds[tid];
   __syncthreads();
+  pdl_launch_dependents();
   float thr[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) thr[i] = (i < n) ? s_thr[i] : 0.0f;
@@ -57,7 +64,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __r
     const int j = grade_one(x[k], thr, n);
 #pragma unroll
     for (int c = 0; c < 9; ++c) cnt[c] += (j == c) ? 1 : 0;
-    bits[k] = ct.width[j];
+    bits[k] = s_width[j];
   }
 
   // Block-wide exclusive scan of the nine per-thread counts: warp shuffles, then
@@ -111,8 +118,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __r
 
 cudaError_t launch_select(const uint16_t* x, int K, const float* thresholds, const ClassTable& ct,
                           uint8_t* bits, int32_t* idx, int32_t* offsets, cudaStream_t st) {
-  select_kernel<<<1, kSelThreads, 0, st>>>(x, K, thresholds, ct, bits, idx, offsets);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, 1);
+  cfg.blockDim = dim3(kSelThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, select_kernel, x, K, thresholds, ct, bits, idx, offsets);
 }
 
 }  // namespace grinqh

@@ -2,170 +2,316 @@
 //
 // Paper: "GRINQH" Fig. 2 and Section 3.3: for every input channel k with
 // b_k > 0 only the b_k most significant slices of row k move from DRAM to the
-// SM; the row is rebuilt on chip and channels with b_k = 0 are bypassed. The
+// SM; the row is rebuilt on chip; channels with b_k = 0 are bypassed. The
 // rebuilt weight is w_hat = s * (code - z), code = c_b * 2^(8-b) + 2^(7-b) for
-// b < 8 (Section 3.3, bias correction) and q for b = 8.
+// b < 8 (the bias correction of Section 3.3) and q for b = 8.
 //
-// Work split. The grid is (column tile t, row split r). Every CTA walks the same
-// class-ordered channel list from grinqh_select; the list is cut into
-// gridDim.y pieces of equal DRAM cost (16 B of scale/zero + 64 B per plane for a
-// 512-column tile), computed in each CTA from the class offsets alone. Because
-// classes are stored in ascending width and only the first can be 0, the rows
-// to read form one contiguous stretch of the list.
+// Work split. The grid is (column tile t of 1024 columns, row split r), one CTA
+// per SM. Every CTA walks the class-ordered channel list written by
+// grinqh_select, skipping the width-0 class (classes are stored by ascending
+// width and only the first can be 0, so the rows to read form one contiguous
+// stretch of the list). CTA r of R takes every R-th row of that stretch, so
+// every CTA gets the same mix of widths: equal DRAM bytes and equal arithmetic
+// per CTA. While staging its rows a CTA also gathers each row's x_k, so the
+// main loop reads no global memory except the weights.
 //
-// Arithmetic. Per row, per 128-column group: a = x_k * s_kg is exact in fp32
-// (two 11-bit significands). The truncated code c (low bits zero) is turned
-// into a float exactly, and the row adds a * c to the column accumulators and
-// a * (mid_b - z) once to a per-thread constant, since every column of a thread
-// shares one group.
+// Data movement (sm_100a). Each of the 16 warps is a "row lane" that takes
+// rows h, h+16, ... of its CTA, two at a time, and owns a private ring of 6
+// two-row slots in shared memory, each with its own mbarrier: 12 rows in
+// flight per warp. Lane 0 fetches a row with ONE 1-D TMA bulk copy
+// (cp.async.bulk, no tensor map, no multicast) of the record's scale/zero
+// words and top b planes, 32 + 128 b contiguous, sector-aligned bytes,
+// completing on the slot's mbarrier. On this part the time of such a copy is
+// set by the number of copies in flight, not by their size (64..512 B copies
+// cost the same), so the record layout keeps one copy per (row, tile) and the
+// tile at 1024 columns. TMA copies also bypass L1's miss tracking, which
+// per-thread copies of short scattered rows exhaust. The 32 threads of the warp
+// then rebuild both rows of the slot, one 32-bit plane word (32 columns) each;
+// two independent rows per wait double the instruction-level parallelism.
 //
-// Reduction. 16 row lanes of a CTA are summed in shared memory; CTAs of one
-// column tile add into an fp32 accumulator in the workspace with L2 atomics.
-// The last CTA of a tile to finish (a ticket counter, no waiting) copies the
-// tile to y and clears the accumulator and the ticket, so the workspace is
-// zero again for the next call.
+// Arithmetic per row and thread. a = x_k * s is exact in fp32 (two 11-bit
+// significands). The b plane words are merged into 8 registers of 4 truncated
+// codes each (one LOP3 per plane plus one rotate, thanks to the bit order chosen
+// at pack time). Codes become floats without a per-code integer extraction:
+// a byte-permute puts two codes c1:c0 in the low 16 bits of an otherwise zero
+// word, i.e. the subnormal float (256 c1 + c0) 2^-149; adding 2^-118 with
+// round-down leaves exactly 2^-118 + c1 2^-141, so one more subtraction gives
+// hi = c1 2^-141 and another gives lo = c0 2^-149, all exact and all on the FP32
+// pipe (B200 runs FFMA with subnormal operands at full rate, while byte
+// extraction would run on the half-rate integer pipe). The products use
+// coefficients a 2^95 and a 2^87, so the accumulators hold a * code * 2^-54
+// (no overflow for |a| <= 2^32, no precision loss for the sizes that matter).
+// The per-row constant a * (mid_b - z) goes to one scalar per thread, since
+// all 32 columns of a thread share one 128-column group.
+//
+// Reduction. The 16 row lanes of a CTA are summed in shared memory into one
+// 1024-column partial, stored with plain coalesced stores into the workspace
+// as partial[r][column]. A second kernel, chained with programmatic dependent
+// launch, sums the R partials of every column in a fixed order and overwrites
+// y. (Adding partials into y with L2 atomics instead costs far more: up to 148
+// CTAs would add into the same 1024..16384 addresses, and same-address
+// reductions serialise in L2.) With a single row split (R = 1) the CTA writes
+// y directly and no second kernel runs.
 #include <cstdint>
 #include <cuda_fp16.h>
 
+#include "async.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
 namespace grinqh {
 
-constexpr int kTile = 512;                 // columns per tile
-constexpr int kWords = kTile / 32;         // plane words per tile row
-constexpr int kThreads = 256;
-constexpr int kLanes = kThreads / kWords;  // rows processed side by side
+constexpr int kWords = kTileN / 32;              // plane words per tile row (32)
+constexpr int kWarps = 16;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kLanes = kWarps;                   // row lanes (warps)
+constexpr int kPairs = 6;                        // two-row slots per row lane (12 rows in flight)
+constexpr int kIdxCap = 2048;                    // rows of a CTA staged per pass
+constexpr int kRedPitch = 33;                    // column c of word w at c*33 + w: conflict-free both ways
+constexpr int kRedStride = 32 * kRedPitch + 16;  // floats per row lane in the reduction buffer
 
-__device__ __forceinline__ float byte_as_float(uint32_t r, int i) {
-  // 0x4B000000 | byte is the float 2^23 + byte; subtracting 2^23 is exact
-  const uint32_t f = __byte_perm(r, 0x4B000000u, 0x7650u | (uint32_t)i);
-  return __uint_as_float(f) - 8388608.0f;
-}
+struct __align__(128) VmmSmem {
+  uint8_t ring[kLanes][kPairs][2][kRecordBytes];
+  uint64_t bar[kLanes][kPairs];                  // one mbarrier per two-row slot
+  uint32_t slot_b[kLanes][kPairs][2];            // widths of the rows in each slot (0: no row)
+  float slot_x[kLanes][kPairs][2];               // x_k of the rows in each slot
+  uint32_t rows[kIdxCap];                        // k | b << 24 of this CTA's rows, one pass
+  float rows_x[kIdxCap];                         // x_k of those rows
+  int off[10];
+  int width[9];
+  int abort;
+};
+static_assert(sizeof(float) * kLanes * kRedStride <= sizeof(uint8_t) * kLanes * kPairs * 2 * kRecordBytes,
+              "reduction buffer must fit in the ring");
 
-// cost of one row of class width b, in 16-byte units of a 512-column tile
-__device__ __forceinline__ long long row_cost(int b) { return b > 0 ? 1 + 4 * b : 0; }
-
-// First list position whose cumulative cost, scaled by R, reaches X.
-__device__ long long split_point(const int* off, const ClassTable& ct, int first_active, int K,
-                                 long long X, int R) {
-  long long C = 0;   // cost before the current class
-  for (int j = first_active; j < ct.n; ++j) {
-    const long long c = row_cost(ct.width[j]);
-    const long long cnt = off[j + 1] - off[j];
-    if ((C + cnt * c) * R >= X) {
-      const long long need = X - C * R;            // > 0 unless X <= C*R
-      long long m = need <= 0 ? 0 : (need + c * R - 1) / (c * R);
-      if (m > cnt) m = cnt;
-      return off[j] + m;
-    }
-    C += cnt * c;
-  }
-  return K;
-}
-
+// One row of one tile: rec = the record (scale/zero words, then the planes);
+// thread w owns plane word w, i.e. columns 32w..32w+31 of the tile.
 template <int B>
-__device__ __forceinline__ void process_rows(const VmmArgs& a, int t, int lo, int hi, int lane_row,
-                                             int w, float (&acc)[32], float& cacc) {
-  const int K = a.K;
-  const uint32_t* plane_base = a.planes + (size_t)t * K * (kTile / 4) + w;
-  const uint32_t* meta_base = a.meta + t * (kTile / kGroup) + (w >> 2);
+__device__ __forceinline__ void row_fma(const uint8_t* __restrict__ rec, int w, float xk, float2 (&acc)[16],
+                                        float& cacc) {
+  const uint32_t m = reinterpret_cast<const uint32_t*>(rec)[w >> 2];
+  uint32_t P[8];
+#pragma unroll
+  for (int p = 0; p < 8; ++p)
+    P[p] = (p < B) ? reinterpret_cast<const uint32_t*>(rec + kMetaBytes + p * kPlaneBytes)[w] : 0u;
+  uint32_t R[8];
+  assemble<B>(P, R);
+  const float s = half_bits_to_float(m);
+  const float z = half_bits_to_float(m >> 16);
+  const float av = xk * s;                                   // exact
   const float mid = (B >= 8) ? 0.0f : (float)(1 << (7 - B));
-  for (int i = lo + lane_row; i < hi; i += kLanes) {
-    const int k = a.idx[i];
-    const uint32_t m = __ldg(meta_base + (size_t)k * a.meta_stride);
-    const float xk = __half2float(__ushort_as_half(__ldg(a.x + k)));
-    const float s = half_bits_to_float(m);
-    const float z = half_bits_to_float(m >> 16);
-    const float av = xk * s;   // exact: 11-bit x 11-bit significands
-    uint32_t P[8];
-    const uint32_t* rec = plane_base + (size_t)k * (kTile / 4);
+  cacc = fmaf(av, mid - z, cacc);
+  const float2 A0 = make_float2(av * 0x1p95f, av * 0x1p95f);   // for c0 2^-149
+  const float2 A1 = make_float2(av * 0x1p87f, av * 0x1p87f);   // for c1 2^-141
+  const float2 M = make_float2(0x1p-118f, 0x1p-118f);
+  const float2 NM = make_float2(-0x1p-118f, -0x1p-118f);
+  const float2 NEG1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
-    for (int p = 0; p < 8; ++p) P[p] = (p < B) ? __ldg(rec + p * kWords) : 0u;
-    uint32_t R[8];
-    assemble<B>(P, R);
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int i4 = 0; i4 < 4; ++i4) acc[4 * j + i4] = fmaf(av, byte_as_float(R[j], i4), acc[4 * j + i4]);
-    cacc = fmaf(av, mid - z, cacc);
+  for (int j = 0; j < 8; ++j) {
+    // X.x = codes of columns 4j+1 : 4j, X.y = columns 4j+3 : 4j+2, as subnormals
+    const float2 X = make_float2(__uint_as_float(__byte_perm(R[j], 0u, 0x4410u)),
+                                 __uint_as_float(__byte_perm(R[j], 0u, 0x4432u)));
+    const float2 u = __fadd2_rd(X, M);           // 2^-118 + c_hi 2^-141
+    const float2 hi = __fadd2_rn(u, NM);         // c_hi 2^-141
+    const float2 lo = __ffma2_rn(hi, NEG1, X);   // c_lo 2^-149
+    acc[2 * j] = __ffma2_rn(A0, lo, acc[2 * j]);           // columns 4j, 4j+2
+    acc[2 * j + 1] = __ffma2_rn(A1, hi, acc[2 * j + 1]);   // columns 4j+1, 4j+3
   }
 }
 
-__global__ void __launch_bounds__(kThreads) vmm_kernel(const VmmArgs a) {
-  __shared__ int s_off[10];
-  __shared__ float s_red[kLanes][kTile + 16];
-  __shared__ int s_last;
+__device__ __forceinline__ void row_any(int b, const uint8_t* rec, int w, float xk, float2 (&acc)[16],
+                                        float& cacc) {
+  switch (b) {
+    case 1: row_fma<1>(rec, w, xk, acc, cacc); break;
+    case 2: row_fma<2>(rec, w, xk, acc, cacc); break;
+    case 3: row_fma<3>(rec, w, xk, acc, cacc); break;
+    case 4: row_fma<4>(rec, w, xk, acc, cacc); break;
+    case 5: row_fma<5>(rec, w, xk, acc, cacc); break;
+    case 6: row_fma<6>(rec, w, xk, acc, cacc); break;
+    case 7: row_fma<7>(rec, w, xk, acc, cacc); break;
+    case 8: row_fma<8>(rec, w, xk, acc, cacc); break;
+    default: break;
+  }
+}
+
+// Both rows of a slot; when they share a width the two rebuilds sit in one
+// basic block, so their independent chains interleave.
+template <int B>
+__device__ __forceinline__ void row_pair(const uint8_t* r0, const uint8_t* r1, int w, float x0, float x1,
+                                         float2 (&acc)[16], float& cacc) {
+  row_fma<B>(r0, w, x0, acc, cacc);
+  row_fma<B>(r1, w, x1, acc, cacc);
+}
+
+// Lane 0 of row lane h: fetch this CTA's rows q0 and q0 + 16 (when < nq) into
+// two-row slot d, one bulk copy per row completing on the slot's mbarrier.
+__device__ __forceinline__ void issue_pair(VmmSmem& s, const VmmArgs& a, int t, int h, int d, int q0, int nq) {
+  uint32_t bytes = 0;
+  uint32_t bb[2], kk[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int q = q0 + kLanes * e;
+    const uint32_t info = (q < nq) ? s.rows[q] : 0u;
+    kk[e] = info & 0xFFFFFFu;
+    bb[e] = info >> 24;
+    s.slot_b[h][d][e] = bb[e];
+    s.slot_x[h][d][e] = (q < nq) ? s.rows_x[q] : 0.0f;
+    bytes += bb[e] ? (uint32_t)kMetaBytes + bb[e] * (uint32_t)kPlaneBytes : 0u;
+  }
+  mbar_arrive_expect_tx(&s.bar[h][d], bytes);
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    if (bb[e]) {
+      const uint8_t* src = a.packed + ((size_t)kk[e] * a.n_tiles + t) * kRecordBytes;
+      bulk_g2s(s.ring[h][d][e], src, (uint32_t)kMetaBytes + bb[e] * (uint32_t)kPlaneBytes, &s.bar[h][d]);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  VmmSmem& s = *reinterpret_cast<VmmSmem*>(smem_raw);
+  const int tid = threadIdx.x, h = tid >> 5, w = tid & 31;   // row lane h = warp, word w = lane
   const int t = blockIdx.x, r = blockIdx.y, R = gridDim.y;
-  const int tid = threadIdx.x;
-  const int lane_row = tid / kWords, w = tid % kWords;
-  const ClassTable& ct = a.ct;
-  if (tid <= ct.n) s_off[tid] = a.offsets[tid];
-  __syncthreads();
 
-  const int first_active = (ct.width[0] == 0) ? 1 : 0;
-  long long W = 0;
-  for (int j = first_active; j < ct.n; ++j) W += (long long)(s_off[j + 1] - s_off[j]) * row_cost(ct.width[j]);
-  const int lo = (int)split_point(s_off, ct, first_active, a.K, W * r, R);
-  const int hi = (int)split_point(s_off, ct, first_active, a.K, W * (r + 1), R);
-
-  float acc[32];
+  if (tid < kLanes * kPairs) mbar_init(&s.bar[tid / kPairs][tid % kPairs], 1);
+  if (tid == 0) s.abort = 0;
+  mbar_fence_init();
+  pdl_wait();   // the selection and x may come from the kernel just before
+  if (tid <= a.ct.n) s.off[tid] = a.offsets[tid];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) acc[c] = 0.0f;
+  for (int c = 0; c < 9; ++c)
+    if (tid == c && c < a.ct.n) s.width[c] = a.ct.width[c];
+  __syncthreads();
+  pdl_launch_dependents();
+
+  const int n = a.ct.n;
+  const int a0 = (s.width[0] == 0) ? s.off[1] : 0;      // first row to read
+  // this CTA's rows: list positions a0 + r + R*q, q = 0 .. nq_total-1
+  const int nq_total = (a.K - a0 > r) ? (a.K - a0 - r + R - 1) / R : 0;
+
+  float2 acc[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) acc[c] = make_float2(0.0f, 0.0f);
   float cacc = 0.0f;
-  for (int j = first_active; j < ct.n; ++j) {
-    const int s0 = max(lo, s_off[j]), s1 = min(hi, s_off[j + 1]);
-    if (s0 >= s1) continue;
-    switch (ct.width[j]) {
-      case 1: process_rows<1>(a, t, s0, s1, lane_row, w, acc, cacc); break;
-      case 2: process_rows<2>(a, t, s0, s1, lane_row, w, acc, cacc); break;
-      case 3: process_rows<3>(a, t, s0, s1, lane_row, w, acc, cacc); break;
-      case 4: process_rows<4>(a, t, s0, s1, lane_row, w, acc, cacc); break;
-      case 5: process_rows<5>(a, t, s0, s1, lane_row, w, acc, cacc); break;
-      case 6: process_rows<6>(a, t, s0, s1, lane_row, w, acc, cacc); break;
-      case 7: process_rows<7>(a, t, s0, s1, lane_row, w, acc, cacc); break;
-      case 8: process_rows<8>(a, t, s0, s1, lane_row, w, acc, cacc); break;
-      default: break;
+
+  int used = 0;     // two-row slots of this lane consumed so far (all passes): slot use index
+  int issued = 0;   // two-row slots of this lane fetched so far (lane 0's count)
+  for (int qb = 0; qb < nq_total; qb += kIdxCap) {
+    const int nq = min(kIdxCap, nq_total - qb);
+    __syncthreads();
+    for (int e = tid; e < nq; e += kThreads) {
+      const int pos = a0 + r + R * (qb + e);
+      int j = 0;
+      for (int c = 1; c < n; ++c) j += (pos >= s.off[c]) ? 1 : 0;
+      const int k = a.idx[pos];
+      s.rows[e] = (uint32_t)k | ((uint32_t)s.width[j] << 24);
+      s.rows_x[e] = __half2float(__ushort_as_half(a.x[k]));
     }
+    __syncthreads();
+    // rows of this lane in the pass: q = h + 16 m; pair i holds m = 2i, 2i+1.
+    // Slot uses continue across passes through `used` so barrier phases stay in step.
+    const int nrow = (nq > h) ? (nq - h + kLanes - 1) / kLanes : 0;
+    const int npair = (nrow + 1) / 2;
+    if (w == 0 && !*(volatile int*)&s.abort)
+      for (; issued < used + min(kPairs, npair); ++issued)
+        issue_pair(s, a, t, h, issued % kPairs, h + 2 * kLanes * (issued - used), nq);
+    int i = 0;
+#pragma unroll 1
+    for (; i < npair; ++i) {
+      const int u = used + i, d = u % kPairs;
+      if (*(volatile int*)&s.abort || !mbar_wait(&s.bar[h][d], (u / kPairs) & 1)) {
+        // a copy never completed: stop, report, and let the CTA finish cleanly
+        if (w == 0) { s.abort = 1; atomicOr(a.status, 1u); }
+        break;
+      }
+      const int b0 = (int)s.slot_b[h][d][0], b1 = (int)s.slot_b[h][d][1];
+      const float x0 = s.slot_x[h][d][0], x1 = s.slot_x[h][d][1];
+      const uint8_t* r0 = s.ring[h][d][0];
+      const uint8_t* r1 = s.ring[h][d][1];
+      if (b0 == b1) {
+        switch (b0) {
+          case 1: row_pair<1>(r0, r1, w, x0, x1, acc, cacc); break;
+          case 2: row_pair<2>(r0, r1, w, x0, x1, acc, cacc); break;
+          case 3: row_pair<3>(r0, r1, w, x0, x1, acc, cacc); break;
+          case 4: row_pair<4>(r0, r1, w, x0, x1, acc, cacc); break;
+          case 5: row_pair<5>(r0, r1, w, x0, x1, acc, cacc); break;
+          case 6: row_pair<6>(r0, r1, w, x0, x1, acc, cacc); break;
+          case 7: row_pair<7>(r0, r1, w, x0, x1, acc, cacc); break;
+          case 8: row_pair<8>(r0, r1, w, x0, x1, acc, cacc); break;
+          default: break;
+        }
+      } else {
+        row_any(b0, r0, w, x0, acc, cacc);
+        row_any(b1, r1, w, x1, acc, cacc);
+      }
+      __syncwarp();
+      if (w == 0 && i + kPairs < npair) {
+        issue_pair(s, a, t, h, d, h + 2 * kLanes * (i + kPairs), nq);
+        ++issued;
+      }
+    }
+    used += i;   // after an abort every later pass stops at i = 0, so passes stay uniform
+  }
+  __syncthreads();
+  if (s.abort) {
+    // let every copy this lane issued land before the shared memory is reused
+    if (w == 0)
+      for (int u = used; u < issued; ++u) (void)mbar_wait(&s.bar[h][u % kPairs], (u / kPairs) & 1);
+    __syncthreads();
   }
 
-  // column (32w + c) of the tile -> shared slot [lane_row][c*16 + w]
+  // ---------------- CTA reduction over the 16 row lanes ----------------
+  float* red = reinterpret_cast<float*>(&s.ring[0][0][0][0]);
+  {
+    float* dst = red + h * kRedStride + w;           // slot c*33 + w holds column 32w + c
 #pragma unroll
-  for (int c = 0; c < 32; ++c) s_red[lane_row][c * kWords + w] = acc[c] + cacc;
-  __syncthreads();
-  float* accum = a.accum + (size_t)t * kTile;
-  if (hi > lo) {
-    for (int e = tid; e < kTile; e += kThreads) {
-      float v = 0.0f;
-#pragma unroll
-      for (int l = 0; l < kLanes; ++l) v += s_red[l][e];
-      const int c = e / kWords, ww = e % kWords;
-      atomicAdd(accum + 32 * ww + c, v);
+    for (int j = 0; j < 8; ++j) {
+      dst[(4 * j + 0) * kRedPitch] = fmaf(acc[2 * j].x, 0x1p54f, cacc);
+      dst[(4 * j + 2) * kRedPitch] = fmaf(acc[2 * j].y, 0x1p54f, cacc);
+      dst[(4 * j + 1) * kRedPitch] = fmaf(acc[2 * j + 1].x, 0x1p54f, cacc);
+      dst[(4 * j + 3) * kRedPitch] = fmaf(acc[2 * j + 1].y, 0x1p54f, cacc);
     }
   }
-  __threadfence();
   __syncthreads();
-  if (tid == 0) {
-    const unsigned prev = atomicAdd(a.counters + t, 1u);
-    s_last = (prev == (unsigned)(R - 1));
-    __threadfence();
-  }
-  __syncthreads();
-  if (s_last) {
-    for (int e = tid; e < kTile; e += kThreads) {
-      const int n = t * kTile + e;
-      const float v = __ldcg(accum + e);
-      if (n < a.N) a.y[n] = v;
-      __stcg(accum + e, 0.0f);
-    }
-    if (tid == 0) a.counters[t] = 0u;
+  // partial[r][column], or y itself when there is a single row split; every
+  // column of the tile is written, zeros included, so no clearing is needed
+  float* out = (R == 1) ? a.y : a.partial + (size_t)r * a.n_tiles * kTileN;
+  const int limit = (R == 1) ? a.N : a.n_tiles * kTileN;
+#pragma unroll
+  for (int e = tid; e < kTileN; e += kThreads) {
+    // column e of the tile sits at slot (e % 32) * 33 + e / 32 of every row lane
+    float v = 0.0f;
+#pragma unroll
+    for (int rl = 0; rl < kLanes; ++rl) v += red[rl * kRedStride + (e % kWords) * kRedPitch + e / kWords];
+    const int col = t * kTileN + e;
+    if (col < limit) out[col] = v;
   }
 }
 
-size_t vmm_workspace_bytes(int n_tiles, int tile_n) {
-  const size_t acc = (size_t)n_tiles * tile_n * sizeof(float);
-  const size_t cnt = (size_t)n_tiles * sizeof(uint32_t);
-  return (acc + cnt + 15) & ~(size_t)15;
+// y[col] = sum over r of partial[r][col]: 256 threads = 32 columns x 8 chains;
+// chain c adds r = c, c+8, ... in ascending order, then the 8 chains are added
+// in a fixed order, so the result does not depend on timing.
+__global__ void __launch_bounds__(256) reduce_partials_kernel(const float* __restrict__ partial, int R,
+                                                              int stride, float* __restrict__ y, int N) {
+  __shared__ float s_part[8][33];
+  pdl_launch_dependents();
+  pdl_wait();   // the partials come from the VMM kernel just before
+  const int lane = threadIdx.x & 31, chain = threadIdx.x >> 5;
+  const int col = blockIdx.x * 32 + lane;
+  float v = 0.0f;
+  if (col < N) {
+#pragma unroll 4
+    for (int r = chain; r < R; r += 8) v += partial[(size_t)r * stride + col];
+  }
+  s_part[chain][lane] = v;
+  __syncthreads();
+  if (chain == 0 && col < N) {
+    float acc = s_part[0][lane];
+#pragma unroll
+    for (int c = 1; c < 8; ++c) acc += s_part[c][lane];
+    y[col] = acc;
+  }
 }
 
 static int sm_count() {
@@ -175,14 +321,51 @@ static int sm_count() {
   return n;
 }
 
+// Row splits per column tile: one CTA per SM in total.
+static int row_splits(int n_tiles) {
+  const int R = sm_count() / n_tiles;
+  return R < 1 ? 1 : R;
+}
+
+// status word (16 B), then partial[R][n_tiles * 1024] floats when R > 1
+size_t vmm_workspace_bytes(int n_tiles, int /*tile_n*/) {
+  const int R = row_splits(n_tiles);
+  return 16 + (R > 1 ? (size_t)R * n_tiles * kTileN * sizeof(float) : 0);
+}
+
 cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st) {
-  const int nsm = sm_count();
-  int R = (2 * nsm + a.n_tiles - 1) / a.n_tiles;
-  if (R < 1) R = 1;
-  if (R > 1024) R = 1024;
-  dim3 grid(a.n_tiles, R);
-  vmm_kernel<<<grid, kThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int smem = (int)sizeof(VmmSmem);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(vmm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+
+  const int R = row_splits(a.n_tiles);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.n_tiles, R, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, vmm_kernel, a);
+  if (e != cudaSuccess || R == 1) return e;
+
+  cudaLaunchConfig_t rc = {};
+  rc.gridDim = dim3((a.N + 31) / 32, 1, 1);
+  rc.blockDim = dim3(256, 1, 1);
+  rc.stream = st;
+  rc.attrs = attr;
+  rc.numAttrs = 1;
+  return cudaLaunchKernelEx(&rc, reduce_partials_kernel, (const float*)a.partial, R, a.n_tiles * kTileN, a.y,
+                            a.N);
 }
 
 }  // namespace grinqh

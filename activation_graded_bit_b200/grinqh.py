@@ -37,8 +37,8 @@ class GrinqhError(RuntimeError):
 
 class Layout(ctypes.Structure):
     _fields_ = [("K", ctypes.c_int32), ("N", ctypes.c_int32), ("n_groups", ctypes.c_int32),
-                ("tile_n", ctypes.c_int32), ("n_tiles", ctypes.c_int32), ("meta_stride", ctypes.c_int32),
-                ("planes_bytes", ctypes.c_int64), ("meta_bytes", ctypes.c_int64)]
+                ("tile_n", ctypes.c_int32), ("n_tiles", ctypes.c_int32), ("record_bytes", ctypes.c_int32),
+                ("packed_bytes", ctypes.c_int64)]
 
 
 _P = ctypes.c_void_p
@@ -56,14 +56,14 @@ def _sig(name, args, res=ctypes.c_int):
 _version = _sig("grinqh_version", [], ctypes.c_char_p)
 _status_string = _sig("grinqh_status_string", [ctypes.c_int], ctypes.c_char_p)
 _layout_init = _sig("grinqh_layout_init", [_I, _I, _LP])
-_pack = _sig("grinqh_pack", [_LP, _P, _P, _P, _P])
+_pack = _sig("grinqh_pack", [_LP, _P, _P, _P])
 _unpack = _sig("grinqh_unpack_codes", [_LP, _P, _P, _P, _P])
 _maxent = _sig("grinqh_maxent_distribution", [_P, _I, ctypes.c_double, _P])
 _cal_ws = _sig("grinqh_calibrate_workspace_bytes", [_I, _I, ctypes.POINTER(ctypes.c_size_t)])
 _calibrate = _sig("grinqh_calibrate", [_P, _I, _I, _P, _I, _P, ctypes.c_double, _P, _P, ctypes.c_size_t, _P])
 _select = _sig("grinqh_select", [_P, _I, _P, _P, _I, _P, _P, _P, _P])
 _vmm_ws = _sig("grinqh_vmm_workspace_bytes", [_LP, ctypes.POINTER(ctypes.c_size_t)])
-_vmm = _sig("grinqh_vmm", [_LP, _P, _P, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
+_vmm = _sig("grinqh_vmm", [_LP, _P, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
 
 # Every exported symbol of the C ABI, for the export check in the tests.
 EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grinqh_pack",
@@ -103,10 +103,9 @@ def layout(K: int, N: int) -> Layout:
 
 @dataclass
 class PackedLayer:
-    """Bit-plane packed K x N layer: planes (uint8 bytes) and meta (int32 words)."""
+    """Bit-plane packed K x N layer: one uint8 buffer of (row, tile) records."""
     layout: Layout
-    planes: torch.Tensor
-    meta: torch.Tensor
+    packed: torch.Tensor
 
     @property
     def K(self):
@@ -116,12 +115,16 @@ class PackedLayer:
     def N(self):
         return self.layout.N
 
+    def meta_words(self) -> torch.Tensor:
+        """uint32 view [K, n_tiles, 8] of the scale | zero << 16 words of every record."""
+        L = self.layout
+        rec = self.packed.view(L.K, L.n_tiles, L.record_bytes)
+        return rec[:, :, :32].contiguous().view(torch.int32).view(L.K, L.n_tiles, 8)
+
 
 def empty_packed(K: int, N: int, device="cuda") -> PackedLayer:
     L = layout(K, N)
-    planes = torch.empty(int(L.planes_bytes), dtype=torch.uint8, device=device)
-    meta = torch.empty(int(L.meta_bytes) // 4, dtype=torch.int32, device=device)
-    return PackedLayer(L, planes, meta)
+    return PackedLayer(L, torch.empty(int(L.packed_bytes), dtype=torch.uint8, device=device))
 
 
 def pack(W: torch.Tensor, out: Optional[PackedLayer] = None, stream=None) -> PackedLayer:
@@ -129,13 +132,13 @@ def pack(W: torch.Tensor, out: Optional[PackedLayer] = None, stream=None) -> Pac
     assert W.dtype == torch.float32 and W.is_cuda and W.is_contiguous() and W.dim() == 2
     K, N = W.shape
     p = out if out is not None else empty_packed(K, N, W.device)
-    _check(_pack(ctypes.byref(p.layout), _ptr(W), _ptr(p.planes), _ptr(p.meta), _stream(stream)), "grinqh_pack")
+    _check(_pack(ctypes.byref(p.layout), _ptr(W), _ptr(p.packed), _stream(stream)), "grinqh_pack")
     return p
 
 
 def unpack_codes(p: PackedLayer, bits: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    codes = torch.empty((p.K, p.N), dtype=torch.uint8, device=p.planes.device)
-    _check(_unpack(ctypes.byref(p.layout), _ptr(p.planes), _ptr(bits), _ptr(codes), _stream(stream)),
+    codes = torch.empty((p.K, p.N), dtype=torch.uint8, device=p.packed.device)
+    _check(_unpack(ctypes.byref(p.layout), _ptr(p.packed), _ptr(bits), _ptr(codes), _stream(stream)),
            "grinqh_unpack_codes")
     return codes
 
@@ -213,9 +216,9 @@ def vmm(p: PackedLayer, x: torch.Tensor, sel: Selection, workspace: torch.Tensor
         y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """grinqh_vmm: y[N] fp32 = x . W_hat over the graded bit planes."""
     if y is None:
-        y = torch.empty(p.N, dtype=torch.float32, device=p.planes.device)
+        y = torch.empty(p.N, dtype=torch.float32, device=p.packed.device)
     cb, n = _classes_buf(sel.classes)
-    _check(_vmm(ctypes.byref(p.layout), _ptr(p.planes), _ptr(p.meta), _ptr(x), _ptr(sel.idx), _ptr(sel.offsets),
+    _check(_vmm(ctypes.byref(p.layout), _ptr(p.packed), _ptr(x), _ptr(sel.idx), _ptr(sel.offsets),
                 ctypes.addressof(cb), n, _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),
                 _stream(stream)), "grinqh_vmm")
     return y

@@ -287,7 +287,7 @@ def run_gpu(args):
             "config": {"workload": WORKLOAD, "pairs_per_step": n_pairs, "classes": list(wl.CLASSES),
                        "l2": "inputs larger than L2: every pair of a step reads its own packed copy; "
                              "%d copies of the layer set (%.2f GB) rotate" % (
-                                 len(pairs), sum(pr["packed"].planes.numel() for pr in pairs) / 1e9),
+                                 len(pairs), sum(pr["packed"].packed.numel() for pr in pairs) / 1e9),
                        "parallelism": "replicas only" if world > 1 else "single GPU"},
             "vmm_us": round(us_vmm, 4), "select_plus_vmm_us": round(us_pair, 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -372,6 +372,35 @@ def run_reference(args):
     print(json.dumps(out))
 
 
+def run_profile_case(args):
+    """One (linear, width) pair, `--iters` eager select+vmm calls, no timing: the
+    small case that ncu captures."""
+    import torch
+    from activation_graded_bit_b200 import grinqh as g
+    from activation_graded_bit_b200 import workloads as wl
+    shapes = {name: (li, K, N) for li, (name, K, N) in enumerate(wl.LLAMA3_8B)}
+    li, K, N = shapes[args.profile]
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1_000_003 * (li + 1))
+    W = torch.randn(K, N, generator=gen, device=dev, dtype=torch.float32) * 0.02
+    p = g.pack(W)
+    del W
+    Xc = wl.activations_outlier(K, 128, key=(1, 0, li, 1), chan_key=(1, 0, li))
+    th = g.calibrate(torch.from_numpy(Xc.view(np.int16)).to(dev), wl.CLASSES, P=None, target_bits=args.bits)
+    x = wl.activations_outlier(K, 1, key=(1, 0, li, 2), chan_key=(1, 0, li))[0]
+    x_d = torch.from_numpy(x.view(np.int16)).to(dev)
+    ws = g.vmm_workspace(p.layout, dev)
+    y = torch.empty(N, dtype=torch.float32, device=dev)
+    sel = g.empty_selection(K, wl.CLASSES, dev)
+    for _ in range(args.iters):
+        g.select(x_d, th, wl.CLASSES, out=sel)
+        g.vmm(p, x_d, sel, ws, y=y)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(y).all())
+    print("profile case %s @ %g bits: %d select+vmm calls" % (args.profile, args.bits, args.iters))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -381,10 +410,15 @@ def main():
     ap.add_argument("--copies", type=int, default=2)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", default=None, help="linear name: run one small case for ncu and exit")
+    ap.add_argument("--bits", type=float, default=4.0)
+    ap.add_argument("--iters", type=int, default=3)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile:
+        run_profile_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

@@ -56,30 +56,29 @@ typedef enum {
 
 /*
  * Physical layout of a packed K x N layer. Filled by grinqh_layout_init; treat
- * as read-only. Two buffers hold the layer:
- *
- *  planes  (device, planes_bytes, 16-byte aligned): n_tiles column tiles of
- *          tile_n columns. Tile t, row k is one record of tile_n bytes at byte
- *          offset (t*K + k)*tile_n, holding the 8 planes MSB first: plane p
- *          (p = 0 is bit 7 of the code, p = 7 is bit 0) fills bytes
- *          [p*tile_n/8, (p+1)*tile_n/8) of the record, so the top b planes of a
- *          row are one contiguous run of b*tile_n/8 bytes. Inside a plane, 32-bit
- *          word w holds local columns 32w..32w+31; local column 32w + 4j + i
- *          (j in 0..7, i in 0..3) sits at bit (8i + j + 7 - p) mod 32 of the
- *          word. Columns >= N are zero bits.
- *  meta    (device, meta_bytes, 16-byte aligned): uint32 [K][meta_stride];
- *          entry g of row k is scale_fp16 | (zero_fp16 << 16) for columns
- *          [128g, 128g+128). Entries g >= n_groups are zero.
+ * as read-only. One device buffer (packed_bytes, 16-byte aligned) holds the
+ * layer. Each row is cut into n_tiles column tiles of tile_n = 1024 columns;
+ * row k, tile t is one record of record_bytes = 1056 bytes at byte offset
+ * (k*n_tiles + t)*record_bytes (a row's tiles are adjacent):
+ *   bytes [0, 32)      8 uint32 words; word g is scale_fp16 | (zero_fp16 << 16)
+ *                      of columns [t*1024 + 128g, +128) (0 past the last group);
+ *   bytes [32, 1056)   the 8 bit planes, MSB first: plane p (p = 0 is bit 7 of
+ *                      the code, p = 7 is bit 0) fills bytes
+ *                      [32 + 128p, 32 + 128(p+1)).
+ * So the scale/zero words and the top b planes of a (row, tile) are one
+ * contiguous, 32-byte-aligned run of 32 + 128b bytes. Inside a plane, 32-bit
+ * word w holds local columns 32w..32w+31; local column 32w + 4j + i (j in 0..7,
+ * i in 0..3) sits at bit (8i + j + 7 - p) mod 32 of the word. Columns >= N are
+ * zero bits.
  */
 typedef struct {
   int32_t K;             /* input channels (rows) */
   int32_t N;             /* output channels (columns) */
   int32_t n_groups;      /* ceil(N / 128) */
-  int32_t tile_n;        /* columns per tile (multiple of 128) */
+  int32_t tile_n;        /* columns per tile (1024) */
   int32_t n_tiles;       /* ceil(N / tile_n) */
-  int32_t meta_stride;   /* uint32 entries per row of meta = n_tiles*tile_n/128 */
-  int64_t planes_bytes;  /* n_tiles * K * tile_n */
-  int64_t meta_bytes;    /* 4 * K * meta_stride */
+  int32_t record_bytes;  /* bytes per (row, tile) record (1056) */
+  int64_t packed_bytes;  /* K * n_tiles * record_bytes */
 } grinqh_layout;
 
 /* Library version string (static storage). */
@@ -105,12 +104,10 @@ grinqh_status grinqh_layout_init(int32_t K, int32_t N, grinqh_layout* out);
  * quotients in fp64, ties to even.
  *   W       device, fp32 [K][N] row-major, finite values (non-finite input
  *           gives unspecified codes), 4-byte aligned.
- *   planes  device, layout->planes_bytes, 16-byte aligned; fully overwritten.
- *   meta    device, layout->meta_bytes, 16-byte aligned; fully overwritten.
+ *   packed  device, layout->packed_bytes, 16-byte aligned; fully overwritten.
  * Errors: INVALID_ARG (NULL pointers, layout inconsistent), ALIGNMENT, CUDA.
  */
-grinqh_status grinqh_pack(const grinqh_layout* layout, const float* W, void* planes,
-                          uint32_t* meta, void* stream);
+grinqh_status grinqh_pack(const grinqh_layout* layout, const float* W, void* packed, void* stream);
 
 /*
  * Decode the codes the VMM uses, for testing the packed format. For each row k
@@ -119,12 +116,12 @@ grinqh_status grinqh_pack(const grinqh_layout* layout, const float* W, void* pla
  *   1 <= b <= 7: c_b * 2^(8-b) + 2^(7-b), c_b = top b bits of q (Section 3.3
  *     reconstruction with its midpoint term);
  *   b = 8: q.
- *   planes  device, as written by grinqh_pack for the same layout.
+ *   packed  device, as written by grinqh_pack for the same layout.
  *   bits    device uint8 [K] of widths 0..8, or NULL.
  *   codes   device uint8 [K][N] row-major; fully overwritten.
  * Errors: INVALID_ARG, ALIGNMENT, CUDA.
  */
-grinqh_status grinqh_unpack_codes(const grinqh_layout* layout, const void* planes,
+grinqh_status grinqh_unpack_codes(const grinqh_layout* layout, const void* packed,
                                   const uint8_t* bits, uint8_t* codes, void* stream);
 
 /*
@@ -194,22 +191,28 @@ grinqh_status grinqh_vmm_workspace_bytes(const grinqh_layout* layout, size_t* by
 /*
  * The graded vector-matrix product (the decode hot path).
  * Paper: Fig. 2 and Section 3.3: for every channel k with b_k > 0, only planes
- * 0..b_k-1 of row k (and its scale/zero pairs) are read; the row is rebuilt as
+ * 0..b_k-1 of row k (and its scale/zero words) are read; the row is rebuilt as
  * w_hat = s * (code - z) with code = c_b * 2^(8-b) + 2^(7-b) for b < 8 and q for
  * b = 8; channels with b_k = 0 are never read and add nothing.
- *   y[n] = sum_k x_k * w_hat[k][n], accumulated in fp32 (order unspecified).
- *   planes, meta  device, from grinqh_pack with this layout.
+ *   y[n] = sum_k x_k * w_hat[k][n], accumulated in fp32.
+ *   packed        device, from grinqh_pack with this layout.
  *   x             device fp16 [K] (the same vector grinqh_select graded).
  *   idx, offsets  device, from grinqh_select with the same classes.
  *   classes       host uint8 [n_classes].
  *   y             device fp32 [N], output (overwritten), 4-byte aligned.
- *   workspace     device, >= grinqh_vmm_workspace_bytes(layout), 16-byte
- *                 aligned. It must be zero-filled once before its first use;
- *                 every call leaves it zero-filled again. Calls that share one
- *                 workspace must not overlap in time (use one stream).
+ *   workspace     device, >= grinqh_vmm_workspace_bytes(layout) (a size that
+ *                 depends on the current device's SM count), 16-byte aligned;
+ *                 its first 16 bytes must be zero-filled once before first use.
+ *                 They hold a sticky status word: 0, or nonzero if a bounded
+ *                 wait inside the kernel gave up (the output of that call is
+ *                 then invalid; clear the word before reusing). The rest holds
+ *                 per-CTA partial sums of y, fully rewritten by every call.
+ *                 Calls that share a workspace must not overlap in time.
+ * y is written with plain stores in a fixed summation order, so repeated calls
+ * on the same inputs give bitwise identical results.
  * Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, CUDA.
  */
-grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* planes, const uint32_t* meta,
+grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* packed,
                          const uint16_t* x, const int32_t* idx, const int32_t* offsets,
                          const uint8_t* classes, int32_t n_classes, float* y, void* workspace,
                          size_t workspace_bytes, void* stream);

@@ -49,7 +49,8 @@ def assert_close(y_gpu, y_ref, bound, what=""):
     return float((err / lim).max()) if err.size else 0.0
 
 
-def meta_split(meta_t, K, stride, n_groups):
-    """Device meta words -> (scale_bits, zero_bits) uint16 [K, n_groups]."""
-    m = meta_t.cpu().numpy().view(np.uint32).reshape(K, stride)[:, :n_groups]
+def meta_split(p):
+    """PackedLayer -> (scale_bits, zero_bits) uint16 [K, n_groups] from the records' head words."""
+    L = p.layout
+    m = p.meta_words().cpu().numpy().view(np.uint32).reshape(L.K, L.n_tiles * 8)[:, :L.n_groups]
     return (m & 0xFFFF).astype(np.uint16), (m >> 16).astype(np.uint16)

@@ -42,11 +42,11 @@ def test_version_and_status_strings(g):
 
 def test_layout(g):
     L = g.layout(4096, 14336)
-    assert (L.K, L.N, L.n_groups, L.tile_n, L.n_tiles) == (4096, 14336, 112, 512, 28)
-    assert L.meta_stride == 28 * 4
-    assert L.planes_bytes == 28 * 4096 * 512 and L.meta_bytes == 4 * 4096 * 112
+    assert (L.K, L.N, L.n_groups, L.tile_n, L.n_tiles) == (4096, 14336, 112, 1024, 14)
+    assert L.record_bytes == 32 + 8 * 128
+    assert L.packed_bytes == 4096 * 14 * 1056
     L = g.layout(4, 4)
-    assert (L.n_groups, L.n_tiles, L.meta_stride) == (1, 1, 4)
+    assert (L.n_groups, L.n_tiles, L.record_bytes) == (1, 1, 1056)
     for K, N in ((0, 4), (4, 0), (-1, 5), (1 << 24 + 1, 1), (1 << 24, 1 << 24)):
         with pytest.raises(g.GrinqhError) as e:
             g.layout(K, N)
@@ -78,14 +78,14 @@ def test_host_validation_rejects_before_launch(g):
     bad_cl = (ctypes.c_uint8 * 3)(0, 4, 4)
     ws = ctypes.c_size_t()
     # NULL layout / NULL pointers
-    assert g._pack(None, P(0x1000), P(0x1000), P(0x1000), None) == 1
-    assert g._pack(_L(g, 8, 8), None, P(0x1000), P(0x1000), None) == 1
+    assert g._pack(None, P(0x1000), P(0x1000), None) == 1
+    assert g._pack(_L(g, 8, 8), None, P(0x1000), None) == 1
     # layout that grinqh_layout_init would not produce
     L = g.layout(8, 8)
-    L.tile_n = 256
-    assert g._pack(ctypes.byref(L), P(0x1000), P(0x1000), P(0x1000), None) == 1
-    # misaligned planes (alignment checked before launch)
-    assert g._pack(_L(g, 8, 8), P(0x1000), P(0x1008), P(0x1000), None) == 2
+    L.tile_n = 512
+    assert g._pack(ctypes.byref(L), P(0x1000), P(0x1000), None) == 1
+    # misaligned packed buffer (alignment checked before launch)
+    assert g._pack(_L(g, 8, 8), P(0x1000), P(0x1008), None) == 2
     # select: bad class sets, bad K, misaligned idx
     assert g._select(P(0x1000), 8, P(0x1000), ctypes.addressof(bad_cl), 3, P(0x1000), P(0x1000), P(0x1000), None) == 1
     assert g._select(P(0x1000), 8, P(0x1000), ctypes.addressof(cl), 10, P(0x1000), P(0x1000), P(0x1000), None) == 1
@@ -95,14 +95,19 @@ def test_host_validation_rejects_before_launch(g):
     # vmm: workspace too small / missing, misaligned y
     L = g.layout(64, 1024)
     need = g.vmm_workspace_bytes(L)
-    args = [ctypes.byref(L), P(0x1000), P(0x1000), P(0x1000), P(0x1000), P(0x1000), ctypes.addressof(cl), 5,
-            P(0x1000)]
+    args = [ctypes.byref(L), P(0x1000), P(0x1000), P(0x1000), P(0x1000), ctypes.addressof(cl), 5, P(0x1000)]
     assert g._vmm(*args, None, need, None) == 4
     assert g._vmm(*args, P(0x1000), need - 1, None) == 4
     a2 = list(args)
-    a2[8] = P(0x1002)
+    a2[7] = P(0x1002)                       # y not 4-byte aligned
     assert g._vmm(*a2, P(0x1000), need, None) == 2
-    assert g._vmm(*args[:6], ctypes.addressof(bad_cl), 3, P(0x1000), P(0x1000), need, None) == 1
+    a3 = list(args)
+    a3[3] = P(0x1002)                       # idx not 4-byte aligned
+    assert g._vmm(*a3, P(0x1000), need, None) == 2
+    a4 = list(args)
+    a4[1] = P(0x1008)                       # packed not 16-byte aligned
+    assert g._vmm(*a4, P(0x1000), need, None) == 2
+    assert g._vmm(*args[:5], ctypes.addressof(bad_cl), 3, P(0x1000), P(0x1000), need, None) == 1
     # calibrate: bad P, missing workspace
     Pbad = (ctypes.c_double * 5)(0.5, 0.5, 0.5, 0.0, 0.0)
     assert g._calibrate(P(0x1000), 4, 16, ctypes.addressof(cl), 5, ctypes.addressof(Pbad), 0.0, P(0x1000),
