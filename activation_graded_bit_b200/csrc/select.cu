@@ -7,10 +7,21 @@
 // the upper class, NaN to class 0), and the channels are then listed class by
 // class in ascending k, which is what the VMM kernel walks.
 //
-// One CTA of 1024 threads. Thread t owns the contiguous chunk
-// [t*E, (t+1)*E) of channels, E = ceil(K / 1024), so "ascending thread, then
-// ascending position inside the chunk" is ascending k: an exclusive scan of the
-// per-thread class counts gives every channel its slot with no sorting.
+// One CTA of 512 threads per chunk of 1024 channels, with no communication
+// between CTAs:
+//  * every CTA streams all of x once (a few KB, resident in L2) and counts, for
+//    each threshold, the channels whose |x| reaches it, both over the whole
+//    vector and over the channels before its own chunk (a snapshot of the running
+//    counts taken where the stream crosses the chunk start); with the thresholds
+//    sorted, those counts give the number of channels of each class overall and
+//    before the chunk, hence the class offsets and this chunk's first slot in
+//    each class;
+//  * inside the chunk, round e of thread t grades channel lo + 512 e + t, so
+//    (round, warp, lane) order is ascending k; one ballot per class and round gives
+//    each channel its rank among the warp's channels of that class, and one warp
+//    per class scans the 32 (round, warp) counts.
+// The class count does not depend on the order of the thresholds, so grading
+// against the sorted copy gives the same j as the definition.
 #include <cstdint>
 #include <cuda_fp16.h>
 
@@ -20,106 +31,198 @@
 
 namespace grinqh {
 
-constexpr int kSelThreads = 1024;
+constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelChunk = 1024;
+constexpr int kSelRounds = kSelChunk / kSelThreads;   // 2
+constexpr int kNoClass = 15;
 
-__device__ __forceinline__ int grade_one(uint16_t h, const float* thr, int n) {
-  const float ax = fabsf(__half2float(__ushort_as_half(h)));   // exact; NaN stays NaN
-  int j = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    if (i < n) j += (ax >= thr[i]) ? 1 : 0;
-  return j;
+static_assert(kSelRounds * kSelWarps == 32, "one scan lane per (round, warp)");
+
+// Total order used to sort the thresholds: -inf < ... < -0 == +0 < ... < +inf < NaN.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  if (v != v) return 0xFFFFFFFFu;
+  uint32_t u = __float_as_uint(v);
+  if (v == 0.0f) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+__device__ __forceinline__ float abs_half(uint16_t h) {
+  return __half2float(__ushort_as_half((uint16_t)(h & 0x7FFFu)));   // exact; NaN stays NaN
+}
+
+template <int NT>
+__device__ __forceinline__ void count_ge(float ax, const float (&sig)[8], int (&c)[8]) {
+#pragma unroll
+  for (int i = 0; i < NT; ++i) c[i] += (ax >= sig[i]) ? 1 : 0;
+}
+
+template <int NT>
+__device__ __forceinline__ void snapshot(const int (&c)[8], int (&cb)[8]) {
+#pragma unroll
+  for (int i = 0; i < NT; ++i) cb[i] = c[i];
+}
+
+// c[i] = #{k : |x_k| >= sig[i]} over this thread's share of [0, K); cb[i] the
+// same over k < lo. lo is a multiple of the chunk (so of 8).
+template <int NT>
+__device__ __forceinline__ void count_all(const uint16_t* __restrict__ x, int K, int lo,
+                                          const float (&sig)[8], int (&c)[8], int (&cb)[8]) {
+  const int tid = threadIdx.x;
+  bool snap = false;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) == 0) {
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    const int g1 = K >> 3, glo = lo >> 3;
+#pragma unroll 1
+    for (int g = tid; g < g1; g += kSelThreads) {
+      if (!snap && g >= glo) {
+        snap = true;
+        snapshot<NT>(c, cb);
+      }
+      const uint4 v = __ldg(xv + g);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        count_ge<NT>(abs_half((uint16_t)(w[q] & 0xFFFFu)), sig, c);
+        count_ge<NT>(abs_half((uint16_t)(w[q] >> 16)), sig, c);
+      }
+    }
+    if (!snap) snapshot<NT>(c, cb);
+    const int k = (g1 << 3) + tid;   // at most 7 tail channels, all at or after lo
+    if (k < K) count_ge<NT>(abs_half(__ldg(x + k)), sig, c);
+  } else {
+#pragma unroll 1
+    for (int k = tid; k < K; k += kSelThreads) {
+      if (!snap && k >= lo) {
+        snap = true;
+        snapshot<NT>(c, cb);
+      }
+      count_ge<NT>(abs_half(__ldg(x + k)), sig, c);
+    }
+    if (!snap) snapshot<NT>(c, cb);
+  }
+}
+
+template <int NT>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __restrict__ x, int K,
                                                              const float* __restrict__ thresholds,
                                                              ClassTable ct, uint8_t* __restrict__ bits,
                                                              int32_t* __restrict__ idx,
                                                              int32_t* __restrict__ offsets) {
-  __shared__ int s_wtot[9][32];     // per-warp class totals, then their exclusive prefix
+  constexpr int NC = NT + 1;
   __shared__ float s_thr[8];
-  __shared__ int s_tot[9];
-  __shared__ int s_off[10];
+  __shared__ float s_sig[8];
+  __shared__ int s_nge[2][8];     // channels before the chunk / overall with |x| >= sigma_i
+  __shared__ int s_cnt[9][32];    // per (round, warp) class counts, then their exclusive prefix
+  __shared__ int s_base[9];
   __shared__ uint8_t s_width[9];
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int n = ct.n - 1;
-#pragma unroll
-  for (int c = 0; c < 9; ++c)
-    if (tid == c && c < ct.n) s_width[c] = ct.width[c];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int lo = blockIdx.x * kSelChunk, hi = min(K, lo + kSelChunk);
+  if (tid < 16) s_nge[tid >> 3][tid & 7] = 0;
+  if (tid >= 32 && tid < 32 + NC) s_width[tid - 32] = ct.width[tid - 32];
   pdl_wait();   // x and the thresholds may come from the kernel just before
-  if (tid < n) s_thr[tid] = thresholds[tid];
+  if (tid < NT) s_thr[tid] = thresholds[tid];
+  uint16_t xo[kSelRounds];
+#pragma unroll
+  for (int e = 0; e < kSelRounds; ++e) {
+    const int k = lo + e * kSelThreads + tid;
+    xo[e] = (k < hi) ? __ldg(x + k) : (uint16_t)0;
+  }
   __syncthreads();
   pdl_launch_dependents();
-  float thr[8];
+  if (tid < NT) {
+    const float v = s_thr[tid];
+    const uint32_t kv = order_key(v);
+    int r = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) thr[i] = (i < n) ? s_thr[i] : 0.0f;
-
-  const int E = (K + kSelThreads - 1) / kSelThreads;
-  const int k0 = min(K, tid * E), k1 = min(K, k0 + E);
-  int cnt[9];
-#pragma unroll
-  for (int c = 0; c < 9; ++c) cnt[c] = 0;
-  for (int k = k0; k < k1; ++k) {
-    const int j = grade_one(x[k], thr, n);
-#pragma unroll
-    for (int c = 0; c < 9; ++c) cnt[c] += (j == c) ? 1 : 0;
-    bits[k] = s_width[j];
-  }
-
-  // Block-wide exclusive scan of the nine per-thread counts: warp shuffles, then
-  // one warp per class scans the 32 warp totals.
-  int inc[9];
-#pragma unroll
-  for (int c = 0; c < 9; ++c) inc[c] = cnt[c];
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-#pragma unroll
-    for (int c = 0; c < 9; ++c) {
-      const int v = __shfl_up_sync(0xffffffffu, inc[c], o);
-      if (lane >= o) inc[c] += v;
+    for (int i = 0; i < NT; ++i) {
+      const uint32_t ki = order_key(s_thr[i]);
+      r += (ki < kv || (ki == kv && i < tid)) ? 1 : 0;
     }
-  }
-  if (lane == 31) {
-#pragma unroll
-    for (int c = 0; c < 9; ++c) s_wtot[c][warp] = inc[c];
+    s_sig[r] = v;
   }
   __syncthreads();
-  if (warp < ct.n) {
-    const int v = s_wtot[warp][lane];
+  float sig[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sig[i] = (i < NT) ? s_sig[i] : 0.0f;
+
+  if (NT > 0) {
+    int c[8] = {0, 0, 0, 0, 0, 0, 0, 0}, cb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    count_all<NT>(x, K, lo, sig, c, cb);
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      const int vb = __reduce_add_sync(0xffffffffu, cb[i]);
+      const int vt = __reduce_add_sync(0xffffffffu, c[i]);
+      if (lane == 0) {
+        if (vb) atomicAdd(&s_nge[0][i], vb);
+        if (vt) atomicAdd(&s_nge[1][i], vt);
+      }
+    }
+  }
+
+  int j[kSelRounds], rank[kSelRounds];
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int e = 0; e < kSelRounds; ++e) {
+    const int k = lo + e * kSelThreads + tid;
+    int jj = 0;
+    const float ax = abs_half(xo[e]);
+#pragma unroll
+    for (int i = 0; i < NT; ++i) jj += (ax >= sig[i]) ? 1 : 0;
+    j[e] = (k < hi) ? jj : kNoClass;
+    rank[e] = 0;
+    if (k < hi) bits[k] = s_width[jj];
+#pragma unroll
+    for (int cl = 0; cl < NC; ++cl) {
+      const uint32_t m = __ballot_sync(0xffffffffu, j[e] == cl);
+      if (lane == 0) s_cnt[cl][e * kSelWarps + warp] = __popc(m);
+      if (j[e] == cl) rank[e] = __popc(m & lt);
+    }
+  }
+  __syncthreads();
+  for (int cl = warp; cl < NC; cl += kSelWarps) {
+    const int v = s_cnt[cl][lane];
     int w = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int u = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += u;
     }
-    s_wtot[warp][lane] = w - v;
-    if (lane == 31) s_tot[warp] = w;
+    s_cnt[cl][lane] = w - v;
+    if (lane == 0) {
+      // #{class >= c} = #{|x| >= sigma_{c-1}}; channels of class < c precede class c
+      const int ge_b = (cl == 0) ? lo : s_nge[0][cl - 1];
+      const int ge_t = (cl == 0) ? K : s_nge[1][cl - 1];
+      const int nx_b = (cl < NT) ? s_nge[0][cl] : 0;
+      const int first = K - ge_t;
+      s_base[cl] = first + ge_b - nx_b;
+      if (blockIdx.x == 0) {
+        offsets[cl] = first;
+        if (cl == NC - 1) offsets[NC] = K;
+      }
+    }
   }
   __syncthreads();
-  if (tid == 0) {
-    int acc = 0;
-    for (int c = 0; c < ct.n; ++c) { s_off[c] = acc; acc += s_tot[c]; }
-    s_off[ct.n] = acc;
+#pragma unroll
+  for (int e = 0; e < kSelRounds; ++e) {
+    if (j[e] != kNoClass) {
+      const int k = lo + e * kSelThreads + tid;
+      idx[s_base[j[e]] + s_cnt[j[e]][e * kSelWarps + warp] + rank[e]] = k;
+    }
   }
-  __syncthreads();
-  if (tid <= ct.n) offsets[tid] = s_off[tid];
+}
 
-  int slot[9];
-#pragma unroll
-  for (int c = 0; c < 9; ++c) slot[c] = (c < ct.n) ? s_off[c] + s_wtot[c][warp] + inc[c] - cnt[c] : 0;
-  for (int k = k0; k < k1; ++k) {
-    const int j = grade_one(x[k], thr, n);
-#pragma unroll
-    for (int c = 0; c < 9; ++c)
-      if (j == c) idx[slot[c]++] = k;
-  }
+template <int NT>
+static cudaError_t launch_select_nt(const cudaLaunchConfig_t& cfg, const uint16_t* x, int K,
+                                    const float* thresholds, const ClassTable& ct, uint8_t* bits,
+                                    int32_t* idx, int32_t* offsets) {
+  return cudaLaunchKernelEx(&cfg, select_kernel<NT>, x, K, thresholds, ct, bits, idx, offsets);
 }
 
 cudaError_t launch_select(const uint16_t* x, int K, const float* thresholds, const ClassTable& ct,
                           uint8_t* bits, int32_t* idx, int32_t* offsets, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(1, 1, 1);
+  cfg.gridDim = dim3((unsigned)((K + kSelChunk - 1) / kSelChunk), 1, 1);
   cfg.blockDim = dim3(kSelThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
@@ -128,7 +231,18 @@ cudaError_t launch_select(const uint16_t* x, int K, const float* thresholds, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, select_kernel, x, K, thresholds, ct, bits, idx, offsets);
+  switch (ct.n - 1) {
+    case 0: return launch_select_nt<0>(cfg, x, K, thresholds, ct, bits, idx, offsets);
+    case 1: return launch_select_nt<1>(cfg, x, K, thresholds, ct, bits, idx, offsets);
+    case 2: return launch_select_nt<2>(cfg, x, K, thresholds, ct, bits, idx, offsets);
+    case 3: return launch_select_nt<3>(cfg, x, K, thresholds, ct, bits, idx, offsets);
+    case 4: return launch_select_nt<4>(cfg, x, K, thresholds, ct, bits, idx, offsets);
+    case 5: return launch_select_nt<5>(cfg, x, K, thresholds, ct, bits, idx, offsets);
+    case 6: return launch_select_nt<6>(cfg, x, K, thresholds, ct, bits, idx, offsets);
+    case 7: return launch_select_nt<7>(cfg, x, K, thresholds, ct, bits, idx, offsets);
+    case 8: return launch_select_nt<8>(cfg, x, K, thresholds, ct, bits, idx, offsets);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace grinqh

@@ -32,7 +32,9 @@
 // Arithmetic per row and thread. a = x_k * s is exact in fp32 (two 11-bit
 // significands). The b plane words are merged into 8 registers of 4 truncated
 // codes each (one LOP3 per plane plus one rotate, thanks to the bit order chosen
-// at pack time). Codes become floats without a per-code integer extraction:
+// at pack time); the merge enters one fall-through sequence at plane b-1, so
+// all widths share one copy of the code (separate copies per width overflow
+// the instruction cache). Codes become floats without a per-code integer extraction:
 // a byte-permute puts two codes c1:c0 in the low 16 bits of an otherwise zero
 // word, i.e. the subnormal float (256 c1 + c0) 2^-149; adding 2^-118 with
 // round-down leaves exactly 2^-118 + c1 2^-141, so one more subtraction gives
@@ -84,25 +86,57 @@ struct __align__(128) VmmSmem {
 static_assert(sizeof(float) * kLanes * kRedStride <= sizeof(uint8_t) * kLanes * kPairs * 2 * kRecordBytes,
               "reduction buffer must fit in the ring");
 
-// One row of one tile: rec = the record (scale/zero words, then the planes);
-// thread w owns plane word w, i.e. columns 32w..32w+31 of the tile.
-template <int B>
-__device__ __forceinline__ void row_fma(const uint8_t* __restrict__ rec, int w, float xk, float2 (&acc)[16],
-                                        float& cacc) {
-  const uint32_t m = reinterpret_cast<const uint32_t*>(rec)[w >> 2];
-  uint32_t P[8];
+// OR plane p's bits for every register j into T[j] (the pack-time bit order
+// puts them under the mask 0x01010101 << ((j + 7 - p) & 7)).
+template <int p>
+__device__ __forceinline__ void merge_plane(uint32_t P, uint32_t (&T)[8]) {
 #pragma unroll
-  for (int p = 0; p < 8; ++p)
-    P[p] = (p < B) ? reinterpret_cast<const uint32_t*>(rec + kMetaBytes + p * kPlaneBytes)[w] : 0u;
-  uint32_t R[8];
-  assemble<B>(P, R);
+  for (int j = 0; j < 8; ++j) T[j] |= P & (0x01010101u << ((j + 7 - p) & 7));
+}
+
+// Truncated codes of the 32 columns of plane word w of a row of width b (any
+// b in 0..8, chosen at run time): one entry point per width into a single
+// fall-through sequence, so every width shares one copy of the code. out[j]
+// byte i = top-b bits of column 4j+i, in place, low bits zero.
+__device__ __forceinline__ void assemble_row(const uint8_t* __restrict__ rec, int w, int b, uint32_t (&out)[8]) {
+  const uint32_t* pw = reinterpret_cast<const uint32_t*>(rec + kMetaBytes) + w;
+  uint32_t T[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) T[j] = 0u;
+  switch (b) {
+    case 8: merge_plane<7>(pw[7 * kWords], T);  // fall through
+    case 7: merge_plane<6>(pw[6 * kWords], T);  // fall through
+    case 6: merge_plane<5>(pw[5 * kWords], T);  // fall through
+    case 5: merge_plane<4>(pw[4 * kWords], T);  // fall through
+    case 4: merge_plane<3>(pw[3 * kWords], T);  // fall through
+    case 3: merge_plane<2>(pw[2 * kWords], T);  // fall through
+    case 2: merge_plane<1>(pw[1 * kWords], T);  // fall through
+    case 1: merge_plane<0>(pw[0], T);           // fall through
+    default: break;
+  }
+  out[0] = T[0];
+#pragma unroll
+  for (int j = 1; j < 8; ++j) out[j] = __funnelshift_r(T[j], T[j], j);
+}
+
+// Per-row coefficients: A0 = a 2^95 (for c_lo 2^-149), A1 = a 2^87 (for c_hi
+// 2^-141), and the row's constant a * (mid_b - z) added to cacc.
+__device__ __forceinline__ void row_coef(const uint8_t* __restrict__ rec, int w, int b, float xk, float& A0,
+                                         float& A1, float& cacc) {
+  // an absent row (b = 0) leaves its slot unfilled: select zeros, never multiply garbage
+  const uint32_t m = (b > 0) ? reinterpret_cast<const uint32_t*>(rec)[w >> 2] : 0u;
   const float s = half_bits_to_float(m);
   const float z = half_bits_to_float(m >> 16);
-  const float av = xk * s;                                   // exact
-  const float mid = (B >= 8) ? 0.0f : (float)(1 << (7 - B));
+  const float av = xk * s;                                      // exact
+  const float mid = (b < 8) ? __int_as_float((134 - b) << 23) : 0.0f;   // 2^(7-b)
   cacc = fmaf(av, mid - z, cacc);
-  const float2 A0 = make_float2(av * 0x1p95f, av * 0x1p95f);   // for c0 2^-149
-  const float2 A1 = make_float2(av * 0x1p87f, av * 0x1p87f);   // for c1 2^-141
+  A0 = av * 0x1p95f;
+  A1 = av * 0x1p87f;
+}
+
+// acc += codes * coefficients for the 32 columns held in R (one row).
+__device__ __forceinline__ void fma_codes(const uint32_t (&R)[8], float A0s, float A1s, float2 (&acc)[16]) {
+  const float2 A0 = make_float2(A0s, A0s), A1 = make_float2(A1s, A1s);
   const float2 M = make_float2(0x1p-118f, 0x1p-118f);
   const float2 NM = make_float2(-0x1p-118f, -0x1p-118f);
   const float2 NEG1 = make_float2(-1.0f, -1.0f);
@@ -119,28 +153,17 @@ __device__ __forceinline__ void row_fma(const uint8_t* __restrict__ rec, int w, 
   }
 }
 
-__device__ __forceinline__ void row_any(int b, const uint8_t* rec, int w, float xk, float2 (&acc)[16],
-                                        float& cacc) {
-  switch (b) {
-    case 1: row_fma<1>(rec, w, xk, acc, cacc); break;
-    case 2: row_fma<2>(rec, w, xk, acc, cacc); break;
-    case 3: row_fma<3>(rec, w, xk, acc, cacc); break;
-    case 4: row_fma<4>(rec, w, xk, acc, cacc); break;
-    case 5: row_fma<5>(rec, w, xk, acc, cacc); break;
-    case 6: row_fma<6>(rec, w, xk, acc, cacc); break;
-    case 7: row_fma<7>(rec, w, xk, acc, cacc); break;
-    case 8: row_fma<8>(rec, w, xk, acc, cacc); break;
-    default: break;
-  }
-}
-
-// Both rows of a slot; when they share a width the two rebuilds sit in one
-// basic block, so their independent chains interleave.
-template <int B>
-__device__ __forceinline__ void row_pair(const uint8_t* r0, const uint8_t* r1, int w, float x0, float x1,
-                                         float2 (&acc)[16], float& cacc) {
-  row_fma<B>(r0, w, x0, acc, cacc);
-  row_fma<B>(r1, w, x1, acc, cacc);
+// Both rows of a two-row slot (b = 0 marks an absent row, which adds nothing).
+__device__ __forceinline__ void pair_fma(const uint8_t* r0, const uint8_t* r1, int b0, int b1, float x0, float x1,
+                                         int w, float2 (&acc)[16], float& cacc) {
+  uint32_t R0[8], R1[8];
+  assemble_row(r0, w, b0, R0);
+  assemble_row(r1, w, b1, R1);
+  float a00, a01, a10, a11;
+  row_coef(r0, w, b0, x0, a00, a01, cacc);
+  row_coef(r1, w, b1, x1, a10, a11, cacc);
+  fma_codes(R0, a00, a01, acc);
+  fma_codes(R1, a10, a11, acc);
 }
 
 // Lane 0 of row lane h: fetch this CTA's rows q0 and q0 + 16 (when < nq) into
@@ -227,24 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
       }
       const int b0 = (int)s.slot_b[h][d][0], b1 = (int)s.slot_b[h][d][1];
       const float x0 = s.slot_x[h][d][0], x1 = s.slot_x[h][d][1];
-      const uint8_t* r0 = s.ring[h][d][0];
-      const uint8_t* r1 = s.ring[h][d][1];
-      if (b0 == b1) {
-        switch (b0) {
-          case 1: row_pair<1>(r0, r1, w, x0, x1, acc, cacc); break;
-          case 2: row_pair<2>(r0, r1, w, x0, x1, acc, cacc); break;
-          case 3: row_pair<3>(r0, r1, w, x0, x1, acc, cacc); break;
-          case 4: row_pair<4>(r0, r1, w, x0, x1, acc, cacc); break;
-          case 5: row_pair<5>(r0, r1, w, x0, x1, acc, cacc); break;
-          case 6: row_pair<6>(r0, r1, w, x0, x1, acc, cacc); break;
-          case 7: row_pair<7>(r0, r1, w, x0, x1, acc, cacc); break;
-          case 8: row_pair<8>(r0, r1, w, x0, x1, acc, cacc); break;
-          default: break;
-        }
-      } else {
-        row_any(b0, r0, w, x0, acc, cacc);
-        row_any(b1, r1, w, x1, acc, cacc);
-      }
+      pair_fma(s.ring[h][d][0], s.ring[h][d][1], b0, b1, x0, x1, w, acc, cacc);
       __syncwarp();
       if (w == 0 && i + kPairs < npair) {
         issue_pair(s, a, t, h, d, h + 2 * kLanes * (i + kPairs), nq);
