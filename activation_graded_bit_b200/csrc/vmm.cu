@@ -12,41 +12,36 @@
 // width and only the first can be 0, so the rows to read form one contiguous
 // stretch of the list). CTA r of R takes every R-th row of that stretch, so
 // every CTA gets the same mix of widths: equal DRAM bytes and equal arithmetic
-// per CTA. While staging its rows a CTA also gathers each row's x_k, so the
-// main loop reads no global memory except the weights.
+// per CTA.
 //
-// Data movement (sm_100a). Each of the 16 warps is a "row lane" that takes
-// rows h, h+16, ... of its CTA, two at a time, and owns a private ring of 6
-// two-row slots in shared memory, each with its own mbarrier: 12 rows in
-// flight per warp. Lane 0 fetches a row with ONE 1-D TMA bulk copy
-// (cp.async.bulk, no tensor map, no multicast) of the record's scale/zero
-// words and top b planes, 32 + 128 b contiguous, sector-aligned bytes,
-// completing on the slot's mbarrier. On this part the time of such a copy is
-// set by the number of copies in flight, not by their size (64..512 B copies
-// cost the same), so the record layout keeps one copy per (row, tile) and the
-// tile at 1024 columns. TMA copies also bypass L1's miss tracking, which
-// per-thread copies of short scattered rows exhaust. The 32 threads of the warp
-// then rebuild both rows of the slot, one 32-bit plane word (32 columns) each;
-// two independent rows per wait double the instruction-level parallelism.
+// Data movement. Each of the 16 warps takes rows h, h+16, ... of its CTA. Lane
+// w of a warp owns columns 32w..32w+31 of the tile, so for a row of width b it
+// needs exactly one 32-bit word of each of planes 0..b-1 (word w: 128
+// contiguous bytes per plane across the warp, one coalesced request) and the
+// scale/zero word of its 128-column group. The lanes load those words straight
+// into registers with plain read-only loads, kDepth rows ahead of the one they
+// are rebuilding: a software pipeline in registers, with no shared-memory
+// staging and no barriers. On this part that reads scattered 300..1100-byte
+// rows faster than bulk (TMA) copies, whose completion rate per issuing warp,
+// not their size, limits the bandwidth for rows this short.
 //
 // Arithmetic per row and thread. a = x_k * s is exact in fp32 (two 11-bit
 // significands). The b plane words are merged into 8 registers of 4 truncated
 // codes each (one LOP3 per plane plus one rotate, thanks to the bit order chosen
 // at pack time); the merge enters one fall-through sequence at plane b-1, so
-// all widths share one copy of the code (separate copies per width overflow
-// the instruction cache). Codes become floats without a per-code integer extraction:
-// a byte-permute puts two codes c1:c0 in the low 16 bits of an otherwise zero
-// word, i.e. the subnormal float (256 c1 + c0) 2^-149; adding 2^-118 with
-// round-down leaves exactly 2^-118 + c1 2^-141, so one more subtraction gives
-// hi = c1 2^-141 and another gives lo = c0 2^-149, all exact and all on the FP32
-// pipe (B200 runs FFMA with subnormal operands at full rate, while byte
-// extraction would run on the half-rate integer pipe). The products use
-// coefficients a 2^95 and a 2^87, so the accumulators hold a * code * 2^-54
-// (no overflow for |a| <= 2^32, no precision loss for the sizes that matter).
-// The per-row constant a * (mid_b - z) goes to one scalar per thread, since
-// all 32 columns of a thread share one 128-column group.
+// all widths share one copy of the code. Codes become floats without a
+// per-code integer extraction: a byte-permute puts two codes c1:c0 in the low
+// 16 bits of an otherwise zero word, i.e. the subnormal float (256 c1 + c0)
+// 2^-149; adding 2^-118 with round-down leaves exactly 2^-118 + c1 2^-141, so
+// one more subtraction gives hi = c1 2^-141 and another gives lo = c0 2^-149,
+// all exact and all on the FP32 pipe (B200 runs FFMA with subnormal operands at
+// full rate, while byte extraction would run on the half-rate integer pipe).
+// The products use coefficients a 2^95 and a 2^87, so the accumulators hold a *
+// code * 2^-54 (no overflow for |a| <= 2^32, no precision loss for the sizes
+// that matter). The per-row constant a * (mid_b - z) goes to one scalar per
+// thread, since all 32 columns of a thread share one 128-column group.
 //
-// Reduction. The 16 row lanes of a CTA are summed in shared memory into one
+// Reduction. The 16 warps of a CTA are summed in shared memory into one
 // 1024-column partial, stored with plain coalesced stores into the workspace
 // as partial[r][column]. A second kernel, chained with programmatic dependent
 // launch, sums the R partials of every column in a fixed order and overwrites
@@ -66,25 +61,33 @@ namespace grinqh {
 constexpr int kWords = kTileN / 32;              // plane words per tile row (32)
 constexpr int kWarps = 16;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kLanes = kWarps;                   // row lanes (warps)
-constexpr int kPairs = 6;                        // two-row slots per row lane (12 rows in flight)
-constexpr int kIdxCap = 2048;                    // rows of a CTA staged per pass
+constexpr int kDepth = 6;                        // rows in flight per warp (register slots)
+constexpr int kIdxCap = 4096;                    // rows of a CTA staged per pass
 constexpr int kRedPitch = 33;                    // column c of word w at c*33 + w: conflict-free both ways
-constexpr int kRedStride = 32 * kRedPitch + 16;  // floats per row lane in the reduction buffer
+constexpr int kRedStride = 32 * kRedPitch + 16;  // floats per warp in the reduction buffer
 
-struct __align__(128) VmmSmem {
-  uint8_t ring[kLanes][kPairs][2][kRecordBytes];
-  uint64_t bar[kLanes][kPairs];                  // one mbarrier per two-row slot
-  uint32_t slot_b[kLanes][kPairs][2];            // widths of the rows in each slot (0: no row)
-  float slot_x[kLanes][kPairs][2];               // x_k of the rows in each slot
-  uint32_t rows[kIdxCap];                        // k | b << 24 of this CTA's rows, one pass
-  float rows_x[kIdxCap];                         // x_k of those rows
+struct __align__(16) VmmSmem {
+  union {
+    uint32_t rows[kIdxCap];                      // k | b << 24 of this CTA's rows, one pass
+    float red[kWarps * kRedStride];              // after the main loop: per-warp column sums
+  } u;
   int off[10];
   int width[9];
-  int abort;
 };
-static_assert(sizeof(float) * kLanes * kRedStride <= sizeof(uint8_t) * kLanes * kPairs * 2 * kRecordBytes,
-              "reduction buffer must fit in the ring");
+
+// One row in flight: this lane's scale/zero word, plane words and x_k.
+struct RowRegs {
+  uint32_t m;
+  uint32_t p[8];
+  uint32_t xh;
+};
+
+// Read-only load that skips L1 allocation (every weight word is read once).
+__device__ __forceinline__ uint32_t ld_stream(const void* ptr) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(ptr));
+  return v;
+}
 
 // OR plane p's bits for every register j into T[j] (the pack-time bit order
 // puts them under the mask 0x01010101 << ((j + 7 - p) & 7)).
@@ -94,42 +97,14 @@ __device__ __forceinline__ void merge_plane(uint32_t P, uint32_t (&T)[8]) {
   for (int j = 0; j < 8; ++j) T[j] |= P & (0x01010101u << ((j + 7 - p) & 7));
 }
 
-// Truncated codes of the 32 columns of plane word w of a row of width b (any
-// b in 0..8, chosen at run time): one entry point per width into a single
-// fall-through sequence, so every width shares one copy of the code. out[j]
-// byte i = top-b bits of column 4j+i, in place, low bits zero.
-__device__ __forceinline__ void assemble_row(const uint8_t* __restrict__ rec, int w, int b, uint32_t (&out)[8]) {
-  const uint32_t* pw = reinterpret_cast<const uint32_t*>(rec + kMetaBytes) + w;
-  uint32_t T[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) T[j] = 0u;
-  switch (b) {
-    case 8: merge_plane<7>(pw[7 * kWords], T);  // fall through
-    case 7: merge_plane<6>(pw[6 * kWords], T);  // fall through
-    case 6: merge_plane<5>(pw[5 * kWords], T);  // fall through
-    case 5: merge_plane<4>(pw[4 * kWords], T);  // fall through
-    case 4: merge_plane<3>(pw[3 * kWords], T);  // fall through
-    case 3: merge_plane<2>(pw[2 * kWords], T);  // fall through
-    case 2: merge_plane<1>(pw[1 * kWords], T);  // fall through
-    case 1: merge_plane<0>(pw[0], T);           // fall through
-    default: break;
-  }
-  out[0] = T[0];
-#pragma unroll
-  for (int j = 1; j < 8; ++j) out[j] = __funnelshift_r(T[j], T[j], j);
-}
-
 // Per-row coefficients: A0 = a 2^95 (for c_lo 2^-149), A1 = a 2^87 (for c_hi
 // 2^-141), and the row's constant a * (mid_b - z) added to cacc.
-__device__ __forceinline__ void row_coef(const uint8_t* __restrict__ rec, int w, int b, float xk, float& A0,
-                                         float& A1, float& cacc) {
-  // an absent row (b = 0) leaves its slot unfilled: select zeros, never multiply garbage
-  const uint32_t m = (b > 0) ? reinterpret_cast<const uint32_t*>(rec)[w >> 2] : 0u;
+__device__ __forceinline__ void row_coef(uint32_t m, int b, float xk, float& A0, float& A1, float& cacc) {
   const float s = half_bits_to_float(m);
   const float z = half_bits_to_float(m >> 16);
-  const float av = xk * s;                                      // exact
+  const float av = (b > 0) ? xk * s : 0.0f;                     // exact; absent row: 0
   const float mid = (b < 8) ? __int_as_float((134 - b) << 23) : 0.0f;   // 2^(7-b)
-  cacc = fmaf(av, mid - z, cacc);
+  cacc = (b > 0) ? fmaf(av, mid - z, cacc) : cacc;
   A0 = av * 0x1p95f;
   A1 = av * 0x1p87f;
 }
@@ -153,53 +128,60 @@ __device__ __forceinline__ void fma_codes(const uint32_t (&R)[8], float A0s, flo
   }
 }
 
-// Both rows of a two-row slot (b = 0 marks an absent row, which adds nothing).
-__device__ __forceinline__ void pair_fma(const uint8_t* r0, const uint8_t* r1, int b0, int b1, float x0, float x1,
-                                         int w, float2 (&acc)[16], float& cacc) {
-  uint32_t R0[8], R1[8];
-  assemble_row(r0, w, b0, R0);
-  assemble_row(r1, w, b1, R1);
-  float a00, a01, a10, a11;
-  row_coef(r0, w, b0, x0, a00, a01, cacc);
-  row_coef(r1, w, b1, x1, a10, a11, cacc);
-  fma_codes(R0, a00, a01, acc);
-  fma_codes(R1, a10, a11, acc);
+// Issue the loads of one row (k | b << 24) into r: the scale/zero word of this
+// lane's group, x_k (a broadcast 2-byte load) and word w of planes 0..b-1 of
+// the row's record (each a coalesced 128-byte request across the warp). The
+// plane loads are volatile so that none is hoisted out of its width test: a
+// narrow row must not read the planes it does not use.
+__device__ __forceinline__ void load_row(const VmmArgs& a, int t, uint32_t info, int w, RowRegs& r) {
+  const uint32_t k = info & 0xFFFFFFu, b = info >> 24;
+  const uint8_t* rec = a.packed + ((size_t)k * a.n_tiles + t) * kRecordBytes;
+  r.m = ld_stream(rec + 4 * (w >> 2));
+  r.xh = __ldg(a.x + k);
+  const uint8_t* pw = rec + kMetaBytes + 4 * w;
+#pragma unroll
+  for (int p = 0; p < 8; ++p)
+    if ((uint32_t)p < b) r.p[p] = ld_stream(pw + p * kPlaneBytes);
 }
 
-// Lane 0 of row lane h: fetch this CTA's rows q0 and q0 + 16 (when < nq) into
-// two-row slot d, one bulk copy per row completing on the slot's mbarrier.
-__device__ __forceinline__ void issue_pair(VmmSmem& s, const VmmArgs& a, int t, int h, int d, int q0, int nq) {
-  uint32_t bytes = 0;
-  uint32_t bb[2], kk[2];
+// Truncated codes of this lane's 32 columns for a row of width b (0..8, chosen
+// at run time): one entry point per width into a single fall-through sequence,
+// so every width shares one copy of the code. out[j] byte i = top-b bits of
+// column 4j+i, in place, low bits zero.
+__device__ __forceinline__ void assemble_row(const RowRegs& r, int b, uint32_t (&out)[8]) {
+  uint32_t T[8];
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const int q = q0 + kLanes * e;
-    const uint32_t info = (q < nq) ? s.rows[q] : 0u;
-    kk[e] = info & 0xFFFFFFu;
-    bb[e] = info >> 24;
-    s.slot_b[h][d][e] = bb[e];
-    s.slot_x[h][d][e] = (q < nq) ? s.rows_x[q] : 0.0f;
-    bytes += bb[e] ? (uint32_t)kMetaBytes + bb[e] * (uint32_t)kPlaneBytes : 0u;
+  for (int j = 0; j < 8; ++j) T[j] = 0u;
+  switch (b) {
+    case 8: merge_plane<7>(r.p[7], T);  // fall through
+    case 7: merge_plane<6>(r.p[6], T);  // fall through
+    case 6: merge_plane<5>(r.p[5], T);  // fall through
+    case 5: merge_plane<4>(r.p[4], T);  // fall through
+    case 4: merge_plane<3>(r.p[3], T);  // fall through
+    case 3: merge_plane<2>(r.p[2], T);  // fall through
+    case 2: merge_plane<1>(r.p[1], T);  // fall through
+    case 1: merge_plane<0>(r.p[0], T);  // fall through
+    default: break;
   }
-  mbar_arrive_expect_tx(&s.bar[h][d], bytes);
+  out[0] = T[0];
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    if (bb[e]) {
-      const uint8_t* src = a.packed + ((size_t)kk[e] * a.n_tiles + t) * kRecordBytes;
-      bulk_g2s(s.ring[h][d][e], src, (uint32_t)kMetaBytes + bb[e] * (uint32_t)kPlaneBytes, &s.bar[h][d]);
-    }
-  }
+  for (int j = 1; j < 8; ++j) out[j] = __funnelshift_r(T[j], T[j], j);
+}
+
+__device__ __forceinline__ void row_fma(const RowRegs& r, int b, float2 (&acc)[16], float& cacc) {
+  uint32_t R[8];
+  assemble_row(r, b, R);
+  float A0, A1;
+  row_coef(r.m, b, __half2float(__ushort_as_half((unsigned short)r.xh)), A0, A1, cacc);
+  fma_codes(R, A0, A1, acc);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];
   VmmSmem& s = *reinterpret_cast<VmmSmem*>(smem_raw);
-  const int tid = threadIdx.x, h = tid >> 5, w = tid & 31;   // row lane h = warp, word w = lane
+  const int tid = threadIdx.x, h = tid >> 5, w = tid & 31;   // warp h, word w = lane
   const int t = blockIdx.x, r = blockIdx.y, R = gridDim.y;
 
-  if (tid < kLanes * kPairs) mbar_init(&s.bar[tid / kPairs][tid % kPairs], 1);
-  if (tid == 0) s.abort = 0;
-  mbar_fence_init();
   pdl_wait();   // the selection and x may come from the kernel just before
   if (tid <= a.ct.n) s.off[tid] = a.offsets[tid];
 #pragma unroll
@@ -218,8 +200,6 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
   for (int c = 0; c < 16; ++c) acc[c] = make_float2(0.0f, 0.0f);
   float cacc = 0.0f;
 
-  int used = 0;     // two-row slots of this lane consumed so far (all passes): slot use index
-  int issued = 0;   // two-row slots of this lane fetched so far (lane 0's count)
   for (int qb = 0; qb < nq_total; qb += kIdxCap) {
     const int nq = min(kIdxCap, nq_total - qb);
     __syncthreads();
@@ -227,48 +207,32 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
       const int pos = a0 + r + R * (qb + e);
       int j = 0;
       for (int c = 1; c < n; ++c) j += (pos >= s.off[c]) ? 1 : 0;
-      const int k = a.idx[pos];
-      s.rows[e] = (uint32_t)k | ((uint32_t)s.width[j] << 24);
-      s.rows_x[e] = __half2float(__ushort_as_half(a.x[k]));
+      s.u.rows[e] = (uint32_t)a.idx[pos] | ((uint32_t)s.width[j] << 24);
     }
     __syncthreads();
-    // rows of this lane in the pass: q = h + 16 m; pair i holds m = 2i, 2i+1.
-    // Slot uses continue across passes through `used` so barrier phases stay in step.
-    const int nrow = (nq > h) ? (nq - h + kLanes - 1) / kLanes : 0;
-    const int npair = (nrow + 1) / 2;
-    if (w == 0 && !*(volatile int*)&s.abort)
-      for (; issued < used + min(kPairs, npair); ++issued)
-        issue_pair(s, a, t, h, issued % kPairs, h + 2 * kLanes * (issued - used), nq);
-    int i = 0;
+    // rows of this warp in the pass: q = h + 16 m, m = 0 .. nrow-1; row m lives
+    // in register slot m % kDepth from its loads until its arithmetic
+    const int nrow = (nq > h) ? (nq - h + kWarps - 1) / kWarps : 0;
+    RowRegs S[kDepth];
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d)
+      if (d < nrow) load_row(a, t, s.u.rows[h + kWarps * d], w, S[d]);
 #pragma unroll 1
-    for (; i < npair; ++i) {
-      const int u = used + i, d = u % kPairs;
-      if (*(volatile int*)&s.abort || !mbar_wait(&s.bar[h][d], (u / kPairs) & 1)) {
-        // a copy never completed: stop, report, and let the CTA finish cleanly
-        if (w == 0) { s.abort = 1; atomicOr(a.status, 1u); }
-        break;
-      }
-      const int b0 = (int)s.slot_b[h][d][0], b1 = (int)s.slot_b[h][d][1];
-      const float x0 = s.slot_x[h][d][0], x1 = s.slot_x[h][d][1];
-      pair_fma(s.ring[h][d][0], s.ring[h][d][1], b0, b1, x0, x1, w, acc, cacc);
-      __syncwarp();
-      if (w == 0 && i + kPairs < npair) {
-        issue_pair(s, a, t, h, d, h + 2 * kLanes * (i + kPairs), nq);
-        ++issued;
+    for (int m0 = 0; m0 < nrow; m0 += kDepth) {
+#pragma unroll
+      for (int d = 0; d < kDepth; ++d) {
+        const int m = m0 + d;
+        if (m < nrow) {
+          row_fma(S[d], (int)(s.u.rows[h + kWarps * m] >> 24), acc, cacc);
+          if (m + kDepth < nrow) load_row(a, t, s.u.rows[h + kWarps * (m + kDepth)], w, S[d]);
+        }
       }
     }
-    used += i;   // after an abort every later pass stops at i = 0, so passes stay uniform
   }
-  __syncthreads();
-  if (s.abort) {
-    // let every copy this lane issued land before the shared memory is reused
-    if (w == 0)
-      for (int u = used; u < issued; ++u) (void)mbar_wait(&s.bar[h][u % kPairs], (u / kPairs) & 1);
-    __syncthreads();
-  }
+  __syncthreads();   // every warp is done with the row list before it becomes the reduction buffer
 
-  // ---------------- CTA reduction over the 16 row lanes ----------------
-  float* red = reinterpret_cast<float*>(&s.ring[0][0][0][0]);
+  // ---------------- CTA reduction over the 16 warps ----------------
+  float* red = s.u.red;
   {
     float* dst = red + h * kRedStride + w;           // slot c*33 + w holds column 32w + c
 #pragma unroll
@@ -286,10 +250,10 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
   const int limit = (R == 1) ? a.N : a.n_tiles * kTileN;
 #pragma unroll
   for (int e = tid; e < kTileN; e += kThreads) {
-    // column e of the tile sits at slot (e % 32) * 33 + e / 32 of every row lane
+    // column e of the tile sits at slot (e % 32) * 33 + e / 32 of every warp
     float v = 0.0f;
 #pragma unroll
-    for (int rl = 0; rl < kLanes; ++rl) v += red[rl * kRedStride + (e % kWords) * kRedPitch + e / kWords];
+    for (int rl = 0; rl < kWarps; ++rl) v += red[rl * kRedStride + (e % kWords) * kRedPitch + e / kWords];
     const int col = t * kTileN + e;
     if (col < limit) out[col] = v;
   }
