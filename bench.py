@@ -268,6 +268,13 @@ def run_gpu(args):
     h2d = sum(2 * pr["K"] for pr in groups[copies[0]])
     d2h = sum(4 * pr["N"] for pr in groups[copies[0]])
 
+    # select + vmm per pair, plus the partial-sum kernel when the layer has more
+    # than one row split (the workspace then holds R x n_tiles x 1024 partials)
+    launches_per_step = 0
+    for pr in groups[copies[0]]:
+        L = pr["packed"].layout
+        launches_per_step += 2 + (1 if pr["ws"].numel() > 16 + L.n_tiles * 4096 else 0)
+
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "vmm_traffic.json")
     if os.path.exists(tpath):
@@ -296,7 +303,7 @@ def run_gpu(args):
             "points": points,
             "e2e": {"value": round(e2e_us, 4), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 2 * n_pairs * args.steps,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }
         if cpu is not None:
@@ -404,8 +411,8 @@ def run_profile_case(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--copies", type=int, default=2)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
