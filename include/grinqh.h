@@ -203,9 +203,9 @@ grinqh_status grinqh_vmm_workspace_bytes(const grinqh_layout* layout, size_t* by
  *   workspace     device, >= grinqh_vmm_workspace_bytes(layout) (a size that
  *                 depends on the current device's SM count), 16-byte aligned;
  *                 its first 16 bytes must be zero-filled once before first use.
- *                 They hold a sticky status word: 0, or nonzero if a bounded
- *                 wait inside the kernel gave up (the output of that call is
- *                 then invalid; clear the word before reusing). The rest holds
+ *                 They hold a status word that stays 0 (reserved: the kernels
+ *                 of this version contain no wait that can time out; a nonzero
+ *                 word would mean the call's output is invalid). The rest holds
  *                 per-CTA partial sums of y, fully rewritten by every call.
  *                 Calls that share a workspace must not overlap in time.
  * y is written with plain stores in a fixed summation order, so repeated calls
