@@ -246,4 +246,30 @@ grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* packed, const 
   return cuda_status(launch_vmm(a, (cudaStream_t)stream));
 }
 
+grinqh_status grinqh_vmm_noalloc(const grinqh_layout* layout, const void* packed, const uint16_t* x,
+                                 const int32_t* idx, const int32_t* offsets, const uint8_t* classes,
+                                 int32_t n_classes, float* y, void* stream) {
+  if (!layout_ok(layout) || !valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
+  if (!packed || !x || !idx || !offsets || !y) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(x, 2) || !aligned(idx, 4) || !aligned(offsets, 4) || !aligned(y, 4))
+    return GRINQH_ERR_ALIGNMENT;
+  const grinqh_layout& L = *layout;
+  if (vmm_workspace_bytes(L.n_tiles, L.tile_n) > vmm_noalloc_scratch_bytes()) return GRINQH_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (vmm_noalloc_scratch(&scratch) != cudaSuccess) return GRINQH_ERR_CUDA;
+  VmmArgs a{};
+  a.K = L.K;
+  a.N = L.N;
+  a.n_tiles = L.n_tiles;
+  a.packed = (const uint8_t*)packed;
+  a.x = x;
+  a.idx = idx;
+  a.offsets = offsets;
+  a.y = y;
+  a.status = (uint32_t*)scratch;
+  a.partial = (float*)((char*)scratch + 16);
+  a.ct = table(classes, n_classes);
+  return cuda_status(launch_vmm(a, (cudaStream_t)stream));
+}
+
 }  // extern "C"

@@ -35,6 +35,11 @@ struct VmmArgs {
 size_t vmm_workspace_bytes(int n_tiles, int tile_n);
 cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st);
 
+// grinqh_vmm_noalloc's shared device scratch: its size, and its address on the
+// current device.
+size_t vmm_noalloc_scratch_bytes();
+cudaError_t vmm_noalloc_scratch(void** ptr);
+
 // Calibration: per-sample order statistics, then the fixed-order mean.
 struct CalibArgs {
   const uint16_t* X;

@@ -51,6 +51,7 @@
 // y directly and no second kernel runs.
 #include <cstdint>
 #include <cuda_fp16.h>
+#include <mutex>
 
 #include "async.cuh"
 #include "common.cuh"
@@ -336,6 +337,39 @@ cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st) {
   rc.numAttrs = 1;
   return cudaLaunchKernelEx(&rc, reduce_partials_kernel, (const float*)a.partial, R, a.n_tiles * kTileN, a.y,
                             a.N);
+}
+
+// ---------------------------------------------------------------------------
+// Scratch of grinqh_vmm_noalloc: one file-scope device array, shared by every
+// call of that entry point on a device. Layout as a caller's workspace: the
+// 16-byte status word (zero from module load, like every static device
+// variable; this version never sets it), then the partials [R][n_tiles * 1024],
+// which every call rewrites completely. Calls that overlap on the GPU race on
+// the partials.
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;   // 1 MiB
+static __device__ __align__(256) uint8_t g_vmm_scratch[kNoAllocScratchBytes];
+
+size_t vmm_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// The scratch's device address on the current device, looked up once per
+// device (with that device current) and remembered.
+cudaError_t vmm_noalloc_scratch(void** ptr) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_vmm_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace grinqh

@@ -64,11 +64,13 @@ _calibrate = _sig("grinqh_calibrate", [_P, _I, _I, _P, _I, _P, ctypes.c_double, 
 _select = _sig("grinqh_select", [_P, _I, _P, _P, _I, _P, _P, _P, _P])
 _vmm_ws = _sig("grinqh_vmm_workspace_bytes", [_LP, ctypes.POINTER(ctypes.c_size_t)])
 _vmm = _sig("grinqh_vmm", [_LP, _P, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
+_vmm_noalloc = _sig("grinqh_vmm_noalloc", [_LP, _P, _P, _P, _P, _P, _I, _P, _P])
 
 # Every exported symbol of the C ABI, for the export check in the tests.
 EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grinqh_pack",
            "grinqh_unpack_codes", "grinqh_maxent_distribution", "grinqh_calibrate_workspace_bytes",
-           "grinqh_calibrate", "grinqh_select", "grinqh_vmm_workspace_bytes", "grinqh_vmm")
+           "grinqh_calibrate", "grinqh_select", "grinqh_vmm_workspace_bytes", "grinqh_vmm",
+           "grinqh_vmm_noalloc")
 
 
 def version() -> str:
@@ -221,4 +223,13 @@ def vmm(p: PackedLayer, x: torch.Tensor, sel: Selection, workspace: torch.Tensor
     _check(_vmm(ctypes.byref(p.layout), _ptr(p.packed), _ptr(x), _ptr(sel.idx), _ptr(sel.offsets),
                 ctypes.addressof(cb), n, _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),
                 _stream(stream)), "grinqh_vmm")
+    return y
+
+
+def vmm_noalloc(p: PackedLayer, x: torch.Tensor, sel: Selection, y: torch.Tensor, stream=None) -> torch.Tensor:
+    """grinqh_vmm_noalloc: as vmm, with the library's shared static scratch instead of a
+    workspace; y (fp32 [N] CUDA tensor) must be given, since this call allocates nothing."""
+    cb, n = _classes_buf(sel.classes)
+    _check(_vmm_noalloc(ctypes.byref(p.layout), _ptr(p.packed), _ptr(x), _ptr(sel.idx), _ptr(sel.offsets),
+                        ctypes.addressof(cb), n, _ptr(y), _stream(stream)), "grinqh_vmm_noalloc")
     return y

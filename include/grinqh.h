@@ -217,6 +217,32 @@ grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* packed,
                          const uint8_t* classes, int32_t n_classes, float* y, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/*
+ * grinqh_vmm without a caller-provided workspace. The paper has no counterpart:
+ * this is a calling convention of the library, not a step of the method.
+ * It computes exactly what grinqh_vmm computes (same kernels, same summation
+ * order, so the same bits of y) but takes its scratch (status word and per-CTA
+ * partial sums) from one static device array of 1 MiB inside the library,
+ * and allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ * routine. It is for callers that have no device allocator to hand a workspace
+ * from: a plain C host that links only this library and the CUDA runtime, or a
+ * process that reserves all device memory up front for a fixed pool, where an
+ * allocation at call time could fail or fragment the pool.
+ *   Arguments as grinqh_vmm, without workspace and workspace_bytes.
+ * The scratch is shared by every call on a device: calls of this entry point
+ * that overlap on the GPU (e.g. on two streams at once) race on it and give
+ * undefined y. Its 16-byte status word starts at zero when the library's
+ * device code is loaded and stays zero in this version; the partial sums need
+ * no clearing.
+ * Limit: a layout whose grinqh_vmm_workspace_bytes exceeds 1 MiB is rejected
+ * with GRINQH_ERR_WORKSPACE (on a 148-SM B200 every layout fits: at most 148
+ * row splits x column tiles of 4 KiB each).
+ * Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, CUDA.
+ */
+grinqh_status grinqh_vmm_noalloc(const grinqh_layout* layout, const void* packed,
+                                 const uint16_t* x, const int32_t* idx, const int32_t* offsets,
+                                 const uint8_t* classes, int32_t n_classes, float* y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
