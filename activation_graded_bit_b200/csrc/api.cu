@@ -272,4 +272,30 @@ grinqh_status grinqh_vmm_noalloc(const grinqh_layout* layout, const void* packed
   return cuda_status(launch_vmm(a, (cudaStream_t)stream));
 }
 
+grinqh_status grinqh_select_vmm(const grinqh_layout* layout, const void* packed, const uint16_t* x,
+                                const float* thresholds, const uint8_t* classes, int32_t n_classes, float* y,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!layout_ok(layout) || !valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
+  if (!packed || !x || !y || (n_classes > 1 && !thresholds)) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(x, 2) || !aligned(y, 4) || (thresholds && !aligned(thresholds, 4)))
+    return GRINQH_ERR_ALIGNMENT;
+  const grinqh_layout& L = *layout;
+  if (L.K > vmm_fused_max_k()) return GRINQH_ERR_UNSUPPORTED;
+  const size_t need = vmm_workspace_bytes(L.n_tiles, L.tile_n);
+  if (!workspace || workspace_bytes < need) return GRINQH_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return GRINQH_ERR_ALIGNMENT;
+  VmmArgs a{};
+  a.K = L.K;
+  a.N = L.N;
+  a.n_tiles = L.n_tiles;
+  a.packed = (const uint8_t*)packed;
+  a.x = x;
+  a.thresholds = thresholds;
+  a.y = y;
+  a.status = (uint32_t*)workspace;
+  a.partial = (float*)((char*)workspace + 16);
+  a.ct = table(classes, n_classes);
+  return cuda_status(launch_vmm(a, (cudaStream_t)stream, true));
+}
+
 }  // extern "C"

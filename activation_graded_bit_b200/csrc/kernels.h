@@ -26,6 +26,7 @@ struct VmmArgs {
   const uint16_t* x;
   const int32_t* idx;
   const int32_t* offsets;
+  const float* thresholds;   // fused grading only: the n_classes - 1 thresholds
   float* y;
   uint32_t* status;     // workspace: sticky error word (bit 0: a bounded wait timed out)
   float* partial;       // workspace: per-row-split partial sums [R][n_tiles * 1024]
@@ -33,7 +34,10 @@ struct VmmArgs {
 };
 
 size_t vmm_workspace_bytes(int n_tiles, int tile_n);
-cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st);
+// fused = true: the kernel grades x itself (a.thresholds) instead of reading
+// a.idx / a.offsets; K <= vmm_fused_max_k().
+cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused = false);
+int vmm_fused_max_k();
 
 // grinqh_vmm_noalloc's shared device scratch: its size, and its address on the
 // current device.

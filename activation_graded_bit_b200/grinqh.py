@@ -65,12 +65,13 @@ _select = _sig("grinqh_select", [_P, _I, _P, _P, _I, _P, _P, _P, _P])
 _vmm_ws = _sig("grinqh_vmm_workspace_bytes", [_LP, ctypes.POINTER(ctypes.c_size_t)])
 _vmm = _sig("grinqh_vmm", [_LP, _P, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
 _vmm_noalloc = _sig("grinqh_vmm_noalloc", [_LP, _P, _P, _P, _P, _P, _I, _P, _P])
+_select_vmm = _sig("grinqh_select_vmm", [_LP, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
 
 # Every exported symbol of the C ABI, for the export check in the tests.
 EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grinqh_pack",
            "grinqh_unpack_codes", "grinqh_maxent_distribution", "grinqh_calibrate_workspace_bytes",
            "grinqh_calibrate", "grinqh_select", "grinqh_vmm_workspace_bytes", "grinqh_vmm",
-           "grinqh_vmm_noalloc")
+           "grinqh_vmm_noalloc", "grinqh_select_vmm")
 
 
 def version() -> str:
@@ -223,6 +224,18 @@ def vmm(p: PackedLayer, x: torch.Tensor, sel: Selection, workspace: torch.Tensor
     _check(_vmm(ctypes.byref(p.layout), _ptr(p.packed), _ptr(x), _ptr(sel.idx), _ptr(sel.offsets),
                 ctypes.addressof(cb), n, _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),
                 _stream(stream)), "grinqh_vmm")
+    return y
+
+
+def select_vmm(p: PackedLayer, x: torch.Tensor, thresholds: Optional[torch.Tensor], classes: Sequence[int],
+               workspace: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """grinqh_select_vmm: grading and the graded product in one call (K <= 16384)."""
+    if y is None:
+        y = torch.empty(p.N, dtype=torch.float32, device=p.packed.device)
+    cb, n = _classes_buf(classes)
+    _check(_select_vmm(ctypes.byref(p.layout), _ptr(p.packed), _ptr(x), _ptr(thresholds), ctypes.addressof(cb), n,
+                       _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+           "grinqh_select_vmm")
     return y
 
 

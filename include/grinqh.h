@@ -218,6 +218,27 @@ grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* packed,
                          size_t workspace_bytes, void* stream);
 
 /*
+ * Grading and the graded product in one call: the same y as grinqh_select
+ * followed by grinqh_vmm (the same rows in the same order, so the same bits),
+ * without the channel lists in memory.
+ * Paper: Section 3.1 (grading, "Dynamic Precision Assignment"), Fig. 2 and
+ * Section 3.3 (the graded product); the fusion is this library's: every CTA
+ * grades all K channels itself and stages the rows it will read, so no
+ * selection kernel, kernel boundary or channel-list read precedes the weights.
+ *   packed, classes, y, workspace, workspace_bytes   as grinqh_vmm (the same
+ *                workspace size, grinqh_vmm_workspace_bytes).
+ *   x            device fp16 [K], 2-byte aligned.
+ *   thresholds   device fp32 [n_classes - 1], 4-byte aligned (NULL allowed
+ *                when n_classes == 1); any order, NaN never reached.
+ * Limit: K <= 16384 (GRINQH_ERR_UNSUPPORTED above; use grinqh_select and
+ * grinqh_vmm there).
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+grinqh_status grinqh_select_vmm(const grinqh_layout* layout, const void* packed, const uint16_t* x,
+                                const float* thresholds, const uint8_t* classes, int32_t n_classes,
+                                float* y, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * grinqh_vmm without a caller-provided workspace. The paper has no counterpart:
  * this is a calling convention of the library, not a step of the method.
  * It computes exactly what grinqh_vmm computes (same kernels, same summation
