@@ -107,6 +107,26 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# replicas: every rank runs the whole workload on its own GPU (no exchange on
+# the data path); the job's time is the slowest rank's
+# ---------------------------------------------------------------------------
+def max_over_ranks(value, world, dist_mod=None, device="cpu"):
+    """The largest `value` over all ranks, on every rank (value itself when world == 1)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return float(t.item())
+
+
+def per_pair_us(ms_total, steps, pairs_per_step, world):
+    """Whole-job microseconds per select+VMM pair: the slowest rank's time for
+    `steps` steps over the pairs that all ranks processed in that time."""
+    return ms_total * 1e3 / (steps * pairs_per_step * world)
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 def build_workload(g, wl, torch, dev, copies=2):
@@ -229,11 +249,8 @@ def run_gpu(args):
             e1.record(stream)
         stream.synchronize()
         torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1)
+        ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
         if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
             dist.barrier()
         return ms
 
@@ -263,8 +280,8 @@ def run_gpu(args):
     us_pair = ms_step * 1e3 / (args.steps * n_pairs)
     us_vmm = ms_vmm * 1e3 / (args.steps * n_pairs)
     achieved = tot_alg * args.steps / (ms_vmm * 1e-3) / 1e9
-    value = ms_step * 1e3 / (args.steps * n_pairs * world)
-    e2e_us = ms_e2e * 1e3 / (args.steps * n_pairs * world)
+    value = per_pair_us(ms_step, args.steps, n_pairs, world)
+    e2e_us = per_pair_us(ms_e2e, args.steps, n_pairs, world)
     h2d = sum(2 * pr["K"] for pr in groups[copies[0]])
     d2h = sum(4 * pr["N"] for pr in groups[copies[0]])
 
