@@ -94,6 +94,14 @@ __device__ __forceinline__ uint32_t ld_stream(const void* ptr) {
   asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(ptr));
   return v;
 }
+// The same at a constant byte offset (folded into the instruction, so a row's
+// plane loads share one address register).
+template <int kOff>
+__device__ __forceinline__ uint32_t ld_stream_at(const void* ptr) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1+%2];" : "=r"(v) : "l"(ptr), "n"(kOff));
+  return v;
+}
 
 // OR plane p's bits for every register j into T[j] (the pack-time bit order
 // puts them under the mask 0x01010101 << ((j + 7 - p) & 7)).
@@ -137,17 +145,22 @@ __device__ __forceinline__ void fma_codes(const uint32_t (&R)[8], float A0s, flo
 // Issue the loads of one row (k | b << 24) into r: the scale/zero word of this
 // lane's group, x_k (a broadcast 2-byte load) and word w of planes 0..b-1 of
 // the row's record (each a coalesced 128-byte request across the warp). The
-// plane loads are volatile so that none is hoisted out of its width test: a
-// narrow row must not read the planes it does not use.
+// plane loads are volatile so that none is hoisted out of its case: a narrow
+// row must not read the planes it does not use.
 __device__ __forceinline__ void load_row(const VmmArgs& a, int t, uint32_t info, int w, RowRegs& r) {
   const uint32_t k = info & 0xFFFFFFu, b = info >> 24;
   const uint8_t* rec = a.packed + ((size_t)k * a.n_tiles + t) * kRecordBytes;
   r.m = ld_stream(rec + 4 * (w >> 2));
   r.xh = __ldg(a.x + k);
   const uint8_t* pw = rec + kMetaBytes + 4 * w;
-#pragma unroll
-  for (int p = 0; p < 8; ++p)
-    if ((uint32_t)p < b) r.p[p] = ld_stream(pw + p * kPlaneBytes);
+  if (b > 0) r.p[0] = ld_stream_at<0>(pw);
+  if (b > 1) r.p[1] = ld_stream_at<1 * kPlaneBytes>(pw);
+  if (b > 2) r.p[2] = ld_stream_at<2 * kPlaneBytes>(pw);
+  if (b > 3) r.p[3] = ld_stream_at<3 * kPlaneBytes>(pw);
+  if (b > 4) r.p[4] = ld_stream_at<4 * kPlaneBytes>(pw);
+  if (b > 5) r.p[5] = ld_stream_at<5 * kPlaneBytes>(pw);
+  if (b > 6) r.p[6] = ld_stream_at<6 * kPlaneBytes>(pw);
+  if (b > 7) r.p[7] = ld_stream_at<7 * kPlaneBytes>(pw);
 }
 
 // Truncated codes of this lane's 32 columns for a row of width b (0..8, chosen
