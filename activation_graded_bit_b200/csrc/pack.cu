@@ -77,15 +77,19 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ W, 
     reinterpret_cast<uint32_t*>(rec)[warp] = live ? ((uint32_t)sb | ((uint32_t)zb << 16)) : 0u;
   __syncthreads();
 
-  // thread -> (plane p, word w): 8 planes x 32 words for a 1024-column tile
-  const int p = threadIdx.x >> 5, w = threadIdx.x & 31;
+  // thread -> (pair s, word wi): 4 plane pairs x 64 words for a 1024-column
+  // tile; word wi is half wi & 1 of lane wi >> 1's 32 columns
+  const int sp = threadIdx.x >> 6, wi = threadIdx.x & 63;
+  const int cbase = 32 * (wi >> 1) + 16 * (wi & 1);
   uint32_t word = 0;
 #pragma unroll 8
   for (int L = 0; L < 32; ++L) {
-    const int c = 32 * w + col_at(p, L);
-    word |= (uint32_t)((codes[c] >> (7 - p)) & 1u) << L;
+    int c16, l;
+    pair_col_at(sp, L, c16, l);
+    const int p = 2 * sp + l;
+    word |= (uint32_t)((codes[cbase + c16] >> (7 - p)) & 1u) << L;
   }
-  reinterpret_cast<uint32_t*>(rec + kMetaBytes + p * kPlaneBytes)[w] = word;
+  reinterpret_cast<uint32_t*>(rec + kMetaBytes + sp * kPairBytes)[wi] = word;
 }
 
 // Decoder: one warp per (row, tile) record, 8 records per CTA.
@@ -93,8 +97,12 @@ template <int B>
 __device__ __forceinline__ void decode_word(const uint8_t* rec, int w, uint32_t (&R)[8]) {
   uint32_t P[8];
 #pragma unroll
-  for (int p = 0; p < 8; ++p)
-    P[p] = (p < B) ? reinterpret_cast<const uint32_t*>(rec + kMetaBytes + p * kPlaneBytes)[w] : 0u;
+  for (int s = 0; s < 4; ++s) {
+    const bool used = 2 * s < B;   // pair s holds planes 2s, 2s+1
+    const uint32_t* pw = reinterpret_cast<const uint32_t*>(rec + kMetaBytes + s * kPairBytes);
+    P[2 * s] = used ? pw[2 * w] : 0u;
+    P[2 * s + 1] = used ? pw[2 * w + 1] : 0u;
+  }
   assemble<B>(P, R);
   const uint32_t mid = midpoint_bytes(B);
 #pragma unroll

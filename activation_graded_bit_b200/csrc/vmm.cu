@@ -81,7 +81,8 @@ struct __align__(16) VmmSmem {
   uint32_t th2[8];                               // fused grading: sorted thresholds, fp16 in both halves
 };
 
-// One row in flight: this lane's scale/zero word, plane words and x_k.
+// One row in flight: this lane's scale/zero word, its two words of each plane
+// pair (p[2s], p[2s+1]) and x_k.
 struct RowRegs {
   uint32_t m;
   uint32_t p[8];
@@ -94,21 +95,11 @@ __device__ __forceinline__ uint32_t ld_stream(const void* ptr) {
   asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(ptr));
   return v;
 }
-// The same at a constant byte offset (folded into the instruction, so a row's
-// plane loads share one address register).
+// Two words at a constant byte offset (folded into the instruction, so a row's
+// plane-pair loads share one address register).
 template <int kOff>
-__device__ __forceinline__ uint32_t ld_stream_at(const void* ptr) {
-  uint32_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1+%2];" : "=r"(v) : "l"(ptr), "n"(kOff));
-  return v;
-}
-
-// OR plane p's bits for every register j into T[j] (the pack-time bit order
-// puts them under the mask 0x01010101 << ((j + 7 - p) & 7)).
-template <int p>
-__device__ __forceinline__ void merge_plane(uint32_t P, uint32_t (&T)[8]) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) T[j] |= P & (0x01010101u << ((j + 7 - p) & 7));
+__device__ __forceinline__ void ld_stream2_at(const void* ptr, uint32_t& lo, uint32_t& hi) {
+  asm volatile("ld.global.nc.L1::no_allocate.v2.b32 {%0, %1}, [%2+%3];" : "=r"(lo), "=r"(hi) : "l"(ptr), "n"(kOff));
 }
 
 // Per-row coefficients: A0 = a 2^95 (for c_lo 2^-149), A1 = a 2^87 (for c_hi
@@ -143,48 +134,48 @@ __device__ __forceinline__ void fma_codes(const uint32_t (&R)[8], float A0s, flo
 }
 
 // Issue the loads of one row (k | b << 24) into r: the scale/zero word of this
-// lane's group, x_k (a broadcast 2-byte load) and word w of planes 0..b-1 of
-// the row's record (each a coalesced 128-byte request across the warp). The
-// plane loads are volatile so that none is hoisted out of its case: a narrow
-// row must not read the planes it does not use.
+// lane's group, x_k (a broadcast 2-byte load) and this lane's two words of
+// plane pairs 0..ceil(b/2)-1 of the row's record (each an 8-byte load, a
+// coalesced 256-byte request across the warp). The loads are volatile so that
+// none is hoisted out of its width test: a narrow row must not read the pairs
+// it does not use.
 __device__ __forceinline__ void load_row(const VmmArgs& a, int t, uint32_t info, int w, RowRegs& r) {
   const uint32_t k = info & 0xFFFFFFu, b = info >> 24;
   const uint8_t* rec = a.packed + ((size_t)k * a.n_tiles + t) * kRecordBytes;
   r.m = ld_stream(rec + 4 * (w >> 2));
   r.xh = __ldg(a.x + k);
-  const uint8_t* pw = rec + kMetaBytes + 4 * w;
-  if (b > 0) r.p[0] = ld_stream_at<0>(pw);
-  if (b > 1) r.p[1] = ld_stream_at<1 * kPlaneBytes>(pw);
-  if (b > 2) r.p[2] = ld_stream_at<2 * kPlaneBytes>(pw);
-  if (b > 3) r.p[3] = ld_stream_at<3 * kPlaneBytes>(pw);
-  if (b > 4) r.p[4] = ld_stream_at<4 * kPlaneBytes>(pw);
-  if (b > 5) r.p[5] = ld_stream_at<5 * kPlaneBytes>(pw);
-  if (b > 6) r.p[6] = ld_stream_at<6 * kPlaneBytes>(pw);
-  if (b > 7) r.p[7] = ld_stream_at<7 * kPlaneBytes>(pw);
+  const uint8_t* pw = rec + kMetaBytes + 8 * w;   // this lane's two words of pair 0
+  if (b > 0) ld_stream2_at<0>(pw, r.p[0], r.p[1]);
+  if (b > 2) ld_stream2_at<1 * kPairBytes>(pw, r.p[2], r.p[3]);
+  if (b > 4) ld_stream2_at<2 * kPairBytes>(pw, r.p[4], r.p[5]);
+  if (b > 6) ld_stream2_at<3 * kPairBytes>(pw, r.p[6], r.p[7]);
 }
 
 // Truncated codes of this lane's 32 columns for a row of width b (0..8, chosen
-// at run time): one entry point per width into a single fall-through sequence,
-// so every width shares one copy of the code. out[j] byte i = top-b bits of
-// column 4j+i, in place, low bits zero.
+// at run time): the top plane of the last pair for odd b, then one entry point
+// per number of full pairs into a single fall-through sequence, so every width
+// shares one copy of the code. out[j] byte i = top-b bits of column 4j+i, in
+// place, low bits zero.
 __device__ __forceinline__ void assemble_row(const RowRegs& r, int b, uint32_t (&out)[8]) {
   uint32_t T[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) T[j] = 0u;
-  switch (b) {
-    case 8: merge_plane<7>(r.p[7], T);  // fall through
-    case 7: merge_plane<6>(r.p[6], T);  // fall through
-    case 6: merge_plane<5>(r.p[5], T);  // fall through
-    case 5: merge_plane<4>(r.p[4], T);  // fall through
-    case 4: merge_plane<3>(r.p[3], T);  // fall through
-    case 3: merge_plane<2>(r.p[2], T);  // fall through
-    case 2: merge_plane<1>(r.p[1], T);  // fall through
-    case 1: merge_plane<0>(r.p[0], T);  // fall through
+  if (b & 1) {
+    switch (b >> 1) {
+      case 0: merge_pair_top<0>(r.p[0], r.p[1], T); break;
+      case 1: merge_pair_top<1>(r.p[2], r.p[3], T); break;
+      case 2: merge_pair_top<2>(r.p[4], r.p[5], T); break;
+      default: merge_pair_top<3>(r.p[6], r.p[7], T); break;
+    }
+  }
+  switch (b >> 1) {
+    case 4: merge_pair<3>(r.p[6], r.p[7], T);  // fall through
+    case 3: merge_pair<2>(r.p[4], r.p[5], T);  // fall through
+    case 2: merge_pair<1>(r.p[2], r.p[3], T);  // fall through
+    case 1: merge_pair<0>(r.p[0], r.p[1], T);  // fall through
     default: break;
   }
-  out[0] = T[0];
-#pragma unroll
-  for (int j = 1; j < 8; ++j) out[j] = __funnelshift_r(T[j], T[j], j);
+  finish_codes(T, out);
 }
 
 __device__ __forceinline__ void row_fma(const RowRegs& r, int b, float2 (&acc)[16], float& cacc) {

@@ -62,14 +62,15 @@ typedef enum {
  * (k*n_tiles + t)*record_bytes (a row's tiles are adjacent):
  *   bytes [0, 32)      8 uint32 words; word g is scale_fp16 | (zero_fp16 << 16)
  *                      of columns [t*1024 + 128g, +128) (0 past the last group);
- *   bytes [32, 1056)   the 8 bit planes, MSB first: plane p (p = 0 is bit 7 of
- *                      the code, p = 7 is bit 0) fills bytes
- *                      [32 + 128p, 32 + 128(p+1)).
+ *   bytes [32, 1056)   the 8 bit planes, MSB first (plane p = 0 is bit 7 of the
+ *                      code, p = 7 is bit 0), in 4 plane pairs: pair s holds
+ *                      planes 2s and 2s+1 in bytes [32 + 256s, 32 + 256(s+1)).
  * So the scale/zero words and the top b planes of a (row, tile) are one
- * contiguous, 32-byte-aligned run of 32 + 128b bytes. Inside a plane, 32-bit
- * word w holds local columns 32w..32w+31; local column 32w + 4j + i (j in 0..7,
- * i in 0..3) sits at bit (8i + j + 7 - p) mod 32 of the word. Columns >= N are
- * zero bits.
+ * contiguous, 32-byte-aligned run of 32 + 256 ceil(b/2) bytes (for odd b the
+ * last pair's second plane is read and not used). Inside pair s, 32-bit word
+ * 2w holds local columns 32w..32w+15 and word 2w+1 columns 32w+16..32w+31; in
+ * either word, column 4j' + i of that half (j' in 0..3, i in 0..3) of plane
+ * 2s + l sits at bit (8i + 2j' + 7 - 2s - l) mod 32. Columns >= N are zero bits.
  */
 typedef struct {
   int32_t K;             /* input channels (rows) */
