@@ -29,14 +29,9 @@ constexpr int kPlaneBytes = kTileN / 8;               // one plane of one tile r
 constexpr int kPairBytes = 2 * kPlaneBytes;           // two planes of one tile row
 constexpr int kRecordBytes = kMetaBytes + kPlanes * kPlaneBytes;   // 1056 = 33 sectors of 32 B
 
-// Bit position, in a pair-s word, of local column c16 (0..15 inside the half)
-// of plane 2s + l.
-__host__ __device__ __forceinline__ int pair_bit(int s, int c16, int l) {
-  return (8 * (c16 & 3) + 2 * (c16 >> 2) + 7 - 2 * s - l) & 31;
-}
-
-// Inverse of pair_bit: the column (0..15 inside the half) and plane offset l
-// stored at bit L of a pair-s word.
+// The column (0..15 inside the half) and plane offset l stored at bit L of a
+// pair-s word (the inverse of the placement above: column 4j'+i of plane 2s+l
+// at bit (8i + 2j' + 7 - 2s - l) mod 32).
 __host__ __device__ __forceinline__ void pair_col_at(int s, int L, int& c16, int& l) {
   const int u = (L - 7 + 2 * s) & 31;   // 8i + 2j' - l (mod 32)
   l = u & 1;
