@@ -202,17 +202,34 @@ def run_gpu(args):
         for pr in groups[c]:
             g.vmm(pr["packed"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
 
-    # e2e: pinned host x in, host y out, per pair
-    for pr in pairs:
-        pr["x_pin"] = torch.from_numpy(pr["x_host"].view(np.int16).copy()).pin_memory()
-        pr["y_pin"] = torch.empty(pr["N"], dtype=torch.float32).pin_memory()
+    # e2e: a step's inputs come from pinned host memory in one copy and its
+    # outputs go back in one copy: every pair's x and y are views into one
+    # device buffer per step (offsets are multiples of 16 bytes)
+    io = {}
+    for c in copies:
+        grp = groups[c]
+        xs_dev = torch.empty(sum(pr["K"] for pr in grp), dtype=torch.int16, device=dev)
+        ys_dev = torch.empty(sum(pr["N"] for pr in grp), dtype=torch.float32, device=dev)
+        xo = yo = 0
+        for pr in grp:
+            xv = xs_dev[xo:xo + pr["K"]]
+            xv.copy_(pr["x"])
+            pr["x"] = xv
+            pr["y"] = ys_dev[yo:yo + pr["N"]]
+            xo += pr["K"]
+            yo += pr["N"]
+        xs_pin = torch.from_numpy(np.concatenate([pr["x_host"] for pr in grp]).view(np.int16).copy()).pin_memory()
+        ys_pin = torch.empty(ys_dev.numel(), dtype=torch.float32).pin_memory()
+        io[c] = (xs_dev, ys_dev, xs_pin, ys_pin)
+    torch.cuda.synchronize()
 
     def e2e_pairs(c):
+        xs_dev, ys_dev, xs_pin, ys_pin = io[c]
+        xs_dev.copy_(xs_pin, non_blocking=True)
         for pr in groups[c]:
-            pr["x"].copy_(pr["x_pin"], non_blocking=True)
             g.select(pr["x"], pr["th"], wl.CLASSES, out=pr["sel"], stream=stream)
             g.vmm(pr["packed"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
-            pr["y_pin"].copy_(pr["y"], non_blocking=True)
+        ys_pin.copy_(ys_dev, non_blocking=True)
 
     def capture(fn):
         graphs = {}
