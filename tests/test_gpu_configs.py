@@ -1,0 +1,105 @@
+"""Parity on the two remaining workload shapes, against the fp64 oracle
+("GRINQH" Section 3.1 grading, Fig. 2 / Section 3.3 graded product):
+
+- the average-bit sweep on a 14336 x 4096 down-proj-shaped layer: targets
+  0.5 .. 8 average bits, Gaussian and SiLU(a)*b activations;
+- a slice of the 32-layer Llama3-8B linear stack: per-layer thresholds for 3
+  average bits, fresh activations every decode step, select + VMM chained on
+  one stream for all seven linears of a layer.
+
+Columns are sampled (whole 128-column groups, always including the last) so
+the oracle finishes in seconds; thresholds, widths and channel lists are
+compared whole."""
+import numpy as np
+import pytest
+import torch
+
+from activation_graded_bit_b200 import workloads as wl
+from gpu_util import assert_close, dev_u16
+
+pytestmark = pytest.mark.gpu
+
+CL = (0, 2, 3, 4, 8)
+SWEEP = (0.5, 1.0, 2.0, 3.0, 4.0, 5.0, 6.0, 8.0)
+
+
+@pytest.fixture(scope="module")
+def g():
+    from activation_graded_bit_b200 import grinqh
+    return grinqh
+
+
+def _cols(N, rng, groups=3):
+    ng = (N + 127) // 128
+    gs = sorted(set(list(rng.choice(ng, groups, replace=False)) + [ng - 1]))
+    return np.concatenate([np.arange(128 * q, min(N, 128 * q + 128)) for q in gs])
+
+
+@pytest.mark.parametrize("dist", ["gaussian", "silu_gated"])
+def test_bit_sweep_down_proj(g, orc, dist):
+    K, N = 14336, 4096
+    W = wl.weights_gaussian(K, N, key=(3, 0))
+    gen = wl.activations_gaussian if dist == "gaussian" else wl.activations_silu_gated
+    Xc = gen(K, 128, key=(3, 1, dist == "gaussian"))
+    x = gen(K, 1, key=(3, 2, dist == "gaussian"))[0]
+    p = g.pack(torch.from_numpy(W).cuda())
+    cols = _cols(N, np.random.default_rng(3))
+    q, s, z = orc.rtn_quantize(W[:, cols])
+    ws = g.vmm_workspace(p.layout)
+    xd = dev_u16(x)
+    cl = np.array(CL, np.uint8)
+    means = []
+    for t in SWEEP:
+        P = orc.maxent_distribution(cl, t)
+        th = g.calibrate(dev_u16(Xc), CL, P=P)
+        th_ref = orc.thresholds(Xc, P)
+        assert np.array_equal(th.cpu().numpy(), th_ref), t
+        sel = g.select(xd, th, CL)
+        y = g.vmm(p, xd, sel, ws)
+        torch.cuda.synchronize()
+        bits, idx, off = orc.select(x, th_ref, cl)
+        assert np.array_equal(sel.bits.cpu().numpy(), bits), t
+        assert np.array_equal(sel.idx.cpu().numpy(), idx), t
+        yr, bound = orc.vmm(x, q, s, z, bits)
+        assert_close(y.cpu().numpy()[cols], yr, bound, "%s %.1f bits" % (dist, t))
+        means.append(bits.mean())
+    assert int(ws[:16].count_nonzero()) == 0
+    # more bits asked, more bits read (calibrated on the same distribution)
+    assert all(a <= b + 1e-9 for a, b in zip(means, means[1:])), means
+    assert means[-1] == 8.0
+
+
+def test_linear_stack_slice(g, orc):
+    """Two of the 32 layers, two decode steps, all seven linears per layer."""
+    cl = np.array(CL, np.uint8)
+    P = orc.maxent_distribution(cl, 3.0)
+    rng = np.random.default_rng(4)
+    stream = torch.cuda.Stream()
+    for layer in (0, 31):
+        layer_data = []
+        for li, (name, K, N) in enumerate(wl.LLAMA3_8B):
+            key = (4, layer, li)
+            W = wl.weights_gaussian(K, N, key=key + (0,))
+            Xc = wl.activations_outlier(K, 128, key=key + (1,), chan_key=key)
+            th_ref = orc.thresholds(Xc, P)
+            cols = _cols(N, rng, groups=2)
+            q, s, z = orc.rtn_quantize(W[:, cols])
+            p = g.pack(torch.from_numpy(W).cuda())
+            layer_data.append(dict(name=name, K=K, N=N, key=key, p=p, cols=cols, q=q, s=s, z=z,
+                                   th=g.calibrate(dev_u16(Xc), CL, P=P), th_ref=th_ref,
+                                   ws=g.vmm_workspace(p.layout)))
+        for step in range(2):
+            xs, ys = [], []
+            with torch.cuda.stream(stream):
+                for d in layer_data:
+                    x = wl.activations_outlier(d["K"], 1, key=d["key"] + (100 + step,), chan_key=d["key"])[0]
+                    xd = dev_u16(x)
+                    sel = g.select(xd, d["th"], CL, stream=stream)
+                    ys.append(g.vmm(d["p"], xd, sel, d["ws"], stream=stream))
+                    xs.append(x)
+            stream.synchronize()
+            for d, x, y in zip(layer_data, xs, ys):
+                assert np.array_equal(d["th"].cpu().numpy(), d["th_ref"])
+                bits, _, _ = orc.select(x, d["th_ref"], cl)
+                yr, bound = orc.vmm(x, d["q"], d["s"], d["z"], bits)
+                assert_close(y.cpu().numpy()[d["cols"]], yr, bound, "layer %d %s step %d" % (layer, d["name"], step))
