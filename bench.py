@@ -442,6 +442,165 @@ def run_profile_case(args):
     print("profile case %s @ %g bits: %d select+vmm calls" % (args.profile, args.bits, args.iters))
 
 
+
+# ---------------------------------------------------------------------------
+# extra measurements: the average-bit sweep and the 32-layer linear stack
+# ---------------------------------------------------------------------------
+def _graph_time_us(torch, stream, fn, reps, warmup=3):
+    """Mean microseconds of one fn(stream) call, replayed from a CUDA graph of
+    `reps` calls, timed with events on the stream (median of 5 replays)."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            fn(stream)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for _ in range(reps):
+                fn(stream)
+        gr.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(5):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            gr.replay()
+            e1.record(stream)
+            stream.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3 / reps)
+    del gr
+    return statistics.median(ts)
+
+
+def run_sweep(args):
+    """Average-bit sweep on a 14336x4096 layer: microseconds and effective GB/s
+    of the VMM (and of select+VMM) against the achieved mean width, Gaussian and
+    SiLU(a)*b activations, and a least-squares line t = a + b * mean_bits."""
+    import torch
+    from activation_graded_bit_b200 import grinqh as g
+    from activation_graded_bit_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    K, N = 14336, 4096
+    classes = wl.CLASSES
+    copies = []
+    for c in range(6):   # 6 x 60 MB: a replay of one point never finds the weights in L2
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(3_000_017 + c)
+        copies.append(g.pack(torch.randn(K, N, generator=gen, device=dev, dtype=torch.float32) * 0.02))
+    stream = torch.cuda.Stream(device=dev)
+    ws = g.vmm_workspace(copies[0].layout, dev)
+    y = torch.empty(N, dtype=torch.float32, device=dev)
+    peak, peak_kind = _peaks()
+    points = []
+    for dist in ("gaussian", "silu_gated"):
+        gen_x = wl.activations_gaussian if dist == "gaussian" else wl.activations_silu_gated
+        Xc = torch.from_numpy(gen_x(K, 128, key=(3, 1, dist == "gaussian")).view(np.int16)).to(dev)
+        x = torch.from_numpy(gen_x(K, 1, key=(3, 2, dist == "gaussian"))[0].view(np.int16)).to(dev)
+        for t in (0.5, 1.0, 2.0, 3.0, 4.0, 5.0, 6.0, 8.0):
+            th = g.calibrate(Xc, classes, target_bits=t)
+            sel = g.select(x, th, classes)
+            torch.cuda.synchronize()
+            bits = sel.bits.cpu().numpy().astype(np.int64)
+            active = int((bits > 0).sum())
+            alg = bits.sum() * N / 8.0 + 4.0 * ((N + 127) // 128) * active + 2.0 * K + 4.0 * active + 4.0 * N
+
+            def vmm_only(st, sel=sel):
+                for p in copies:
+                    g.vmm(p, x, sel, ws, y=y, stream=st)
+
+            def pair(st, sel=sel, th=th):
+                for p in copies:
+                    g.select(x, th, classes, out=sel, stream=st)
+                    g.vmm(p, x, sel, ws, y=y, stream=st)
+            tv = _graph_time_us(torch, stream, vmm_only, reps=8) / len(copies)
+            tp = _graph_time_us(torch, stream, pair, reps=8) / len(copies)
+            points.append(dict(dist=dist, target_bits=t, mean_bits=round(float(bits.mean()), 4),
+                               active_frac=round(active / K, 4), alg_bytes=int(alg), vmm_us=round(tv, 3),
+                               select_plus_vmm_us=round(tp, 3), gbs=round(alg / (tv * 1e-6) / 1e9, 1),
+                               frac=round(alg / (tv * 1e-6) / 1e9 / peak, 4)))
+    fits = {}
+    for dist in ("gaussian", "silu_gated"):
+        pts = [q for q in points if q["dist"] == dist]
+        xb = np.array([q["mean_bits"] for q in pts])
+        tt = np.array([q["vmm_us"] for q in pts])
+        slope, icpt = np.polyfit(xb, tt, 1)
+        pred = icpt + slope * xb
+        r2 = 1.0 - float(((tt - pred) ** 2).sum() / ((tt - tt.mean()) ** 2).sum())
+        fits[dist] = dict(us_per_bit=round(float(slope), 4), us_at_0_bits=round(float(icpt), 4), r2=round(r2, 5))
+    print(json.dumps({"metric": "vmm us and effective GB/s vs average bits (14336x4096 sweep)", "unit": UNIT,
+                      "higher_is_better": False, "data": "synthetic", "peak": peak, "peak_kind": peak_kind,
+                      "config": {"workload": "down-proj-shaped 14336x4096, classes %s, 6 packed copies rotated"
+                                 % (list(classes),)}, "points": points, "linear_fit": fits}))
+
+
+def run_stack(args):
+    """The 32-layer Llama3-8B linear stack (7 linears per layer), batch-1 decode
+    at 3 average bits: select + VMM for all 224 linears of a step chained on one
+    stream; tokens/s = steps / time. Activations rotate over 8 seeded sets (one
+    graph each): per layer one x for q/k/v, one for o, one for gate/up, one for
+    down."""
+    import torch
+    from activation_graded_bit_b200 import grinqh as g
+    from activation_graded_bit_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    classes = wl.CLASSES
+    n_layers, n_sets = 32, 8
+    src = {"q_proj": 0, "k_proj": 0, "v_proj": 0, "o_proj": 1, "gate_proj": 2, "up_proj": 2, "down_proj": 3}
+    lin = []
+    for layer in range(n_layers):
+        for li, (name, K, N) in enumerate(wl.LLAMA3_8B):
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(4_000_037 * (layer + 1) + li)
+            p = g.pack(torch.randn(K, N, generator=gen, device=dev, dtype=torch.float32) * 0.02)
+            Xc = wl.activations_outlier(K, 128, key=(4, layer, li, 1), chan_key=(4, layer, li))
+            th = g.calibrate(torch.from_numpy(Xc.view(np.int16)).to(dev), classes, target_bits=3.0)
+            lin.append(dict(layer=layer, name=name, K=K, N=N, p=p, th=th, sel=g.empty_selection(K, classes, dev),
+                            ws=g.vmm_workspace(p.layout, dev), y=torch.empty(N, dtype=torch.float32, device=dev)))
+    # x[set][layer][source]
+    xs = [[[torch.from_numpy(wl.activations_outlier(14336 if s == 3 else 4096, 1, key=(4, 9, k, layer, s),
+                                                    chan_key=(4, layer, 0))[0].view(np.int16)).to(dev)
+            for s in range(4)] for layer in range(n_layers)] for k in range(n_sets)]
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(st, k):
+        for d in lin:
+            x = xs[k][d["layer"]][src[d["name"]]]
+            g.select(x, d["th"], classes, out=d["sel"], stream=st)
+            g.vmm(d["p"], x, d["sel"], d["ws"], y=d["y"], stream=st)
+    graphs = []
+    with torch.cuda.stream(stream):
+        for k in range(n_sets):
+            step(stream, k)
+        torch.cuda.synchronize()
+        for k in range(n_sets):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                step(stream, k)
+            graphs.append(gr)
+        for i in range(max(args.warmup, 3)):
+            graphs[i % n_sets].replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.stack_steps):
+            graphs[i % n_sets].replay()
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1)
+    assert all(bool(torch.isfinite(d["y"]).all()) for d in lin[:7])
+    packed_gb = sum(d["p"].packed.numel() for d in lin) / 1e9
+    print(json.dumps({"metric": "linear-stack tokens/s (32 x 7 Llama3-8B linears, batch 1, 3 average bits)",
+                      "value": round(args.stack_steps / (ms * 1e-3), 2), "unit": "tokens/s", "higher_is_better": True,
+                      "steps": args.stack_steps, "warmup": max(args.warmup, 3), "ms_per_token": round(ms / args.stack_steps, 4),
+                      "data": "synthetic", "config": {"workload": "32-layer Llama3-8B linear stack, %.2f GB packed, "
+                                                      "8 activation sets rotated" % packed_gb},
+                      "gpu_launches_per_token": 2 * len(lin) + sum(1 for d in lin if d["ws"].numel() > 16)}))
+    del graphs
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -454,9 +613,18 @@ def main():
     ap.add_argument("--profile", default=None, help="linear name: run one small case for ncu and exit")
     ap.add_argument("--bits", type=float, default=4.0)
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--sweep", action="store_true", help="average-bit sweep on a 14336x4096 layer (one JSON line)")
+    ap.add_argument("--stack", action="store_true", help="32-layer linear stack tokens/s (one JSON line)")
+    ap.add_argument("--stack-steps", type=int, default=256)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.sweep:
+        run_sweep(args)
+        return
+    if args.stack:
+        run_stack(args)
+        return
     if args.profile:
         run_profile_case(args)
     elif args.impl == "reference":
