@@ -25,10 +25,13 @@
 // no shared-memory staging and no barriers. On this part that reads scattered
 // 300..1100-byte rows faster than bulk (TMA) copies, whose completion rate per
 // issuing warp, not their size, limits the bandwidth for rows this short. The
-// registers bound the pipeline at six rows, so the record prefixes of the next
-// kL2Ahead rows beyond it are requested into L2 (one 128-byte line per lane, no
-// register): their register loads then hit L2 instead of DRAM (measured 10%
-// faster on the 4096 x 14336 and 14336 x 4096 layers).
+// record prefixes of the kL2Ahead rows beyond the pipeline are requested into
+// L2 (one 128-byte line per lane, no register), so the register loads hit L2
+// instead of DRAM. With those requests a pipeline of three rows is enough, and
+// the registers it frees go to the compiler's scheduling (measured: 3 rows in
+// flight 13% faster than 6 on the 14336 x 4096 layer). Blocks of kDepth rows
+// whose loads and requests all exist run without per-row tests; the loads of
+// narrower rows are switched off by predicates, not branches.
 //
 // Arithmetic per row and thread. a = x_k * s is exact in fp32 (two 11-bit
 // significands). The plane pairs are merged into 8 registers of 4 truncated
@@ -67,7 +70,7 @@ namespace grinqh {
 constexpr int kWords = kTileN / 32;              // plane words per tile row (32)
 constexpr int kWarps = 16;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kDepth = 6;                        // rows in flight per warp (register slots)
+constexpr int kDepth = 3;                        // rows in flight per warp (register slots)
 constexpr int kL2Ahead = 3;                      // rows beyond those whose records are prefetched to L2
 constexpr int kIdxCap = 16384;                   // rows of a CTA staged per pass (64 KB)
 constexpr int kFusedMaxK = 32 * kThreads;        // fused grading: at most 32 channels per thread
@@ -111,15 +114,26 @@ template <int kOff>
 __device__ __forceinline__ void ld_stream2_at(const void* ptr, uint32_t& lo, uint32_t& hi) {
   asm volatile("ld.global.nc.L1::no_allocate.v2.b32 {%0, %1}, [%2+%3];" : "=r"(lo), "=r"(hi) : "l"(ptr), "n"(kOff));
 }
+// The same load under a predicate instead of a branch; when it is off the
+// registers keep what they held.
+template <int kOff>
+__device__ __forceinline__ void ld_stream2_at_if(bool on, const void* ptr, uint32_t& lo, uint32_t& hi) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %3, 0;\n\t"
+      "@p ld.global.nc.L1::no_allocate.v2.b32 {%0, %1}, [%2+%4];\n\t}"
+      : "+r"(lo), "+r"(hi)
+      : "l"(ptr), "r"((uint32_t)on), "n"(kOff));
+}
 
 // Per-row coefficients: A0 = a 2^95 (for c_lo 2^-149), A1 = a 2^87 (for c_hi
-// 2^-141), and the row's constant a * (mid_b - z) added to cacc.
+// 2^-141), and the row's constant a * (mid_b - z) added to cacc. Every row that
+// reaches the arithmetic has b >= 1 (the width-0 class is never staged).
 __device__ __forceinline__ void row_coef(uint32_t m, int b, float xk, float& A0, float& A1, float& cacc) {
   const float s = half_bits_to_float(m);
   const float z = half_bits_to_float(m >> 16);
-  const float av = (b > 0) ? xk * s : 0.0f;                     // exact; absent row: 0
+  const float av = xk * s;                                      // exact
   const float mid = (b < 8) ? __int_as_float((134 - b) << 23) : 0.0f;   // 2^(7-b)
-  cacc = (b > 0) ? fmaf(av, mid - z, cacc) : cacc;
+  cacc = fmaf(av, mid - z, cacc);
   A0 = av * 0x1p95f;
   A1 = av * 0x1p87f;
 }
@@ -143,57 +157,61 @@ __device__ __forceinline__ void fma_codes(const uint32_t (&R)[8], float A0s, flo
   }
 }
 
-// Issue the loads of one row (k | b << 24) into r: the scale/zero word of this
-// lane's group, x_k (a broadcast 2-byte load) and this lane's two words of
-// plane pairs 0..ceil(b/2)-1 of the row's record (each an 8-byte load, a
-// coalesced 256-byte request across the warp). The loads are volatile so that
-// none is hoisted out of its width test: a narrow row must not read the pairs
-// it does not use.
+// Issue the loads of one row (k | b << 24, b >= 1) into r: the scale/zero word
+// of this lane's group, x_k (a broadcast 2-byte load) and this lane's two words
+// of plane pairs 0..ceil(b/2)-1 of the row's record (each an 8-byte load, a
+// coalesced 256-byte request across the warp). Pairs 1..3 are loaded under a
+// predicate: a narrow row reads no pair it does not use, and no branch is taken.
 __device__ __forceinline__ void load_row(const VmmArgs& a, int t, uint32_t info, int w, RowRegs& r) {
   const uint32_t k = info & 0xFFFFFFu, b = info >> 24;
   const uint8_t* rec = a.packed + ((size_t)k * a.n_tiles + t) * kRecordBytes;
   r.m = ld_stream(rec + 4 * (w >> 2));
   r.xh = __ldg(a.x + k);
   const uint8_t* pw = rec + kMetaBytes + 8 * w;   // this lane's two words of pair 0
-  if (b > 0) ld_stream2_at<0>(pw, r.p[0], r.p[1]);
-  if (b > 2) ld_stream2_at<1 * kPairBytes>(pw, r.p[2], r.p[3]);
-  if (b > 4) ld_stream2_at<2 * kPairBytes>(pw, r.p[4], r.p[5]);
-  if (b > 6) ld_stream2_at<3 * kPairBytes>(pw, r.p[6], r.p[7]);
+  ld_stream2_at<0>(pw, r.p[0], r.p[1]);
+  ld_stream2_at_if<1 * kPairBytes>(b > 2, pw, r.p[2], r.p[3]);
+  ld_stream2_at_if<2 * kPairBytes>(b > 4, pw, r.p[4], r.p[5]);
+  ld_stream2_at_if<3 * kPairBytes>(b > 6, pw, r.p[6], r.p[7]);
 }
 
-// Truncated codes of this lane's 32 columns for a row of width b (0..8, chosen
-// at run time): the top plane of the last pair for odd b, then one entry point
-// per number of full pairs into a single fall-through sequence, so every width
-// shares one copy of the code. out[j] byte i = top-b bits of column 4j+i, in
-// place, low bits zero.
+// Truncated codes of this lane's 32 columns for a row of width b (1..8, chosen
+// at run time), with one indirect jump: the top plane of the last pair for odd
+// b, the full pair for even b, then the full pairs below it in one shared
+// sequence. out[j] byte i = top-b bits of column 4j+i, in place, low bits zero.
 __device__ __forceinline__ void assemble_row(const RowRegs& r, int b, uint32_t (&out)[8]) {
   uint32_t T[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) T[j] = 0u;
-  if (b & 1) {
-    switch (b >> 1) {
-      case 0: merge_pair_top<0>(r.p[0], r.p[1], T); break;
-      case 1: merge_pair_top<1>(r.p[2], r.p[3], T); break;
-      case 2: merge_pair_top<2>(r.p[4], r.p[5], T); break;
-      default: merge_pair_top<3>(r.p[6], r.p[7], T); break;
-    }
-  }
-  switch (b >> 1) {
-    case 4: merge_pair<3>(r.p[6], r.p[7], T);  // fall through
-    case 3: merge_pair<2>(r.p[4], r.p[5], T);  // fall through
-    case 2: merge_pair<1>(r.p[2], r.p[3], T);  // fall through
-    case 1: merge_pair<0>(r.p[0], r.p[1], T);  // fall through
-    default: break;
+  switch (b) {
+    case 8: merge_pair<3>(r.p[6], r.p[7], T); goto pairs3;
+    case 7: merge_pair_top<3>(r.p[6], r.p[7], T);  // fall through
+    case 6:
+    pairs3:
+      merge_pair<2>(r.p[4], r.p[5], T);
+      goto pairs2;
+    case 5: merge_pair_top<2>(r.p[4], r.p[5], T);  // fall through
+    case 4:
+    pairs2:
+      merge_pair<1>(r.p[2], r.p[3], T);
+      goto pairs1;
+    case 3: merge_pair_top<1>(r.p[2], r.p[3], T);  // fall through
+    case 2:
+    pairs1:
+      merge_pair<0>(r.p[0], r.p[1], T);
+      break;
+    default: merge_pair_top<0>(r.p[0], r.p[1], T); break;   // b == 1
   }
   finish_codes(T, out);
 }
 
-// Ask L2 for the record prefix of one row (k | b << 24): one 128-byte line per lane.
+// Ask L2 for the record prefix of one row (k | b << 24): one 128-byte line per
+// lane, issued under a predicate (no branch) for the lines inside the prefix.
 __device__ __forceinline__ void prefetch_row_l2(const VmmArgs& a, int t, uint32_t info, int w) {
   const uintptr_t rec = reinterpret_cast<uintptr_t>(a.packed) + ((size_t)(info & 0xFFFFFFu) * a.n_tiles + t) * kRecordBytes;
   const uint32_t bytes = kMetaBytes + kPairBytes * (((info >> 24) + 1) >> 1);
   const uintptr_t line = (rec & ~(uintptr_t)127) + 128u * (uint32_t)w;
-  if (line < rec + bytes) prefetch_l2(reinterpret_cast<const void*>(line));
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.lt.u64 p, %0, %1;\n\t@p prefetch.global.L2 [%0];\n\t}" ::"l"(line),
+               "l"(rec + bytes));
 }
 
 __device__ __forceinline__ void row_fma(const RowRegs& r, int b, float2 (&acc)[16], float& cacc) {
@@ -478,17 +496,32 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
       if (d < nrow) load_row(a, t, s.u.rows[h + kWarps * d], w, S[d]);
 #pragma unroll 1
     for (int m = kDepth; m < min(nrow, kDepth + kL2Ahead); ++m) prefetch_row_l2(a, t, s.u.rows[h + kWarps * m], w);
+    int m0 = 0;
+    // blocks whose loads and prefetches all exist: no per-row tests
 #pragma unroll 1
-    for (int m0 = 0; m0 < nrow; m0 += kDepth) {
+    for (; m0 + 2 * kDepth + kL2Ahead <= nrow; m0 += kDepth) {
+#pragma unroll
+      for (int d = 0; d < kDepth; ++d) {
+        const int m = m0 + d;
+        row_fma(S[d], (int)(s.u.rows[h + kWarps * m] >> 24), acc, cacc);
+        load_row(a, t, s.u.rows[h + kWarps * (m + kDepth)], w, S[d]);
+        // the record prefix of the row kL2Ahead rows further on goes to L2 now,
+        // one 128-byte line per lane, so its register loads later hit L2
+        prefetch_row_l2(a, t, s.u.rows[h + kWarps * (m + kDepth + kL2Ahead)], w);
+      }
+    }
+    // the last blocks, row by row: first the record prefixes of the rows that no
+    // block above sent to L2
+#pragma unroll 1
+    for (int m = m0 + kDepth + kL2Ahead; m < nrow; ++m) prefetch_row_l2(a, t, s.u.rows[h + kWarps * m], w);
+#pragma unroll 1
+    for (; m0 < nrow; m0 += kDepth) {
 #pragma unroll
       for (int d = 0; d < kDepth; ++d) {
         const int m = m0 + d;
         if (m < nrow) {
           row_fma(S[d], (int)(s.u.rows[h + kWarps * m] >> 24), acc, cacc);
           if (m + kDepth < nrow) load_row(a, t, s.u.rows[h + kWarps * (m + kDepth)], w, S[d]);
-          // the record prefix of the row kL2Ahead rows further on goes to L2 now,
-          // one 128-byte line per lane, so its register loads later hit L2
-          if (m + kDepth + kL2Ahead < nrow) prefetch_row_l2(a, t, s.u.rows[h + kWarps * (m + kDepth + kL2Ahead)], w);
         }
       }
     }
