@@ -73,7 +73,7 @@ constexpr int kThreads = 32 * kWarps;
 constexpr int kDepth = 3;                        // rows in flight per warp (register slots)
 constexpr int kL2Ahead = 3;                      // rows beyond those whose records are prefetched to L2
 constexpr int kIdxCap = 16384;                   // rows of a CTA staged per pass (64 KB)
-constexpr int kFusedMaxK = 32 * kThreads;        // fused grading: at most 32 channels per thread
+constexpr int kFusedMaxK = kIdxCap;              // fused grading: every CTA's rows fit one pass
 constexpr int kRedPitch = 33;                    // column c of word w at c*33 + w: conflict-free both ways
 constexpr int kRedStride = 32 * kRedPitch + 16;  // floats per warp in the reduction buffer
 
@@ -84,9 +84,7 @@ struct __align__(16) VmmSmem {
   } u;
   int off[10];
   int width[9];
-  unsigned long long wtot[kWarps][3];            // fused grading: per-warp class counts, then prefixes
-  unsigned long long ctot[3];                    // fused grading: class totals (16-bit fields)
-  uint32_t th2[8];                               // fused grading: sorted thresholds, fp16 in both halves
+  int wcnt[2][kWarps];                           // fused grading: rows kept per warp, two rounds
 };
 
 // One row in flight: this lane's scale/zero word, its two words of each plane
@@ -223,201 +221,55 @@ __device__ __forceinline__ void row_fma(const RowRegs& r, int b, float2 (&acc)[1
 }
 
 // ---------------------------------------------------------------------------
-// Fused grading (grinqh_select_vmm): every CTA grades all K channels itself and
-// stages its own rows, so no selection kernel, no kernel boundary and no
-// dependent loads of a channel list sit in front of the weights.
-
-// Total order for sorting the thresholds: -inf < ... < -0 == +0 < ... < +inf < NaN,
-// and its inverse (NaN maps back to a NaN, -0 to +0: the same comparisons).
-__device__ __forceinline__ uint32_t th_key(float v) {
-  if (v != v) return 0xFFFFFFFFu;
-  uint32_t u = __float_as_uint(v);
-  if (v == 0.0f) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float th_from_key(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
-
-// Position of the m-th (0-based) set bit of v (m < popc(v)): binary search on
-// popcounts of the low halves.
-__device__ __forceinline__ int nth_set_bit(uint32_t v, int m) {
-  int pos = 0;
-#pragma unroll
-  for (int w = 16; w >= 1; w >>= 1) {
-    const int c = __popc(v & ((1u << w) - 1u));
-    const bool up = m >= c;
-    m -= up ? c : 0;
-    v = up ? (v >> w) : v;
-    pos += up ? w : 0;
-  }
-  return pos;
-}
-
-// Thread t grades channels [t E, t E + E), E = ceil(K / 512) rounded up to
-// even (<= 32), two per fp16x2 compare, against the sorted thresholds
-// s_0 <= s_1 <= ...: bit e of ge[i] says |x| >= s_i for its e-th channel, so
-// class c is ge[c-1] & ~ge[c] (the class is a count of the thresholds reached,
-// which does not depend on their order; NaN reaches none).
-// A block scan of the class counts gives every channel its position in the
-// class-major, ascending-k list that grinqh_select writes, and the thread
-// stages the positions r + R e that belong to this CTA (past the width-0
-// class) as s.u.rows[e - e0].
-// Returns the number of rows of this CTA.
+// Fused grading (grinqh_select_vmm): CTA r of R grades the channels k = r,
+// r + R, r + 2R, ... itself (the class is the number of thresholds |x_k|
+// reaches, whatever their order; NaN reaches none) and stages those of nonzero
+// width in ascending k as s.u.rows (k | b << 24). Every CTA so gets every R-th
+// channel, a random mix of widths as with the list positions of grinqh_vmm, and
+// grades only its own K/R channels: no selection kernel, no kernel boundary, no
+// channel list and no grading repeated across CTAs. s.width must be filled.
+// Returns the number of rows staged (K <= kFusedMaxK = kIdxCap: one pass).
 __device__ __forceinline__ int stage_fused(const VmmArgs& a, VmmSmem& s, int r, int R) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int n = a.ct.n, nt = n - 1;
-  // x into shared memory (the row buffer is free until the rows are staged),
-  // 16 bytes at a time when x is 16-byte aligned; the loads go out first
-  uint16_t* xs = reinterpret_cast<uint16_t*>(s.u.rows);
-  if ((reinterpret_cast<uintptr_t>(a.x) & 15u) == 0) {
-    const int g8 = a.K >> 3;
-    for (int g = tid; g < g8; g += kThreads)
-      reinterpret_cast<uint4*>(xs)[g] = __ldg(reinterpret_cast<const uint4*>(a.x) + g);
-    for (int k = (g8 << 3) + tid; k < a.K; k += kThreads) xs[k] = __ldg(a.x + k);
-  } else {
-    for (int k = tid; k < a.K; k += kThreads) xs[k] = __ldg(a.x + k);
-  }
-  // thresholds, sorted, then rounded up to fp16: |x| is an fp16 value, so
-  // |x| >= s exactly when |x| >= ceil_fp16(s) (NaN stays NaN and is never
-  // reached; s <= 0 rounds to a value every non-NaN |x| reaches). Lane i of
-  // warp 0 places threshold i by its rank (ties broken by index).
-  if (warp == 0) {
-    const uint32_t kv = (lane < nt) ? th_key(__ldg(a.thresholds + lane)) : 0xFFFFFFFFu;
-    int rank = 0;
+  const int nt = a.ct.n - 1;
+  float th[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t ki = __shfl_sync(0xffffffffu, kv, i);
-      rank += (i < nt && (ki < kv || (ki == kv && i < lane))) ? 1 : 0;
-    }
-    if (lane < nt) {
-      const uint32_t hb = __half_as_ushort(__float2half_ru(th_from_key(kv)));
-      s.th2[rank] = hb | (hb << 16);
-    }
-  }
-  __syncthreads();
-  // this thread's channels [k0, k0 + cnt), an even count per thread, two per compare
-  const int E = (((a.K + kThreads - 1) / kThreads) + 1) & ~1;
-  const int k0 = min(a.K, tid * E);
-  const int cnt = min(a.K, k0 + E) - k0;
-  uint32_t t2[8];   // the sorted, rounded thresholds, in both halves
-#pragma unroll
-  for (int i = 0; i < 8; ++i) t2[i] = (i < nt) ? s.th2[i] : 0x7E007E00u;
-  uint32_t ge[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) ge[i] = 0u;
-#pragma unroll 2
-  for (int e = 0; e < cnt; e += 2) {
-    const uint32_t ax = *reinterpret_cast<const uint32_t*>(xs + k0 + e) & 0x7FFF7FFFu;
-    const uint32_t b0 = 1u << e, b1 = 2u << e;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i >= nt) break;
-      asm("{\n\t.reg .pred p, q;\n\tsetp.ge.f16x2 p|q, %1, %2;\n\t@p or.b32 %0, %0, %3;\n\t@q or.b32 %0, %0, %4;\n\t}"
-          : "+r"(ge[i])
-          : "r"(ax), "r"(t2[i]), "r"(b0), "r"(b1));
-    }
-  }
-  __syncthreads();   // x is no longer needed: the buffer takes the rows from here on
-  const uint32_t valid = (cnt >= 32) ? 0xFFFFFFFFu : ((1u << cnt) - 1u);
-  // class masks (class c = ge[c-1] & ~ge[c]) and their counts, packed four
-  // classes per 64-bit word in 16-bit fields (a CTA has at most 16384 channels)
-  uint32_t cm[9];
-  unsigned long long pk[3] = {0ull, 0ull, 0ull};
-#pragma unroll
-  for (int c = 0; c < 9; ++c) {
-    const uint32_t upper = (c == 0) ? valid : ge[(c - 1) & 7];
-    const uint32_t next = (c < nt) ? ge[c & 7] : 0u;
-    cm[c] = (c < n) ? (upper & ~next & valid) : 0u;
-    pk[c >> 2] |= (unsigned long long)__popc(cm[c]) << (16 * (c & 3));
-  }
-  unsigned long long inc[3] = {pk[0], pk[1], pk[2]};
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-#pragma unroll
-    for (int q = 0; q < 3; ++q) {
-      const unsigned long long u = __shfl_up_sync(0xffffffffu, inc[q], o);
-      if (lane >= o) inc[q] += u;
-    }
-  }
-  if (lane == 31) {
-#pragma unroll
-    for (int q = 0; q < 3; ++q) s.wtot[warp][q] = inc[q];
-  }
-  __syncthreads();
-  if (warp == 0) {
-    unsigned long long v[3], w2[3];
-#pragma unroll
-    for (int q = 0; q < 3; ++q) {
-      v[q] = (lane < kWarps) ? s.wtot[lane][q] : 0ull;
-      w2[q] = v[q];
-    }
-#pragma unroll
-    for (int o = 1; o < kWarps; o <<= 1) {
-#pragma unroll
-      for (int q = 0; q < 3; ++q) {
-        const unsigned long long u = __shfl_up_sync(0xffffffffu, w2[q], o);
-        if (lane >= o) w2[q] += u;
-      }
-    }
-    __syncwarp();
-    if (lane < kWarps) {
-#pragma unroll
-      for (int q = 0; q < 3; ++q) s.wtot[lane][q] = w2[q] - v[q];
-    }
-    if (lane == kWarps - 1) {
-#pragma unroll
-      for (int q = 0; q < 3; ++q) s.ctot[q] = w2[q];
-    }
-  }
-  __syncthreads();
-  unsigned long long pre[3];   // this thread's first position inside each class
-#pragma unroll
-  for (int q = 0; q < 3; ++q) pre[q] = s.wtot[warp][q] + inc[q] - pk[q];
-  // this CTA takes list positions r + R e; the width-0 class (if any) is the
-  // prefix of the list, e < e0, and is skipped; row q of this CTA is e = e0 + q
-  const int a0 = (s.width[0] == 0) ? (int)(s.ctot[0] & 0xFFFFull) : 0;
-  const int nfull = (a.K > r) ? (a.K - r + R - 1) / R : 0;
-  const int e0 = (a0 > r) ? (a0 - r + R - 1) / R : 0;
-  const int nq = nfull - e0;
-  const float rinv = 1.0f / (float)R;
-  // One compact loop over the classes (this code runs once per CTA, so its size,
-  // not its instruction count, sets its cost): this thread's first list
-  // position in class c (u0, counted from a0), the first of its class-c
-  // channels that falls to this CTA (offset d) and that row's index q.
-  uint32_t cml[9];
-#pragma unroll
-  for (int c = 0; c < 9; ++c) cml[c] = cm[c];
-  int first = 0;   // first list position of class c
+  for (int q = 0; q < 8; ++q) th[q] = (q < nt) ? __ldg(a.thresholds + q) : 0.0f;
+  const int nk = (a.K > r) ? (a.K - r + R - 1) / R : 0;
+  const uint32_t lt = (1u << lane) - 1u;
+  int base = 0;
 #pragma unroll 1
-  for (int c = 0; c < n; ++c) {
-    const int shift = 16 * (c & 3);
-    const int cc = (int)((pk[c >> 2] >> shift) & 0xFFFFull);
-    const int total = (int)((s.ctot[c >> 2] >> shift) & 0xFFFFull);
-    const int width = s.width[c];
-    if (width > 0 && cc > 0) {
-      const int u0 = first + (int)((pre[c >> 2] >> shift) & 0xFFFFull);   // list position
-      const int x = u0 - r;
-      int d = 0, q = 0;
-      if (x <= 0) {
-        d = -x;
-      } else {
-        int qq = __float2int_rz((float)x * rinv);   // exact up to one step for x < 2^24
-        int rem = x - qq * R;
-        if (rem < 0) { --qq; rem += R; }
-        if (rem >= R) { ++qq; rem -= R; }
-        d = rem ? R - rem : 0;
-        q = qq + (rem ? 1 : 0);
-      }
-      const uint32_t mk = cml[c];
-      const uint32_t wbits = (uint32_t)width << 24;
-      q -= e0;   // width > 0, so these positions are past the width-0 prefix
-      for (int m = d; m < cc; m += R) s.u.rows[q++] = (uint32_t)(k0 + nth_set_bit(mk, m)) | wbits;
+  for (int i0 = 0, rnd = 0; i0 < nk; i0 += kThreads, rnd ^= 1) {
+    const int i = i0 + tid;
+    uint32_t info = 0u;
+    bool keep = false;
+    if (i < nk) {
+      const int k = r + R * i;
+      const float ax = fabsf(__half2float(__ushort_as_half(__ldg(a.x + k))));
+      int c = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) c += (q < nt && ax >= th[q]) ? 1 : 0;
+      const int b = s.width[c];
+      keep = b > 0;
+      info = (uint32_t)k | ((uint32_t)b << 24);
     }
-    first += total;
+    // ascending k: warp by warp, lane by lane (rounds alternate their count
+    // buffer, so one barrier per round suffices)
+    const uint32_t m = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) s.wcnt[rnd][warp] = __popc(m);
+    __syncthreads();
+    int off = base;
+#pragma unroll
+    for (int q = 0; q < kWarps; ++q) {
+      const int cq = s.wcnt[rnd][q];
+      off += (q < warp) ? cq : 0;
+      base += cq;
+    }
+    if (keep) s.u.rows[off + __popc(m & lt)] = info;
   }
-  return nq;
+  return base;
 }
+
 
 template <bool kFused>
 __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {

@@ -202,6 +202,12 @@ def run_gpu(args):
         for pr in groups[c]:
             g.vmm(pr["packed"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
 
+    # the same graded products through the one-call entry point (grading inside
+    # the VMM kernel, no channel lists): reported beside the headline
+    def fused_pairs(c):
+        for pr in groups[c]:
+            g.select_vmm(pr["packed"], pr["x"], pr["th"], wl.CLASSES, pr["ws"], y=pr["y"], stream=stream)
+
     # e2e: a step's inputs come from pinned host memory in one copy and its
     # outputs go back in one copy: every pair's x and y are views into one
     # device buffer per step (offsets are multiples of 16 bytes)
@@ -248,6 +254,7 @@ def run_gpu(args):
     g_step = capture(step_pairs)
     g_vmm = capture(vmm_only)
     g_e2e = capture(e2e_pairs)
+    g_fused = capture(fused_pairs)
 
     def timed(graphs, steps, warmup):
         with torch.cuda.stream(stream):
@@ -277,6 +284,7 @@ def run_gpu(args):
     clocks = clk.summary()
     ms_vmm = timed(g_vmm, args.steps, args.warmup)
     ms_e2e = timed(g_e2e, args.steps, args.warmup)
+    ms_fused = timed(g_fused, args.steps, args.warmup)
 
     # correctness spot check of the timed path (one pair) before reporting
     torch.cuda.synchronize()
@@ -297,6 +305,8 @@ def run_gpu(args):
     us_pair = ms_step * 1e3 / (args.steps * n_pairs)
     us_vmm = ms_vmm * 1e3 / (args.steps * n_pairs)
     achieved = tot_alg * args.steps / (ms_vmm * 1e-3) / 1e9
+    us_fused = ms_fused * 1e3 / (args.steps * n_pairs)
+    achieved_fused = tot_alg * args.steps / (ms_fused * 1e-3) / 1e9
     value = per_pair_us(ms_step, args.steps, n_pairs, world)
     e2e_us = per_pair_us(ms_e2e, args.steps, n_pairs, world)
     h2d = sum(2 * pr["K"] for pr in groups[copies[0]])
@@ -331,6 +341,10 @@ def run_gpu(args):
                                  len(pairs), sum(pr["packed"].packed.numel() for pr in pairs) / 1e9),
                        "parallelism": "replicas only" if world > 1 else "single GPU"},
             "vmm_us": round(us_vmm, 4), "select_plus_vmm_us": round(us_pair, 4),
+            "select_vmm_fused": {"us": round(us_fused, 4), "achieved": round(achieved_fused, 1), "unit": "GB/s",
+                                 "frac": round(achieved_fused / peak, 4),
+                                 "what": "grinqh_select_vmm per (linear, width): grading inside the VMM "
+                                         "kernel, no channel lists, same y within the bound"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
                          "kernel": "grinqh vmm_kernel"},
@@ -513,11 +527,16 @@ def run_sweep(args):
                 for p in copies:
                     g.select(x, th, classes, out=sel, stream=st)
                     g.vmm(p, x, sel, ws, y=y, stream=st)
+            def fused(st, th=th):
+                for p in copies:
+                    g.select_vmm(p, x, th, classes, ws, y=y, stream=st)
             tv = _graph_time_us(torch, stream, vmm_only, reps=8) / len(copies)
             tp = _graph_time_us(torch, stream, pair, reps=8) / len(copies)
+            tf = _graph_time_us(torch, stream, fused, reps=8) / len(copies)
             points.append(dict(dist=dist, target_bits=t, mean_bits=round(float(bits.mean()), 4),
                                active_frac=round(active / K, 4), alg_bytes=int(alg), vmm_us=round(tv, 3),
-                               select_plus_vmm_us=round(tp, 3), gbs=round(alg / (tv * 1e-6) / 1e9, 1),
+                               select_plus_vmm_us=round(tp, 3), select_vmm_fused_us=round(tf, 3),
+                               gbs=round(alg / (tv * 1e-6) / 1e9, 1),
                                frac=round(alg / (tv * 1e-6) / 1e9 / peak, 4)))
     fits = {}
     for dist in ("gaussian", "silu_gated"):

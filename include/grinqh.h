@@ -219,13 +219,17 @@ grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* packed,
                          size_t workspace_bytes, void* stream);
 
 /*
- * Grading and the graded product in one call: the same y as grinqh_select
- * followed by grinqh_vmm (the same rows in the same order, so the same bits),
- * without the channel lists in memory.
+ * Grading and the graded product in one call: y = x . W_hat over the same
+ * graded rows as grinqh_select followed by grinqh_vmm (every channel gets the
+ * class and width grinqh_select gives it), without the channel lists in
+ * memory. The rows are summed in another order than grinqh_vmm's, so the two
+ * agree within fp32 rounding (both meet the same error bound), not bitwise;
+ * repeated calls on the same inputs give bitwise identical results.
  * Paper: Section 3.1 (grading, "Dynamic Precision Assignment"), Fig. 2 and
- * Section 3.3 (the graded product); the fusion is this library's: every CTA
- * grades all K channels itself and stages the rows it will read, so no
- * selection kernel, kernel boundary or channel-list read precedes the weights.
+ * Section 3.3 (the graded product); the fusion is this library's: the CTAs of
+ * row split r grade the channels k = r, r + R, r + 2R, ... themselves and read
+ * the rows of those with nonzero width, so no selection kernel, no kernel
+ * boundary and no channel-list read precede the weights.
  *   packed, classes, y, workspace, workspace_bytes   as grinqh_vmm (the same
  *                workspace size, grinqh_vmm_workspace_bytes).
  *   x            device fp16 [K], 2-byte aligned.
