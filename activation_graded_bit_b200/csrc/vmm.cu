@@ -93,7 +93,34 @@ struct RowRegs {
   uint32_t m;
   uint32_t p[8];
   uint32_t xh;
+  uint32_t b;
 };
+
+// Per-thread constants of the row addressing: a row's record starts at
+// packed + 32 * (k * n_tiles * 33 + t * 33) (records are 33 sectors of 32 B),
+// so one integer multiply-add gives its offset in sectors (below 2^32: a valid
+// layout has K * N <= 2^34, so K * n_tiles <= 2^25) and one wide multiply-add
+// each of this lane's addresses in it.
+struct RowAddr {
+  const uint8_t* meta;    // packed + this lane's scale/zero word within a record
+  const uint8_t* pairs;   // packed + this lane's two words of pair 0 within a record
+  const uint8_t* lines;   // packed + 128 * lane (the lane's L2 line within a record prefix)
+  uint32_t nt33, t33;     // sectors per row of records, sector offset of tile t
+  uint32_t lane128;       // 128 * lane
+};
+
+__device__ __forceinline__ RowAddr row_addr(const VmmArgs& a, int t, int w) {
+  constexpr uint32_t kSectors = kRecordBytes / 32;
+  static_assert(kRecordBytes % 32 == 0, "records are whole 32-byte sectors");
+  RowAddr ra;
+  ra.meta = a.packed + 4 * (w >> 2);
+  ra.pairs = a.packed + kMetaBytes + 8 * w;
+  ra.lines = a.packed + 128 * w;
+  ra.nt33 = (uint32_t)a.n_tiles * kSectors;
+  ra.t33 = (uint32_t)t * kSectors;
+  ra.lane128 = 128u * (uint32_t)w;
+  return ra;
+}
 
 // Ask L2 to fetch the cache line holding ptr (no register, no completion).
 __device__ __forceinline__ void prefetch_l2(const void* ptr) {
@@ -124,13 +151,12 @@ __device__ __forceinline__ void ld_stream2_at_if(bool on, const void* ptr, uint3
 }
 
 // Per-row coefficients: A0 = a 2^95 (for c_lo 2^-149), A1 = a 2^87 (for c_hi
-// 2^-141), and the row's constant a * (mid_b - z) added to cacc. Every row that
-// reaches the arithmetic has b >= 1 (the width-0 class is never staged).
-__device__ __forceinline__ void row_coef(uint32_t m, int b, float xk, float& A0, float& A1, float& cacc) {
+// 2^-141), and the row's constant a * (mid - z) added to cacc (mid = 2^(7-b)
+// for b < 8, 0 for b = 8).
+__device__ __forceinline__ void row_coef(uint32_t m, float mid, float xk, float& A0, float& A1, float& cacc) {
   const float s = half_bits_to_float(m);
   const float z = half_bits_to_float(m >> 16);
   const float av = xk * s;                                      // exact
-  const float mid = (b < 8) ? __int_as_float((134 - b) << 23) : 0.0f;   // 2^(7-b)
   cacc = fmaf(av, mid - z, cacc);
   A0 = av * 0x1p95f;
   A1 = av * 0x1p87f;
@@ -160,12 +186,14 @@ __device__ __forceinline__ void fma_codes(const uint32_t (&R)[8], float A0s, flo
 // of plane pairs 0..ceil(b/2)-1 of the row's record (each an 8-byte load, a
 // coalesced 256-byte request across the warp). Pairs 1..3 are loaded under a
 // predicate: a narrow row reads no pair it does not use, and no branch is taken.
-__device__ __forceinline__ void load_row(const VmmArgs& a, int t, uint32_t info, int w, RowRegs& r) {
+// Every row that reaches the loop has b >= 1 (the width-0 class is never staged).
+__device__ __forceinline__ void load_row(const VmmArgs& a, const RowAddr& ra, uint32_t info, RowRegs& r) {
   const uint32_t k = info & 0xFFFFFFu, b = info >> 24;
-  const uint8_t* rec = a.packed + ((size_t)k * a.n_tiles + t) * kRecordBytes;
-  r.m = ld_stream(rec + 4 * (w >> 2));
+  const uint32_t sec = k * ra.nt33 + ra.t33;                  // record offset in 32-byte sectors
+  r.b = b;
+  r.m = ld_stream(ra.meta + 32ull * sec);
   r.xh = __ldg(a.x + k);
-  const uint8_t* pw = rec + kMetaBytes + 8 * w;   // this lane's two words of pair 0
+  const uint8_t* pw = ra.pairs + 32ull * sec;                  // this lane's two words of pair 0
   ld_stream2_at<0>(pw, r.p[0], r.p[1]);
   ld_stream2_at_if<1 * kPairBytes>(b > 2, pw, r.p[2], r.p[3]);
   ld_stream2_at_if<2 * kPairBytes>(b > 4, pw, r.p[4], r.p[5]);
@@ -175,48 +203,55 @@ __device__ __forceinline__ void load_row(const VmmArgs& a, int t, uint32_t info,
 // Truncated codes of this lane's 32 columns for a row of width b (1..8, chosen
 // at run time), with one indirect jump: the top plane of the last pair for odd
 // b, the full pair for even b, then the full pairs below it in one shared
-// sequence. out[j] byte i = top-b bits of column 4j+i, in place, low bits zero.
-__device__ __forceinline__ void assemble_row(const RowRegs& r, int b, uint32_t (&out)[8]) {
+// sequence. out[j] byte i = top-b bits of column 4j+i, in place, low bits zero;
+// mid = the bin midpoint 2^(7-b) (0 for b = 8), fixed by the jump target.
+__device__ __forceinline__ void assemble_row(const RowRegs& r, uint32_t (&out)[8], float& mid) {
   uint32_t T[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) T[j] = 0u;
-  switch (b) {
-    case 8: merge_pair<3>(r.p[6], r.p[7], T); goto pairs3;
-    case 7: merge_pair_top<3>(r.p[6], r.p[7], T);  // fall through
+  switch (r.b) {
+    case 8: mid = 0.0f; merge_pair<3>(r.p[6], r.p[7], T); goto pairs3;
+    case 7: mid = 1.0f; merge_pair_top<3>(r.p[6], r.p[7], T); goto pairs3;
     case 6:
+      mid = 2.0f;
     pairs3:
       merge_pair<2>(r.p[4], r.p[5], T);
       goto pairs2;
-    case 5: merge_pair_top<2>(r.p[4], r.p[5], T);  // fall through
+    case 5: mid = 4.0f; merge_pair_top<2>(r.p[4], r.p[5], T); goto pairs2;
     case 4:
+      mid = 8.0f;
     pairs2:
       merge_pair<1>(r.p[2], r.p[3], T);
       goto pairs1;
-    case 3: merge_pair_top<1>(r.p[2], r.p[3], T);  // fall through
+    case 3: mid = 16.0f; merge_pair_top<1>(r.p[2], r.p[3], T); goto pairs1;
     case 2:
+      mid = 32.0f;
     pairs1:
       merge_pair<0>(r.p[0], r.p[1], T);
       break;
-    default: merge_pair_top<0>(r.p[0], r.p[1], T); break;   // b == 1
+    default: mid = 64.0f; merge_pair_top<0>(r.p[0], r.p[1], T); break;   // b == 1
   }
   finish_codes(T, out);
 }
 
-// Ask L2 for the record prefix of one row (k | b << 24): one 128-byte line per
-// lane, issued under a predicate (no branch) for the lines inside the prefix.
-__device__ __forceinline__ void prefetch_row_l2(const VmmArgs& a, int t, uint32_t info, int w) {
-  const uintptr_t rec = reinterpret_cast<uintptr_t>(a.packed) + ((size_t)(info & 0xFFFFFFu) * a.n_tiles + t) * kRecordBytes;
-  const uint32_t bytes = kMetaBytes + kPairBytes * (((info >> 24) + 1) >> 1);
-  const uintptr_t line = (rec & ~(uintptr_t)127) + 128u * (uint32_t)w;
-  asm volatile("{\n\t.reg .pred p;\n\tsetp.lt.u64 p, %0, %1;\n\t@p prefetch.global.L2 [%0];\n\t}" ::"l"(line),
-               "l"(rec + bytes));
+// Ask L2 for the record prefix of one row (k | b << 24): 32 + 256 ceil(b/2)
+// bytes from the record start, one 128-byte line per lane, issued under a
+// predicate (no branch) for the lines the prefix touches.
+__device__ __forceinline__ void prefetch_row_l2(const RowAddr& ra, uint32_t info) {
+  const uint32_t sec = (info & 0xFFFFFFu) * ra.nt33 + ra.t33;
+  const uint32_t bytes = kMetaBytes + 128u * (((info >> 24) + 1u) & ~1u);
+  const uint8_t* line = ra.lines + 128ull * (sec >> 2);      // the record's first line, plus this lane's
+  const uint32_t on = (ra.lane128 < 32u * (sec & 3u) + bytes) ? 1u : 0u;
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p prefetch.global.L2 [%0];\n\t}" ::"l"(line),
+               "r"(on));
 }
 
-__device__ __forceinline__ void row_fma(const RowRegs& r, int b, float2 (&acc)[16], float& cacc) {
+__device__ __forceinline__ void row_fma(const RowRegs& r, float2 (&acc)[16], float& cacc) {
   uint32_t R[8];
-  assemble_row(r, b, R);
+  float mid;
+  assemble_row(r, R, mid);
   float A0, A1;
-  row_coef(r.m, b, __half2float(__ushort_as_half((unsigned short)r.xh)), A0, A1, cacc);
+  row_coef(r.m, mid, __half2float(__ushort_as_half((unsigned short)r.xh)), A0, A1, cacc);
   fma_codes(R, A0, A1, acc);
 }
 
@@ -342,12 +377,13 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
     // rows of this warp in the pass: q = h + 16 m, m = 0 .. nrow-1; row m lives
     // in register slot m % kDepth from its loads until its arithmetic
     const int nrow = (nq > h) ? (nq - h + kWarps - 1) / kWarps : 0;
+    const RowAddr ra = row_addr(a, t, w);
     RowRegs S[kDepth];
 #pragma unroll
     for (int d = 0; d < kDepth; ++d)
-      if (d < nrow) load_row(a, t, s.u.rows[h + kWarps * d], w, S[d]);
+      if (d < nrow) load_row(a, ra, s.u.rows[h + kWarps * d], S[d]);
 #pragma unroll 1
-    for (int m = kDepth; m < min(nrow, kDepth + kL2Ahead); ++m) prefetch_row_l2(a, t, s.u.rows[h + kWarps * m], w);
+    for (int m = kDepth; m < min(nrow, kDepth + kL2Ahead); ++m) prefetch_row_l2(ra, s.u.rows[h + kWarps * m]);
     int m0 = 0;
     // blocks whose loads and prefetches all exist: no per-row tests
 #pragma unroll 1
@@ -355,25 +391,25 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
 #pragma unroll
       for (int d = 0; d < kDepth; ++d) {
         const int m = m0 + d;
-        row_fma(S[d], (int)(s.u.rows[h + kWarps * m] >> 24), acc, cacc);
-        load_row(a, t, s.u.rows[h + kWarps * (m + kDepth)], w, S[d]);
+        row_fma(S[d], acc, cacc);
+        load_row(a, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
         // the record prefix of the row kL2Ahead rows further on goes to L2 now,
         // one 128-byte line per lane, so its register loads later hit L2
-        prefetch_row_l2(a, t, s.u.rows[h + kWarps * (m + kDepth + kL2Ahead)], w);
+        prefetch_row_l2(ra, s.u.rows[h + kWarps * (m + kDepth + kL2Ahead)]);
       }
     }
     // the last blocks, row by row: first the record prefixes of the rows that no
     // block above sent to L2
 #pragma unroll 1
-    for (int m = m0 + kDepth + kL2Ahead; m < nrow; ++m) prefetch_row_l2(a, t, s.u.rows[h + kWarps * m], w);
+    for (int m = m0 + kDepth + kL2Ahead; m < nrow; ++m) prefetch_row_l2(ra, s.u.rows[h + kWarps * m]);
 #pragma unroll 1
     for (; m0 < nrow; m0 += kDepth) {
 #pragma unroll
       for (int d = 0; d < kDepth; ++d) {
         const int m = m0 + d;
         if (m < nrow) {
-          row_fma(S[d], (int)(s.u.rows[h + kWarps * m] >> 24), acc, cacc);
-          if (m + kDepth < nrow) load_row(a, t, s.u.rows[h + kWarps * (m + kDepth)], w, S[d]);
+          row_fma(S[d], acc, cacc);
+          if (m + kDepth < nrow) load_row(a, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
         }
       }
     }
