@@ -78,9 +78,9 @@ constexpr int kRedPitch = 33;                    // column c of word w at c*33 +
 constexpr int kRedStride = 32 * kRedPitch + 16;  // floats per warp in the reduction buffer
 
 struct __align__(16) VmmSmem {
-  union {
+  struct {
     uint32_t rows[kIdxCap];                      // k | b << 24 of this CTA's rows, one pass
-    float red[kWarps * kRedStride];              // after the main loop: per-warp column sums
+    float red[kWarps * kRedStride];              // per-warp column sums, written as each warp finishes
   } u;
   int off[10];
   int width[9];
@@ -414,9 +414,10 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
       }
     }
   }
-  __syncthreads();   // every warp is done with the row list before it becomes the reduction buffer
-
   // ---------------- CTA reduction over the 16 warps ----------------
+  // Each warp stores its column sums as soon as its own rows are done (the
+  // buffer is not shared with the row list), so only the slowest warp's
+  // stores and the final sum follow the barrier.
   float* red = s.u.red;
   {
     float* dst = red + h * kRedStride + w;           // slot c*33 + w holds column 32w + c
@@ -444,27 +445,39 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
   }
 }
 
-// y[col] = sum over r of partial[r][col]: 256 threads = 32 columns x 8 chains;
-// chain c adds r = c, c+8, ... in ascending order, then the 8 chains are added
-// in a fixed order, so the result does not depend on timing.
-__global__ void __launch_bounds__(256) reduce_partials_kernel(const float* __restrict__ partial, int R,
-                                                              int stride, float* __restrict__ y, int N) {
-  __shared__ float s_part[8][33];
+// y[col] = sum over r of partial[r][col]: 512 threads = 32 columns x 16
+// chains; chain c adds r = c, c + 16, ... in ascending order, then the 16 chains
+// are added in a fixed order, so the result does not depend on timing. A chain
+// issues all its loads (up to kRedLoads) before it adds, so the partials of a
+// column arrive in one memory round trip.
+constexpr int kRedChains = 16;
+constexpr int kRedLoads = 8;   // R <= 128 in one round trip; larger R loops
+__global__ void __launch_bounds__(32 * kRedChains) reduce_partials_kernel(const float* __restrict__ partial, int R,
+                                                                         int stride, float* __restrict__ y, int N) {
+  __shared__ float s_part[kRedChains][33];
   pdl_launch_dependents();
   pdl_wait();   // the partials come from the VMM kernel just before
   const int lane = threadIdx.x & 31, chain = threadIdx.x >> 5;
   const int col = blockIdx.x * 32 + lane;
   float v = 0.0f;
   if (col < N) {
-#pragma unroll 4
-    for (int r = chain; r < R; r += 8) v += partial[(size_t)r * stride + col];
+    for (int r0 = chain; r0 < R; r0 += kRedChains * kRedLoads) {
+      float p[kRedLoads];
+#pragma unroll
+      for (int i = 0; i < kRedLoads; ++i) {
+        const int r = r0 + kRedChains * i;
+        p[i] = (r < R) ? __ldcg(partial + (size_t)r * stride + col) : 0.0f;
+      }
+#pragma unroll
+      for (int i = 0; i < kRedLoads; ++i) v += p[i];
+    }
   }
   s_part[chain][lane] = v;
   __syncthreads();
   if (chain == 0 && col < N) {
     float acc = s_part[0][lane];
 #pragma unroll
-    for (int c = 1; c < 8; ++c) acc += s_part[c][lane];
+    for (int c = 1; c < kRedChains; ++c) acc += s_part[c][lane];
     y[col] = acc;
   }
 }
@@ -520,7 +533,7 @@ cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused) {
 
   cudaLaunchConfig_t rc = {};
   rc.gridDim = dim3((a.N + 31) / 32, 1, 1);
-  rc.blockDim = dim3(256, 1, 1);
+  rc.blockDim = dim3(32 * kRedChains, 1, 1);
   rc.stream = st;
   rc.attrs = attr;
   rc.numAttrs = 1;
