@@ -30,13 +30,17 @@ def lib():
         L.orc_f64_to_f16.argtypes = [ctypes.c_double]
         L.orc_f64_to_f16.restype = ctypes.c_uint16
         L.orc_rtn_quantize.argtypes = [P, i32, i32, P, P, P]
+        L.orc_rtn_quantize_bmax.argtypes = [P, i32, i32, i32, P, P, P]
         L.orc_code.argtypes = [i32, i32]
+        L.orc_code_bmax.argtypes = [i32, i32, i32]
         L.orc_grade.argtypes = [P, i32, P, i32, P, P]
         L.orc_compact.argtypes = [P, i32, P, i32, P, P]
         L.orc_vmm.argtypes = [P, P, P, P, P, i32, i32, P, P, i32]
+        L.orc_vmm_bmax.argtypes = [P, P, P, P, P, i32, i32, i32, P, P, i32]
         L.orc_maxent_distribution.argtypes = [P, i32, ctypes.c_double, P]
         L.orc_thresholds.argtypes = [P, i32, i32, P, i32, P]
-        for f in ("orc_rtn_quantize", "orc_code", "orc_grade", "orc_compact", "orc_vmm",
+        for f in ("orc_rtn_quantize", "orc_rtn_quantize_bmax", "orc_code", "orc_code_bmax", "orc_grade",
+                  "orc_compact", "orc_vmm", "orc_vmm_bmax",
                   "orc_maxent_distribution", "orc_thresholds"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -61,8 +65,8 @@ def f64_to_f16(v):
     return lib().orc_f64_to_f16(float(v))
 
 
-def rtn_quantize(W):
-    """8-bit asymmetric RTN per (row, 128-column group): Section 3.3 and Section 4.
+def rtn_quantize(W, bmax=8):
+    """b_max-bit asymmetric RTN per (row, 128-column group): Section 3.3 and Section 4.
 
     Returns (q uint8 [K,N], scale uint16 [K,n_g], zero uint16 [K,n_g])."""
     W = _c(W, np.float32)
@@ -71,14 +75,20 @@ def rtn_quantize(W):
     q = np.empty((K, N), np.uint8)
     s = np.empty((K, ng), np.uint16)
     z = np.empty((K, ng), np.uint16)
-    if lib().orc_rtn_quantize(_p(W), K, N, _p(q), _p(s), _p(z)) != 0:
-        raise ValueError("bad sizes")
+    if bmax == 8:
+        rc = lib().orc_rtn_quantize(_p(W), K, N, _p(q), _p(s), _p(z))
+    else:
+        rc = lib().orc_rtn_quantize_bmax(_p(W), K, N, int(bmax), _p(q), _p(s), _p(z))
+    if rc != 0:
+        raise ValueError("bad sizes or b_max")
     return q, s, z
 
 
-def code(q, b):
-    """Nested reconstruction code of q at width b (Section 3.3); -1 for b = 0."""
-    return lib().orc_code(int(q), int(b))
+def code(q, b, bmax=8):
+    """Nested reconstruction code of the b_max-bit code q at width b (Section 3.3); -1 for b = 0."""
+    if bmax == 8:
+        return lib().orc_code(int(q), int(b))
+    return lib().orc_code_bmax(int(q), int(b), int(bmax))
 
 
 def grade(x_bits, theta, classes):
@@ -105,8 +115,9 @@ def compact(bits, classes):
     return idx, off
 
 
-def vmm(x_bits, q, scale, zero, bits, nthreads=1):
-    """fp64 graded product y and the tolerance scale bound = sum |x_k * w_hat_kn|."""
+def vmm(x_bits, q, scale, zero, bits, nthreads=1, bmax=8):
+    """fp64 graded product y and the tolerance scale bound = sum |x_k * w_hat_kn|
+    (codes q of b_max bits, Section 3.3)."""
     x_bits = _c(x_bits, np.uint16)
     q = _c(q, np.uint8)
     scale = _c(scale, np.uint16)
@@ -115,8 +126,12 @@ def vmm(x_bits, q, scale, zero, bits, nthreads=1):
     K, N = q.shape
     y = np.empty(N, np.float64)
     bound = np.empty(N, np.float64)
-    rc = lib().orc_vmm(_p(x_bits), _p(q), _p(scale), _p(zero), _p(bits), K, N, _p(y), _p(bound),
-                       int(nthreads))
+    if bmax == 8:
+        rc = lib().orc_vmm(_p(x_bits), _p(q), _p(scale), _p(zero), _p(bits), K, N, _p(y), _p(bound),
+                           int(nthreads))
+    else:
+        rc = lib().orc_vmm_bmax(_p(x_bits), _p(q), _p(scale), _p(zero), _p(bits), K, N, int(bmax), _p(y),
+                                _p(bound), int(nthreads))
     if rc != 0:
         raise ValueError("bad sizes")
     return y, bound

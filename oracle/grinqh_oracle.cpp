@@ -74,22 +74,25 @@ uint16_t orc_f64_to_f16(double v) {
 }
 
 // ---------------------------------------------------------------------------
-// RTN 8-bit asymmetric quantisation per (row k, 128-column group g).
-// Paper: Section 3.3 (uniform quantisation to a b_max-bit integer q, with scale
-// s and zero point z fixed at full precision), Section 4 (RTN, G = 128) and
-// Appendix E.1 (the 8-bit RTN model is the parent of every truncated width).
-// Library convention: s = fp16(range / 255) rounded to nearest even straight
-// from fp64, s := 1 if that rounds to 0, s := 65504 if it overflows;
-// z = clamp(rne(-min / s), 0, 255) stored as fp16 (exact, and +0 rather than -0);
-// q = clamp(rne(w / s) + z, 0, 255). Quotients are taken in fp64; for a binary32
-// numerator and a binary16 denominator the fp64 quotient never lands on, or
-// crosses, a half-integer that the exact quotient does not, so rne of it equals
-// rne of the exact rational.
+// RTN asymmetric quantisation to b_max bits per (row k, 128-column group g).
+// Paper: Section 3.3 ("each weight w_ij is quantized to a b_max-bit integer",
+// with scale s and zero point z fixed at full b_max precision; b_max in
+// {4, 6, 8} is evaluated), Section 4 (RTN, G = 128) and Appendix E.1 (the RTN
+// model at b_max is the parent of every truncated width).
+// Library convention, with L = 2^b_max - 1 levels: s = fp16(range / L) rounded
+// to nearest even straight from fp64, s := 1 if that rounds to 0, s := 65504
+// if it overflows; z = clamp(rne(-min / s), 0, L) stored as fp16 (exact, and +0
+// rather than -0); q = clamp(rne(w / s) + z, 0, L). Quotients are taken in
+// fp64; for a binary32 numerator and a binary16 denominator the fp64 quotient
+// never lands on, or crosses, a half-integer that the exact quotient does not,
+// so rne of it equals rne of the exact rational.
 // Outputs: q[K*N] row-major, scale[K*n_g], zero[K*n_g] with n_g = ceil(N/128).
-// Returns 0, or -1 on bad sizes.
+// Returns 0, or -1 on bad sizes or b_max outside 1..8.
 // ---------------------------------------------------------------------------
-int orc_rtn_quantize(const float* W, int K, int N, uint8_t* q, uint16_t* scale, uint16_t* zero) {
-  if (K <= 0 || N <= 0) return -1;
+int orc_rtn_quantize_bmax(const float* W, int K, int N, int bmax, uint8_t* q, uint16_t* scale,
+                          uint16_t* zero) {
+  if (K <= 0 || N <= 0 || bmax < 1 || bmax > 8) return -1;
+  const double levels = (double)((1 << bmax) - 1);
   const int ng = (N + 127) / 128;
   for (int k = 0; k < K; ++k) {
     for (int g = 0; g < ng; ++g) {
@@ -101,20 +104,20 @@ int orc_rtn_quantize(const float* W, int K, int N, uint8_t* q, uint16_t* scale, 
         if (w > mx) mx = w;
       }
       const double range = mx - mn;
-      uint16_t sb = orc_f64_to_f16(range / 255.0);
+      uint16_t sb = orc_f64_to_f16(range / levels);
       double s = orc_f16_to_f64(sb);
       if (s == 0.0) { sb = 0x3C00; s = 1.0; }
       if (std::isinf(s)) { sb = 0x7BFF; s = 65504.0; }
       double z = std::nearbyint(-mn / s);
       if (z < 0.0) z = 0.0;
-      if (z > 255.0) z = 255.0;
+      if (z > levels) z = levels;
       z = z + 0.0;   // a zero point of -0 (min = +0) is stored as +0
       scale[(size_t)k * ng + g] = sb;
       zero[(size_t)k * ng + g] = orc_f64_to_f16(z);
       for (int n = c0; n < c1; ++n) {
         double v = std::nearbyint((double)W[(size_t)k * N + n] / s) + z;
         if (v < 0.0) v = 0.0;
-        if (v > 255.0) v = 255.0;
+        if (v > levels) v = levels;
         q[(size_t)k * N + n] = (uint8_t)v;
       }
     }
@@ -122,20 +125,27 @@ int orc_rtn_quantize(const float* W, int K, int N, uint8_t* q, uint16_t* scale, 
   return 0;
 }
 
+// The 8-bit case (b_max = 8, 255 levels), the library's default layout.
+int orc_rtn_quantize(const float* W, int K, int N, uint8_t* q, uint16_t* scale, uint16_t* zero) {
+  return orc_rtn_quantize_bmax(W, K, N, 8, q, scale, zero);
+}
+
 // ---------------------------------------------------------------------------
-// Nested reconstruction code of an 8-bit code q read at width b.
+// Nested reconstruction code of a b_max-bit code q read at width b.
 // Paper: Section 3.3, "Weight Reconstruction and Bias Correction": the top b
 // bits q_b, scaled back by 2^(b_max - b), plus the midpoint term
-// phi = 2^(b_max - b - 1). Library convention: phi is applied for 1 <= b <= 7
-// only (b = 8 reads q unchanged); b = 0 means the row is skipped entirely, and
-// this function returns -1 for it.
+// phi = 2^(b_max - b - 1). Library convention: phi is applied for
+// 1 <= b < b_max only (b = b_max reads q unchanged); b = 0 means the row is
+// skipped entirely, and these functions return -1 for it.
 // ---------------------------------------------------------------------------
-int orc_code(int q, int b) {
+int orc_code_bmax(int q, int b, int bmax) {
   if (b <= 0) return -1;
-  if (b >= 8) return q;
-  const int qb = q >> (8 - b);            // the b most significant bits
-  return qb * (1 << (8 - b)) + (1 << (7 - b));
+  if (b >= bmax) return q;
+  const int qb = q >> (bmax - b);         // the b most significant of the b_max bits
+  return qb * (1 << (bmax - b)) + (1 << (bmax - b - 1));
 }
+
+int orc_code(int q, int b) { return orc_code_bmax(q, b, 8); }
 
 // ---------------------------------------------------------------------------
 // Grading. Paper: Section 3.1 "Dynamic Precision Assignment": b_i = b_k when
@@ -183,16 +193,16 @@ int orc_compact(const uint8_t* bits, int K, const uint8_t* classes, int n_classe
 // The graded vector-matrix product, in fp64.
 // Paper: Section 3 / Fig. 2 (only the top b_k bits of row k take part, b = 0
 // rows are bypassed) and the reconstruction of Section 3.3 with the library's
-// zero-point form w_hat = s * (code - z).
+// zero-point form w_hat = s * (code - z), code = orc_code_bmax(q, b, b_max).
 // y[n] = sum over k ascending with bits[k] > 0 of x_k * w_hat[k][n];
 // bound[n] = sum of |x_k * w_hat[k][n]| over the same k (the scale of the
 // parity tolerance). x, scale, zero are fp16 bit patterns.
 // nthreads > 1 splits the COLUMNS across OpenMP threads; every y[n] is still
 // summed over k in ascending order.
 // ---------------------------------------------------------------------------
-int orc_vmm(const uint16_t* x, const uint8_t* q, const uint16_t* scale, const uint16_t* zero,
-            const uint8_t* bits, int K, int N, double* y, double* bound, int nthreads) {
-  if (K < 0 || N <= 0) return -1;
+int orc_vmm_bmax(const uint16_t* x, const uint8_t* q, const uint16_t* scale, const uint16_t* zero,
+                 const uint8_t* bits, int K, int N, int bmax, double* y, double* bound, int nthreads) {
+  if (K < 0 || N <= 0 || bmax < 1 || bmax > 8) return -1;
   const int ng = (N + 127) / 128;
   for (int n = 0; n < N; ++n) { y[n] = 0.0; if (bound) bound[n] = 0.0; }
   if (nthreads < 1) nthreads = 1;
@@ -209,7 +219,7 @@ int orc_vmm(const uint16_t* x, const uint8_t* q, const uint16_t* scale, const ui
         const int g = n / 128;
         const double s = orc_f16_to_f64(scale[(size_t)k * ng + g]);
         const double z = orc_f16_to_f64(zero[(size_t)k * ng + g]);
-        const double w = s * ((double)orc_code(q[(size_t)k * N + n], b) - z);
+        const double w = s * ((double)orc_code_bmax(q[(size_t)k * N + n], b, bmax) - z);
         const double t2 = xk * w;
         y[n] += t2;
         if (bound) bound[n] += std::fabs(t2);
@@ -217,6 +227,11 @@ int orc_vmm(const uint16_t* x, const uint8_t* q, const uint16_t* scale, const ui
     }
   }
   return 0;
+}
+
+int orc_vmm(const uint16_t* x, const uint8_t* q, const uint16_t* scale, const uint16_t* zero,
+            const uint8_t* bits, int K, int N, double* y, double* bound, int nthreads) {
+  return orc_vmm_bmax(x, q, scale, zero, bits, K, N, 8, y, bound, nthreads);
 }
 
 // ---------------------------------------------------------------------------
