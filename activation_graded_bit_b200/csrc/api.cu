@@ -33,8 +33,15 @@ bool valid_classes(const uint8_t* classes, int32_t n) {
 bool layout_ok(const grinqh_layout* L) {
   if (!L) return false;
   grinqh_layout ref;
-  if (grinqh_layout_init(L->K, L->N, &ref) != GRINQH_OK) return false;
+  if (grinqh_layout_init_bmax(L->K, L->N, L->b_max, &ref) != GRINQH_OK) return false;
   return std::memcmp(&ref, L, sizeof(ref)) == 0;
+}
+
+// Every class width fits the layout's stored planes.
+bool classes_fit(const uint8_t* classes, int32_t n, int32_t b_max) {
+  for (int i = 0; i < n; ++i)
+    if (classes[i] > b_max) return false;
+  return true;
 }
 
 ClassTable table(const uint8_t* classes, int32_t n) {
@@ -80,7 +87,12 @@ const char* grinqh_status_string(grinqh_status s) {
 }
 
 grinqh_status grinqh_layout_init(int32_t K, int32_t N, grinqh_layout* out) {
+  return grinqh_layout_init_bmax(K, N, kPlanes, out);
+}
+
+grinqh_status grinqh_layout_init_bmax(int32_t K, int32_t N, int32_t b_max, grinqh_layout* out) {
   if (!out) return GRINQH_ERR_INVALID_ARG;
+  if (b_max != 2 && b_max != 4 && b_max != 6 && b_max != 8) return GRINQH_ERR_INVALID_ARG;
   if (K < 1 || N < 1 || K > kMaxDim || N > kMaxDim) return GRINQH_ERR_INVALID_ARG;
   if ((int64_t)K * N > kMaxElems) return GRINQH_ERR_INVALID_ARG;
   grinqh_layout L;
@@ -90,8 +102,10 @@ grinqh_status grinqh_layout_init(int32_t K, int32_t N, grinqh_layout* out) {
   L.n_groups = (N + GRINQH_GROUP - 1) / GRINQH_GROUP;
   L.tile_n = kTileN;
   L.n_tiles = (N + kTileN - 1) / kTileN;
-  L.record_bytes = kRecordBytes;
-  L.packed_bytes = (int64_t)K * L.n_tiles * kRecordBytes;
+  L.record_bytes = record_bytes_for(b_max);
+  L.b_max = b_max;
+  L.reserved = 0;
+  L.packed_bytes = (int64_t)K * L.n_tiles * L.record_bytes;
   *out = L;
   return GRINQH_OK;
 }
@@ -100,7 +114,7 @@ grinqh_status grinqh_pack(const grinqh_layout* layout, const float* W, void* pac
   if (!layout_ok(layout) || !W || !packed) return GRINQH_ERR_INVALID_ARG;
   if (!aligned(W, 4) || !aligned(packed, 16)) return GRINQH_ERR_ALIGNMENT;
   const grinqh_layout& L = *layout;
-  return cuda_status(launch_pack(W, L.K, L.N, L.n_tiles, L.n_groups, packed, (cudaStream_t)stream));
+  return cuda_status(launch_pack(W, L.K, L.N, L.n_tiles, L.n_groups, L.b_max, packed, (cudaStream_t)stream));
 }
 
 grinqh_status grinqh_unpack_codes(const grinqh_layout* layout, const void* packed, const uint8_t* bits,
@@ -108,7 +122,7 @@ grinqh_status grinqh_unpack_codes(const grinqh_layout* layout, const void* packe
   if (!layout_ok(layout) || !packed || !codes) return GRINQH_ERR_INVALID_ARG;
   if (!aligned(packed, 16)) return GRINQH_ERR_ALIGNMENT;
   const grinqh_layout& L = *layout;
-  return cuda_status(launch_unpack(packed, bits, L.K, L.N, L.n_tiles, codes, (cudaStream_t)stream));
+  return cuda_status(launch_unpack(packed, bits, L.K, L.N, L.n_tiles, L.b_max, codes, (cudaStream_t)stream));
 }
 
 grinqh_status grinqh_maxent_distribution(const uint8_t* classes, int32_t n_classes, double target_bits,
@@ -224,6 +238,7 @@ grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* packed, const 
                          const int32_t* offsets, const uint8_t* classes, int32_t n_classes, float* y,
                          void* workspace, size_t workspace_bytes, void* stream) {
   if (!layout_ok(layout) || !valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
+  if (!classes_fit(classes, n_classes, layout->b_max)) return GRINQH_ERR_INVALID_ARG;
   if (!packed || !x || !idx || !offsets || !y) return GRINQH_ERR_INVALID_ARG;
   if (!aligned(packed, 16) || !aligned(x, 2) || !aligned(idx, 4) || !aligned(offsets, 4) || !aligned(y, 4))
     return GRINQH_ERR_ALIGNMENT;
@@ -235,6 +250,7 @@ grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* packed, const 
   a.K = L.K;
   a.N = L.N;
   a.n_tiles = L.n_tiles;
+  a.b_max = L.b_max;
   a.packed = (const uint8_t*)packed;
   a.x = x;
   a.idx = idx;
@@ -250,6 +266,7 @@ grinqh_status grinqh_vmm_noalloc(const grinqh_layout* layout, const void* packed
                                  const int32_t* idx, const int32_t* offsets, const uint8_t* classes,
                                  int32_t n_classes, float* y, void* stream) {
   if (!layout_ok(layout) || !valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
+  if (!classes_fit(classes, n_classes, layout->b_max)) return GRINQH_ERR_INVALID_ARG;
   if (!packed || !x || !idx || !offsets || !y) return GRINQH_ERR_INVALID_ARG;
   if (!aligned(packed, 16) || !aligned(x, 2) || !aligned(idx, 4) || !aligned(offsets, 4) || !aligned(y, 4))
     return GRINQH_ERR_ALIGNMENT;
@@ -261,6 +278,7 @@ grinqh_status grinqh_vmm_noalloc(const grinqh_layout* layout, const void* packed
   a.K = L.K;
   a.N = L.N;
   a.n_tiles = L.n_tiles;
+  a.b_max = L.b_max;
   a.packed = (const uint8_t*)packed;
   a.x = x;
   a.idx = idx;
@@ -276,6 +294,7 @@ grinqh_status grinqh_select_vmm(const grinqh_layout* layout, const void* packed,
                                 const float* thresholds, const uint8_t* classes, int32_t n_classes, float* y,
                                 void* workspace, size_t workspace_bytes, void* stream) {
   if (!layout_ok(layout) || !valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
+  if (!classes_fit(classes, n_classes, layout->b_max)) return GRINQH_ERR_INVALID_ARG;
   if (!packed || !x || !y || (n_classes > 1 && !thresholds)) return GRINQH_ERR_INVALID_ARG;
   if (!aligned(packed, 16) || !aligned(x, 2) || !aligned(y, 4) || (thresholds && !aligned(thresholds, 4)))
     return GRINQH_ERR_ALIGNMENT;
@@ -288,6 +307,7 @@ grinqh_status grinqh_select_vmm(const grinqh_layout* layout, const void* packed,
   a.K = L.K;
   a.N = L.N;
   a.n_tiles = L.n_tiles;
+  a.b_max = L.b_max;
   a.packed = (const uint8_t*)packed;
   a.x = x;
   a.thresholds = thresholds;

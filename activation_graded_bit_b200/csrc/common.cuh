@@ -29,6 +29,10 @@ constexpr int kPlaneBytes = kTileN / 8;               // one plane of one tile r
 constexpr int kPairBytes = 2 * kPlaneBytes;           // two planes of one tile row
 constexpr int kRecordBytes = kMetaBytes + kPlanes * kPlaneBytes;   // 1056 = 33 sectors of 32 B
 
+// Bytes of a (row, tile) record that stores b_max planes: the scale/zero words,
+// then b_max / 2 plane pairs (a whole number of 32-byte sectors).
+__host__ __device__ constexpr int record_bytes_for(int b_max) { return kMetaBytes + b_max * kPlaneBytes; }
+
 // The column (0..15 inside the half) and plane offset l stored at bit L of a
 // pair-s word (the inverse of the placement above: column 4j'+i of plane 2s+l
 // at bit (8i + 2j' + 7 - 2s - l) mod 32).
@@ -78,13 +82,6 @@ __device__ __forceinline__ void assemble(const uint32_t (&P)[8], uint32_t (&out)
   if (B == 5) merge_pair_top<2>(P[4], P[5], T);
   if (B == 7) merge_pair_top<3>(P[6], P[7], T);
   finish_codes(T, out);
-}
-
-// Midpoint term of the nested reconstruction for width b (0 for b = 8):
-// 2^(7-b) in every byte (the low 8-b bits of a truncated code are zero, so an
-// OR adds it).
-__host__ __device__ __forceinline__ uint32_t midpoint_bytes(int b) {
-  return b >= 8 ? 0u : 0x01010101u * (1u << (7 - b));
 }
 
 __device__ __forceinline__ float half_bits_to_float(uint32_t h) {

@@ -7,10 +7,11 @@
 
 namespace grinqh {
 
-cudaError_t launch_pack(const float* W, int K, int N, int n_tiles, int n_groups, void* packed, cudaStream_t st);
+cudaError_t launch_pack(const float* W, int K, int N, int n_tiles, int n_groups, int b_max, void* packed,
+                        cudaStream_t st);
 
-cudaError_t launch_unpack(const void* packed, const uint8_t* bits, int K, int N, int n_tiles, uint8_t* codes,
-                          cudaStream_t st);
+cudaError_t launch_unpack(const void* packed, const uint8_t* bits, int K, int N, int n_tiles, int b_max,
+                          uint8_t* codes, cudaStream_t st);
 
 struct ClassTable {
   int n;              // number of classes (1..9)
@@ -22,6 +23,7 @@ cudaError_t launch_select(const uint16_t* x, int K, const float* thresholds, con
 
 struct VmmArgs {
   int K, N, n_tiles;
+  int b_max;                 // bits per stored code (2, 4, 6 or 8); records of record_bytes_for(b_max)
   const uint8_t* packed;
   const uint16_t* x;
   const int32_t* idx;

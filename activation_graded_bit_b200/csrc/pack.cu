@@ -1,5 +1,5 @@
-// Offline packing: 8-bit RTN per (row, 128-column group) + MSB-first bit planes,
-// and the test-only decoder of the packed format.
+// Offline packing: b_max-bit RTN per (row, 128-column group) + MSB-first bit
+// planes (b_max = 2, 4, 6 or 8), and the test-only decoder of the packed format.
 //
 // Paper: "GRINQH" Section 3.3 (uniform b_max-bit codes split into significance
 // slices, input-major storage), Section 4 (RTN with group size 128) and
@@ -25,16 +25,19 @@ __device__ __forceinline__ double f16_to_f64(uint16_t h) {
 }
 
 // One CTA per (row k, tile t): 8 warps, warp g handles the tile's group g
-// (128 columns), then 256 threads build the 8 x 32 plane words of the record.
+// (128 columns), then 64 threads per plane pair build the b_max/2 pairs of
+// plane words of the record.
 __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ W, int K, int N, int n_tiles,
-                                                   int n_groups, uint8_t* __restrict__ packed) {
+                                                   int n_groups, int b_max, uint8_t* __restrict__ packed) {
   __shared__ uint8_t codes[kTileN];
   const int k = blockIdx.x, t = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gl = t * (kTileN / kGroup) + warp;     // global group index
   const int c0 = gl * kGroup;                      // first column of the group
   const float* row = W + (size_t)k * N;
-  uint8_t* rec = packed + ((size_t)k * n_tiles + t) * kRecordBytes;
+  const int rbytes = record_bytes_for(b_max);
+  const double levels = (double)((1 << b_max) - 1);
+  uint8_t* rec = packed + ((size_t)k * n_tiles + t) * rbytes;
 
   float v[4];
   float mn = INFINITY, mx = -INFINITY;
@@ -54,12 +57,12 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ W, 
   uint16_t sb = 0, zb = 0;
   if (live) {
     const double range = __dsub_rn((double)mx, (double)mn);
-    sb = f64_to_f16_rn(__ddiv_rn(range, 255.0));
+    sb = f64_to_f16_rn(__ddiv_rn(range, levels));
     s = f16_to_f64(sb);
     if (s == 0.0) { sb = 0x3C00; s = 1.0; }
     if (isinf(s)) { sb = 0x7BFF; s = 65504.0; }
     z = rint(__ddiv_rn(-(double)mn, s));
-    z = __dadd_rn(fmin(fmax(z, 0.0), 255.0), 0.0);   // -0 -> +0
+    z = __dadd_rn(fmin(fmax(z, 0.0), levels), 0.0);   // -0 -> +0
     zb = f64_to_f16_rn(z);
   }
 #pragma unroll
@@ -68,7 +71,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ W, 
     uint8_t q = 0;
     if (live && n < N) {
       double qv = __dadd_rn(rint(__ddiv_rn((double)v[e], s)), z);
-      qv = fmin(fmax(qv, 0.0), 255.0);
+      qv = fmin(fmax(qv, 0.0), levels);
       q = (uint8_t)qv;
     }
     codes[warp * kGroup + lane + 32 * e] = q;
@@ -77,9 +80,11 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ W, 
     reinterpret_cast<uint32_t*>(rec)[warp] = live ? ((uint32_t)sb | ((uint32_t)zb << 16)) : 0u;
   __syncthreads();
 
-  // thread -> (pair s, word wi): 4 plane pairs x 64 words for a 1024-column
-  // tile; word wi is half wi & 1 of lane wi >> 1's 32 columns
+  // thread -> (pair s, word wi): b_max/2 plane pairs x 64 words for a
+  // 1024-column tile; word wi is half wi & 1 of lane wi >> 1's 32 columns;
+  // plane p holds bit b_max-1-p of the code
   const int sp = threadIdx.x >> 6, wi = threadIdx.x & 63;
+  if (2 * sp >= b_max) return;
   const int cbase = 32 * (wi >> 1) + 16 * (wi & 1);
   uint32_t word = 0;
 #pragma unroll 8
@@ -87,14 +92,16 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ W, 
     int c16, l;
     pair_col_at(sp, L, c16, l);
     const int p = 2 * sp + l;
-    word |= (uint32_t)((codes[cbase + c16] >> (7 - p)) & 1u) << L;
+    word |= (uint32_t)((codes[cbase + c16] >> (b_max - 1 - p)) & 1u) << L;
   }
   reinterpret_cast<uint32_t*>(rec + kMetaBytes + sp * kPairBytes)[wi] = word;
 }
 
-// Decoder: one warp per (row, tile) record, 8 records per CTA.
+// Decoder: one warp per (row, tile) record, 8 records per CTA. The planes are
+// rebuilt in the 8-bit frame (plane p at bit 7-p), then shifted down to the
+// b_max-bit code with the midpoint 2^(b_max-B-1) of a width B < b_max.
 template <int B>
-__device__ __forceinline__ void decode_word(const uint8_t* rec, int w, uint32_t (&R)[8]) {
+__device__ __forceinline__ void decode_word(const uint8_t* rec, int w, int b_max, uint32_t (&R)[8]) {
   uint32_t P[8];
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
@@ -104,30 +111,32 @@ __device__ __forceinline__ void decode_word(const uint8_t* rec, int w, uint32_t 
     P[2 * s + 1] = used ? pw[2 * w + 1] : 0u;
   }
   assemble<B>(P, R);
-  const uint32_t mid = midpoint_bytes(B);
+  const int sh = 8 - b_max;
+  const uint32_t keep = 0x01010101u * ((1u << b_max) - 1u);
+  const uint32_t mid = (B < b_max) ? 0x01010101u * (1u << (b_max - B - 1)) : 0u;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) R[j] |= mid;
+  for (int j = 0; j < 8; ++j) R[j] = ((R[j] >> sh) & keep) | mid;
 }
 
 __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__ packed,
                                                      const uint8_t* __restrict__ bits, int K, int N,
-                                                     int n_tiles, uint8_t* __restrict__ codes) {
+                                                     int n_tiles, int b_max, uint8_t* __restrict__ codes) {
   const int t = blockIdx.y;
   const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int w = threadIdx.x & 31;
   if (k >= K) return;
-  const int b = bits ? bits[k] : 8;
-  const uint8_t* rec = packed + ((size_t)k * n_tiles + t) * kRecordBytes;
+  const int b = min(bits ? (int)bits[k] : b_max, b_max);   // a width above b_max decodes as b_max
+  const uint8_t* rec = packed + ((size_t)k * n_tiles + t) * record_bytes_for(b_max);
   uint32_t R[8];
   switch (b) {
-    case 1: decode_word<1>(rec, w, R); break;
-    case 2: decode_word<2>(rec, w, R); break;
-    case 3: decode_word<3>(rec, w, R); break;
-    case 4: decode_word<4>(rec, w, R); break;
-    case 5: decode_word<5>(rec, w, R); break;
-    case 6: decode_word<6>(rec, w, R); break;
-    case 7: decode_word<7>(rec, w, R); break;
-    case 8: decode_word<8>(rec, w, R); break;
+    case 1: decode_word<1>(rec, w, b_max, R); break;
+    case 2: decode_word<2>(rec, w, b_max, R); break;
+    case 3: decode_word<3>(rec, w, b_max, R); break;
+    case 4: decode_word<4>(rec, w, b_max, R); break;
+    case 5: decode_word<5>(rec, w, b_max, R); break;
+    case 6: decode_word<6>(rec, w, b_max, R); break;
+    case 7: decode_word<7>(rec, w, b_max, R); break;
+    case 8: decode_word<8>(rec, w, b_max, R); break;
     default:
 #pragma unroll
       for (int j = 0; j < 8; ++j) R[j] = 0u;
@@ -143,16 +152,17 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
     }
 }
 
-cudaError_t launch_pack(const float* W, int K, int N, int n_tiles, int n_groups, void* packed, cudaStream_t st) {
+cudaError_t launch_pack(const float* W, int K, int N, int n_tiles, int n_groups, int b_max, void* packed,
+                        cudaStream_t st) {
   dim3 grid(K, n_tiles);
-  pack_kernel<<<grid, 256, 0, st>>>(W, K, N, n_tiles, n_groups, (uint8_t*)packed);
+  pack_kernel<<<grid, 256, 0, st>>>(W, K, N, n_tiles, n_groups, b_max, (uint8_t*)packed);
   return cudaGetLastError();
 }
 
-cudaError_t launch_unpack(const void* packed, const uint8_t* bits, int K, int N, int n_tiles, uint8_t* codes,
-                          cudaStream_t st) {
+cudaError_t launch_unpack(const void* packed, const uint8_t* bits, int K, int N, int n_tiles, int b_max,
+                          uint8_t* codes, cudaStream_t st) {
   dim3 grid((K + 7) / 8, n_tiles);
-  unpack_kernel<<<grid, 256, 0, st>>>((const uint8_t*)packed, bits, K, N, n_tiles, codes);
+  unpack_kernel<<<grid, 256, 0, st>>>((const uint8_t*)packed, bits, K, N, n_tiles, b_max, codes);
   return cudaGetLastError();
 }
 

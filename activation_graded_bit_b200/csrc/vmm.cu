@@ -97,7 +97,8 @@ struct RowRegs {
 };
 
 // Per-thread constants of the row addressing: a row's record starts at
-// packed + 32 * (k * n_tiles * 33 + t * 33) (records are 33 sectors of 32 B),
+// packed + 32 * (k * n_tiles * S + t * S) (records are S = 1 + 4 b_max sectors
+// of 32 B: 33 for b_max = 8),
 // so one integer multiply-add gives its offset in sectors (below 2^32: a valid
 // layout has K * N <= 2^34, so K * n_tiles <= 2^25) and one wide multiply-add
 // each of this lane's addresses in it.
@@ -110,8 +111,8 @@ struct RowAddr {
 };
 
 __device__ __forceinline__ RowAddr row_addr(const VmmArgs& a, int t, int w) {
-  constexpr uint32_t kSectors = kRecordBytes / 32;
-  static_assert(kRecordBytes % 32 == 0, "records are whole 32-byte sectors");
+  const uint32_t kSectors = (uint32_t)record_bytes_for(a.b_max) / 32u;   // 9, 17, 25 or 33
+  static_assert(kMetaBytes % 32 == 0 && kPlaneBytes % 16 == 0, "records are whole 32-byte sectors");
   RowAddr ra;
   ra.meta = a.packed + 4 * (w >> 2);
   ra.pairs = a.packed + kMetaBytes + 8 * w;
@@ -150,16 +151,26 @@ __device__ __forceinline__ void ld_stream2_at_if(bool on, const void* ptr, uint3
       : "l"(ptr), "r"((uint32_t)on), "n"(kOff));
 }
 
-// Per-row coefficients: A0 = a 2^95 (for c_lo 2^-149), A1 = a 2^87 (for c_hi
-// 2^-141), and the row's constant a * (mid - z) added to cacc (mid = 2^(7-b)
-// for b < 8, 0 for b = 8).
+// Per-row coefficients for codes of kBmax bits, rebuilt in the 8-bit frame
+// (plane p at bit 7-p, so a code c of kBmax bits reads as c 2^(8-kBmax)):
+// A0 = a 2^(87+kBmax) (for c_lo 2^-149), A1 = a 2^(79+kBmax) (for c_hi 2^-141),
+// so the products carry a * c 2^-54 in kBmax-bit units, and the row's constant
+// a * (mid - z) is added to cacc (mid = 2^(kBmax-b-1) for b < kBmax, 0 at
+// b = kBmax, in the same units as z).
+template <int kBmax>
 __device__ __forceinline__ void row_coef(uint32_t m, float mid, float xk, float& A0, float& A1, float& cacc) {
   const float s = half_bits_to_float(m);
   const float z = half_bits_to_float(m >> 16);
   const float av = xk * s;                                      // exact
   cacc = fmaf(av, mid - z, cacc);
-  A0 = av * 0x1p95f;
-  A1 = av * 0x1p87f;
+  A0 = av * (float)(1ull << (23 + kBmax)) * 0x1p64f;
+  A1 = av * (float)(1ull << (15 + kBmax)) * 0x1p64f;
+}
+
+// The bin midpoint of width b for codes of kBmax bits, 0 at full width.
+template <int kBmax>
+__device__ __forceinline__ constexpr float midpoint(int b) {
+  return b >= kBmax ? 0.0f : (float)(1u << (kBmax - b - 1));
 }
 
 // acc += codes * coefficients for the 32 columns held in R (one row).
@@ -204,32 +215,34 @@ __device__ __forceinline__ void load_row(const VmmArgs& a, const RowAddr& ra, ui
 // at run time), with one indirect jump: the top plane of the last pair for odd
 // b, the full pair for even b, then the full pairs below it in one shared
 // sequence. out[j] byte i = top-b bits of column 4j+i, in place, low bits zero;
-// mid = the bin midpoint 2^(7-b) (0 for b = 8), fixed by the jump target.
+// mid = the bin midpoint in kBmax-bit units (0 at b = kBmax), fixed by the jump
+// target. Widths above kBmax never reach the kernel (the host rejects them).
+template <int kBmax>
 __device__ __forceinline__ void assemble_row(const RowRegs& r, uint32_t (&out)[8], float& mid) {
   uint32_t T[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) T[j] = 0u;
   switch (r.b) {
-    case 8: mid = 0.0f; merge_pair<3>(r.p[6], r.p[7], T); goto pairs3;
-    case 7: mid = 1.0f; merge_pair_top<3>(r.p[6], r.p[7], T); goto pairs3;
+    case 8: mid = midpoint<kBmax>(8); merge_pair<3>(r.p[6], r.p[7], T); goto pairs3;
+    case 7: mid = midpoint<kBmax>(7); merge_pair_top<3>(r.p[6], r.p[7], T); goto pairs3;
     case 6:
-      mid = 2.0f;
+      mid = midpoint<kBmax>(6);
     pairs3:
       merge_pair<2>(r.p[4], r.p[5], T);
       goto pairs2;
-    case 5: mid = 4.0f; merge_pair_top<2>(r.p[4], r.p[5], T); goto pairs2;
+    case 5: mid = midpoint<kBmax>(5); merge_pair_top<2>(r.p[4], r.p[5], T); goto pairs2;
     case 4:
-      mid = 8.0f;
+      mid = midpoint<kBmax>(4);
     pairs2:
       merge_pair<1>(r.p[2], r.p[3], T);
       goto pairs1;
-    case 3: mid = 16.0f; merge_pair_top<1>(r.p[2], r.p[3], T); goto pairs1;
+    case 3: mid = midpoint<kBmax>(3); merge_pair_top<1>(r.p[2], r.p[3], T); goto pairs1;
     case 2:
-      mid = 32.0f;
+      mid = midpoint<kBmax>(2);
     pairs1:
       merge_pair<0>(r.p[0], r.p[1], T);
       break;
-    default: mid = 64.0f; merge_pair_top<0>(r.p[0], r.p[1], T); break;   // b == 1
+    default: mid = midpoint<kBmax>(1); merge_pair_top<0>(r.p[0], r.p[1], T); break;   // b == 1
   }
   finish_codes(T, out);
 }
@@ -246,12 +259,13 @@ __device__ __forceinline__ void prefetch_row_l2(const RowAddr& ra, uint32_t info
                "r"(on));
 }
 
+template <int kBmax>
 __device__ __forceinline__ void row_fma(const RowRegs& r, float2 (&acc)[16], float& cacc) {
   uint32_t R[8];
   float mid;
-  assemble_row(r, R, mid);
+  assemble_row<kBmax>(r, R, mid);
   float A0, A1;
-  row_coef(r.m, mid, __half2float(__ushort_as_half((unsigned short)r.xh)), A0, A1, cacc);
+  row_coef<kBmax>(r.m, mid, __half2float(__ushort_as_half((unsigned short)r.xh)), A0, A1, cacc);
   fma_codes(R, A0, A1, acc);
 }
 
@@ -306,7 +320,7 @@ __device__ __forceinline__ int stage_fused(const VmmArgs& a, VmmSmem& s, int r, 
 }
 
 
-template <bool kFused>
+template <bool kFused, int kBmax>
 __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   VmmSmem& s = *reinterpret_cast<VmmSmem*>(smem_raw);
@@ -391,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
 #pragma unroll
       for (int d = 0; d < kDepth; ++d) {
         const int m = m0 + d;
-        row_fma(S[d], acc, cacc);
+        row_fma<kBmax>(S[d], acc, cacc);
         load_row(a, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
         // the record prefix of the row kL2Ahead rows further on goes to L2 now,
         // one 128-byte line per lane, so its register loads later hit L2
@@ -408,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
       for (int d = 0; d < kDepth; ++d) {
         const int m = m0 + d;
         if (m < nrow) {
-          row_fma(S[d], acc, cacc);
+          row_fma<kBmax>(S[d], acc, cacc);
           if (m + kDepth < nrow) load_row(a, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
         }
       }
@@ -505,14 +519,30 @@ size_t vmm_workspace_bytes(int n_tiles, int /*tile_n*/) {
   return 16 + (R > 1 ? (size_t)R * n_tiles * kTileN * sizeof(float) : 0);
 }
 
+template <int kBmax>
+static cudaError_t set_smem_attr() {
+  const int smem = (int)sizeof(VmmSmem);
+  cudaError_t e = cudaFuncSetAttribute(vmm_kernel<false, kBmax>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(vmm_kernel<true, kBmax>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return e;
+}
+
+template <int kBmax>
+static cudaError_t launch_one(const cudaLaunchConfig_t& cfg, const VmmArgs& a, bool fused) {
+  return fused ? cudaLaunchKernelEx(&cfg, vmm_kernel<true, kBmax>, a) : cudaLaunchKernelEx(&cfg, vmm_kernel<false, kBmax>, a);
+}
+
 cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   const int smem = (int)sizeof(VmmSmem);
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(vmm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(vmm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_smem_attr<8>();
+    if (e == cudaSuccess) e = set_smem_attr<6>();
+    if (e == cudaSuccess) e = set_smem_attr<4>();
+    if (e == cudaSuccess) e = set_smem_attr<2>();
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
@@ -528,7 +558,14 @@ cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused) {
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = fused ? cudaLaunchKernelEx(&cfg, vmm_kernel<true>, a) : cudaLaunchKernelEx(&cfg, vmm_kernel<false>, a);
+  cudaError_t e;
+  switch (a.b_max) {
+    case 2: e = launch_one<2>(cfg, a, fused); break;
+    case 4: e = launch_one<4>(cfg, a, fused); break;
+    case 6: e = launch_one<6>(cfg, a, fused); break;
+    case 8: e = launch_one<8>(cfg, a, fused); break;
+    default: return cudaErrorInvalidValue;
+  }
   if (e != cudaSuccess || R == 1) return e;
 
   cudaLaunchConfig_t rc = {};

@@ -38,7 +38,7 @@ class GrinqhError(RuntimeError):
 class Layout(ctypes.Structure):
     _fields_ = [("K", ctypes.c_int32), ("N", ctypes.c_int32), ("n_groups", ctypes.c_int32),
                 ("tile_n", ctypes.c_int32), ("n_tiles", ctypes.c_int32), ("record_bytes", ctypes.c_int32),
-                ("packed_bytes", ctypes.c_int64)]
+                ("b_max", ctypes.c_int32), ("reserved", ctypes.c_int32), ("packed_bytes", ctypes.c_int64)]
 
 
 _P = ctypes.c_void_p
@@ -56,6 +56,7 @@ def _sig(name, args, res=ctypes.c_int):
 _version = _sig("grinqh_version", [], ctypes.c_char_p)
 _status_string = _sig("grinqh_status_string", [ctypes.c_int], ctypes.c_char_p)
 _layout_init = _sig("grinqh_layout_init", [_I, _I, _LP])
+_layout_init_bmax = _sig("grinqh_layout_init_bmax", [_I, _I, _I, _LP])
 _pack = _sig("grinqh_pack", [_LP, _P, _P, _P])
 _unpack = _sig("grinqh_unpack_codes", [_LP, _P, _P, _P, _P])
 _maxent = _sig("grinqh_maxent_distribution", [_P, _I, ctypes.c_double, _P])
@@ -68,7 +69,7 @@ _vmm_noalloc = _sig("grinqh_vmm_noalloc", [_LP, _P, _P, _P, _P, _P, _I, _P, _P])
 _select_vmm = _sig("grinqh_select_vmm", [_LP, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
 
 # Every exported symbol of the C ABI, for the export check in the tests.
-EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grinqh_pack",
+EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grinqh_layout_init_bmax", "grinqh_pack",
            "grinqh_unpack_codes", "grinqh_maxent_distribution", "grinqh_calibrate_workspace_bytes",
            "grinqh_calibrate", "grinqh_select", "grinqh_vmm_workspace_bytes", "grinqh_vmm",
            "grinqh_vmm_noalloc", "grinqh_select_vmm")
@@ -98,9 +99,12 @@ def _classes_buf(classes: Sequence[int]):
     return arr, len(classes)
 
 
-def layout(K: int, N: int) -> Layout:
+def layout(K: int, N: int, b_max: int = 8) -> Layout:
     L = Layout()
-    _check(_layout_init(int(K), int(N), ctypes.byref(L)), "grinqh_layout_init")
+    if b_max == 8:
+        _check(_layout_init(int(K), int(N), ctypes.byref(L)), "grinqh_layout_init")
+    else:
+        _check(_layout_init_bmax(int(K), int(N), int(b_max), ctypes.byref(L)), "grinqh_layout_init_bmax")
     return L
 
 
@@ -118,6 +122,10 @@ class PackedLayer:
     def N(self):
         return self.layout.N
 
+    @property
+    def b_max(self):
+        return self.layout.b_max
+
     def meta_words(self) -> torch.Tensor:
         """uint32 view [K, n_tiles, 8] of the scale | zero << 16 words of every record."""
         L = self.layout
@@ -125,16 +133,17 @@ class PackedLayer:
         return rec[:, :, :32].contiguous().view(torch.int32).view(L.K, L.n_tiles, 8)
 
 
-def empty_packed(K: int, N: int, device="cuda") -> PackedLayer:
-    L = layout(K, N)
+def empty_packed(K: int, N: int, device="cuda", b_max: int = 8) -> PackedLayer:
+    L = layout(K, N, b_max)
     return PackedLayer(L, torch.empty(int(L.packed_bytes), dtype=torch.uint8, device=device))
 
 
-def pack(W: torch.Tensor, out: Optional[PackedLayer] = None, stream=None) -> PackedLayer:
-    """grinqh_pack: W is a contiguous fp32 [K, N] CUDA tensor."""
+def pack(W: torch.Tensor, out: Optional[PackedLayer] = None, stream=None, b_max: int = 8) -> PackedLayer:
+    """grinqh_pack: W is a contiguous fp32 [K, N] CUDA tensor; codes of b_max bits
+    (out, when given, fixes b_max through its layout)."""
     assert W.dtype == torch.float32 and W.is_cuda and W.is_contiguous() and W.dim() == 2
     K, N = W.shape
-    p = out if out is not None else empty_packed(K, N, W.device)
+    p = out if out is not None else empty_packed(K, N, W.device, b_max)
     _check(_pack(ctypes.byref(p.layout), _ptr(W), _ptr(p.packed), _stream(stream)), "grinqh_pack")
     return p
 

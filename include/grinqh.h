@@ -4,15 +4,17 @@
  * GRINQH ("GRINQH: Graded Input-based Quantization Hierarchy for Efficient LLM
  * Generation", arXiv 2606.23419) speeds up batch-1 decoding by reading, for each
  * input channel k of a linear layer, only the b_k most significant bits of that
- * channel's 8-bit weights, where b_k is chosen per token from |x_k| against
- * calibrated thresholds (Section 3.1), and b_k = 0 skips the channel entirely.
+ * channel's b_max-bit weights (b_max = 8 by default; 2, 4 or 6 on request),
+ * where b_k is chosen per token from |x_k| against calibrated thresholds
+ * (Section 3.1), and b_k = 0 skips the channel entirely.
  * The weights are stored once, as MSB-first bit planes, so every narrower width
  * is a prefix of the wider one (Section 3.3, "Storage Layout and Weight
  * Loading").
  *
  * Calls, in the order a user makes them:
  *   grinqh_layout_init       sizes of the packed buffers for a K x N layer
- *   grinqh_pack              offline 8-bit RTN + bit-plane packing
+ *                            (grinqh_layout_init_bmax for b_max < 8)
+ *   grinqh_pack              offline b_max-bit RTN + bit-plane packing
  *   grinqh_maxent_distribution / grinqh_calibrate   thresholds for a target width
  *   grinqh_select            per-token grading + per-class channel lists
  *   grinqh_vmm               y = x . W_hat over the graded bit planes
@@ -43,7 +45,7 @@ extern "C" {
 
 #define GRINQH_GROUP 128       /* columns per (row, group) scale/zero pair */
 #define GRINQH_MAX_CLASSES 9   /* widths 0..8 */
-#define GRINQH_PLANES 8        /* b_max = 8 */
+#define GRINQH_PLANES 8        /* largest b_max (the default) */
 
 typedef enum {
   GRINQH_OK = 0,
@@ -55,16 +57,19 @@ typedef enum {
 } grinqh_status;
 
 /*
- * Physical layout of a packed K x N layer. Filled by grinqh_layout_init; treat
- * as read-only. One device buffer (packed_bytes, 16-byte aligned) holds the
- * layer. Each row is cut into n_tiles column tiles of tile_n = 1024 columns;
- * row k, tile t is one record of record_bytes = 1056 bytes at byte offset
+ * Physical layout of a packed K x N layer. Filled by grinqh_layout_init or
+ * grinqh_layout_init_bmax; treat as read-only. One device buffer (packed_bytes,
+ * 16-byte aligned) holds the layer. Each row is cut into n_tiles column tiles
+ * of tile_n = 1024 columns; row k, tile t is one record of record_bytes =
+ * 32 + 128 * b_max bytes (1056 for b_max = 8) at byte offset
  * (k*n_tiles + t)*record_bytes (a row's tiles are adjacent):
  *   bytes [0, 32)      8 uint32 words; word g is scale_fp16 | (zero_fp16 << 16)
  *                      of columns [t*1024 + 128g, +128) (0 past the last group);
- *   bytes [32, 1056)   the 8 bit planes, MSB first (plane p = 0 is bit 7 of the
- *                      code, p = 7 is bit 0), in 4 plane pairs: pair s holds
- *                      planes 2s and 2s+1 in bytes [32 + 256s, 32 + 256(s+1)).
+ *   bytes [32, ...)    the b_max bit planes of the b_max-bit codes, MSB first
+ *                      (plane p = 0 is bit b_max-1 of the code, p = b_max-1 is
+ *                      bit 0), in b_max/2 plane pairs (the paper's 2-bit
+ *                      segments): pair s holds planes 2s and 2s+1 in bytes
+ *                      [32 + 256s, 32 + 256(s+1)).
  * So the scale/zero words and the top b planes of a (row, tile) are one
  * contiguous, 32-byte-aligned run of 32 + 256 ceil(b/2) bytes (for odd b the
  * last pair's second plane is read and not used). Inside pair s, 32-bit word
@@ -78,7 +83,9 @@ typedef struct {
   int32_t n_groups;      /* ceil(N / 128) */
   int32_t tile_n;        /* columns per tile (1024) */
   int32_t n_tiles;       /* ceil(N / tile_n) */
-  int32_t record_bytes;  /* bytes per (row, tile) record (1056) */
+  int32_t record_bytes;  /* bytes per (row, tile) record: 32 + 128 * b_max */
+  int32_t b_max;         /* bits per stored code: 2, 4, 6 or 8 */
+  int32_t reserved;      /* 0 */
   int64_t packed_bytes;  /* K * n_tiles * record_bytes */
 } grinqh_layout;
 
@@ -89,19 +96,31 @@ const char* grinqh_version(void);
 const char* grinqh_status_string(grinqh_status s);
 
 /*
- * Fill *out with the packed layout of a K x N layer. Host only.
+ * Fill *out with the packed layout of a K x N layer of 8-bit codes. Host only.
  * Errors: INVALID_ARG for out == NULL or sizes outside the limits above.
  */
 grinqh_status grinqh_layout_init(int32_t K, int32_t N, grinqh_layout* out);
 
 /*
- * Offline 8-bit RTN quantisation and bit-plane packing.
+ * The same for codes of b_max bits. Paper: Section 3.3 ("each weight is
+ * quantized to a b_max-bit integer", stored as 2-bit segments, so widths
+ * b in {0, 2, ..., b_max} can be fetched; b_max in {4, 6, 8} is evaluated).
+ * This library takes any width 0..b_max (1-bit planes in pairs) and
+ * b_max in {2, 4, 6, 8}; grinqh_layout_init(K, N, out) is b_max = 8. Host only.
+ * Errors: INVALID_ARG for out == NULL, sizes outside the limits above or b_max
+ * not in {2, 4, 6, 8}.
+ */
+grinqh_status grinqh_layout_init_bmax(int32_t K, int32_t N, int32_t b_max, grinqh_layout* out);
+
+/*
+ * Offline b_max-bit RTN quantisation and bit-plane packing (b_max from the
+ * layout, L = 2^b_max - 1 levels; L = 255 for the default b_max = 8).
  * Paper: Section 3.3 (uniform b_max-bit quantisation, nested slices, input-major
  * storage), Section 4 (RTN, group size G = 128), Appendix C.1 (same-significance
  * bits of neighbouring weights packed into 32-bit words).
- * Per (row k, group g): s = fp16_rne((max - min) / 255) computed in fp64 and
+ * Per (row k, group g): s = fp16_rne((max - min) / L) computed in fp64 and
  * rounded straight to fp16 (s := 1 if it rounds to 0, s := 65504 if it
- * overflows); z = clamp(rne(-min / s), 0, 255); q = clamp(rne(w / s) + z, 0, 255),
+ * overflows); z = clamp(rne(-min / s), 0, L); q = clamp(rne(w / s) + z, 0, L),
  * quotients in fp64, ties to even.
  *   W       device, fp32 [K][N] row-major, finite values (non-finite input
  *           gives unspecified codes), 4-byte aligned.
@@ -112,13 +131,14 @@ grinqh_status grinqh_pack(const grinqh_layout* layout, const float* W, void* pac
 
 /*
  * Decode the codes the VMM uses, for testing the packed format. For each row k
- * with width b = bits[k] (8 for every row when bits == NULL):
+ * with width b = bits[k] (b_max for every row when bits == NULL):
  *   b = 0: code 0 (the row is never read by grinqh_vmm);
- *   1 <= b <= 7: c_b * 2^(8-b) + 2^(7-b), c_b = top b bits of q (Section 3.3
- *     reconstruction with its midpoint term);
- *   b = 8: q.
+ *   1 <= b < b_max: c_b * 2^(b_max-b) + 2^(b_max-b-1), c_b = top b bits of the
+ *     b_max-bit code q (Section 3.3 reconstruction with its midpoint term);
+ *   b = b_max: q.
  *   packed  device, as written by grinqh_pack for the same layout.
- *   bits    device uint8 [K] of widths 0..8, or NULL.
+ *   bits    device uint8 [K] of widths 0..b_max (a larger width decodes as
+ *           b_max), or NULL.
  *   codes   device uint8 [K][N] row-major; fully overwritten.
  * Errors: INVALID_ARG, ALIGNMENT, CUDA.
  */
@@ -193,13 +213,15 @@ grinqh_status grinqh_vmm_workspace_bytes(const grinqh_layout* layout, size_t* by
  * The graded vector-matrix product (the decode hot path).
  * Paper: Fig. 2 and Section 3.3: for every channel k with b_k > 0, only planes
  * 0..b_k-1 of row k (and its scale/zero words) are read; the row is rebuilt as
- * w_hat = s * (code - z) with code = c_b * 2^(8-b) + 2^(7-b) for b < 8 and q for
- * b = 8; channels with b_k = 0 are never read and add nothing.
+ * w_hat = s * (code - z) with code = c_b * 2^(b_max-b) + 2^(b_max-b-1) for
+ * b < b_max and q for b = b_max (b_max = 8 unless the layout says otherwise);
+ * channels with b_k = 0 are never read and add nothing.
  *   y[n] = sum_k x_k * w_hat[k][n], accumulated in fp32.
  *   packed        device, from grinqh_pack with this layout.
  *   x             device fp16 [K] (the same vector grinqh_select graded).
  *   idx, offsets  device, from grinqh_select with the same classes.
- *   classes       host uint8 [n_classes].
+ *   classes       host uint8 [n_classes]; every width at most the layout's
+ *                 b_max (INVALID_ARG otherwise).
  *   y             device fp32 [N], output (overwritten), 4-byte aligned.
  *   workspace     device, >= grinqh_vmm_workspace_bytes(layout) (a size that
  *                 depends on the current device's SM count), 16-byte aligned;

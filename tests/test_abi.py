@@ -122,3 +122,39 @@ def test_host_validation_rejects_before_launch(g):
                         None) == 1
     assert g._cal_ws(70000, 5, ctypes.byref(ws)) == 1
     assert g._cal_ws(128, 5, ctypes.byref(ws)) == 0 and ws.value >= 128 * 4 * 8
+
+
+def test_layout_bmax(g):
+    for bmax, rec in ((2, 288), (4, 544), (6, 800), (8, 1056)):
+        L = g.layout(4096, 4096, bmax)
+        assert (L.b_max, L.record_bytes, L.reserved) == (bmax, rec, 0)
+        assert L.record_bytes == 32 + 128 * bmax and L.record_bytes % 32 == 0
+        assert L.packed_bytes == 4096 * 4 * rec
+    assert g.layout(8, 8).b_max == 8
+    for bad in (0, 1, 3, 5, 7, 9, 16, -2):
+        with pytest.raises(g.GrinqhError) as e:
+            g.layout(8, 8, bad)
+        assert e.value.code == 1
+    assert g._layout_init_bmax(8, 8, 4, None) == 1
+
+
+def test_bmax_validation_rejects_before_launch(g):
+    P = ctypes.c_void_p
+    L = g.layout(64, 1024, 4)
+    need = g.vmm_workspace_bytes(L)
+    wide = (ctypes.c_uint8 * 4)(0, 2, 4, 6)      # a width above b_max = 4
+    ok = (ctypes.c_uint8 * 3)(0, 2, 4)
+    base = [ctypes.byref(L), P(0x1000), P(0x1000), P(0x1000), P(0x1000)]
+    assert g._vmm(*base, ctypes.addressof(wide), 4, P(0x1000), P(0x1000), need, None) == 1
+    assert g._vmm_noalloc(*base, ctypes.addressof(wide), 4, P(0x1000), None) == 1
+    assert g._select_vmm(ctypes.byref(L), P(0x1000), P(0x1000), P(0x1000), ctypes.addressof(wide), 4, P(0x1000),
+                         P(0x1000), need, None) == 1
+    # the same call with classes that fit fails only on the workspace it lacks
+    assert g._vmm(*base, ctypes.addressof(ok), 3, P(0x1000), None, need, None) == 4
+    # a layout whose b_max field was edited is not one grinqh_layout_init_bmax makes
+    L2 = g.layout(64, 1024, 4)
+    L2.b_max = 6
+    assert g._pack(ctypes.byref(L2), P(0x1000), P(0x1000), None) == 1
+    L3 = g.layout(64, 1024, 4)
+    L3.reserved = 1
+    assert g._pack(ctypes.byref(L3), P(0x1000), P(0x1000), None) == 1
