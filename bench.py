@@ -38,6 +38,11 @@ METRIC = "µs per batch-1 VMM and effective HBM GB/s (% of peak) vs average bits
 UNIT = "µs"
 TARGETS = (4.0, 3.0, 2.0)
 WORKLOAD = "llama3-8b decode linears (q,k,v,o,gate,up,down), batch 1, avg bits 4/3/2"
+# Stored code width and class set of the workload: b_max = 8 with classes
+# {0,2,3,4,8} by default; --bmax 4 or 6 stores b_max-bit codes and grades into
+# the paper's even classes {0, 2, ..., b_max} (Section 3.3, b_max in {4, 6, 8}).
+BMAX = 8
+CLASSES = None   # set in main()
 
 
 def _peaks():
@@ -132,7 +137,7 @@ def per_pair_us(ms_total, steps, pairs_per_step, world):
 def build_workload(g, wl, torch, dev, copies=2):
     """Pack `copies` x 3 (one per width) copies of the 7 linears, calibrate per
     linear and width, and draw one input vector per pair."""
-    classes = wl.CLASSES
+    classes = CLASSES
     pairs = []
     gen = torch.Generator(device=dev)
     for li, (name, K, N) in enumerate(wl.LLAMA3_8B):
@@ -145,7 +150,7 @@ def build_workload(g, wl, torch, dev, copies=2):
             for ti, t in enumerate(TARGETS):
                 gen.manual_seed(1_000_003 * (li + 1) + 7919 * c + 31 * ti)
                 W = torch.randn(K, N, generator=gen, device=dev, dtype=torch.float32) * 0.02
-                p = g.pack(W)
+                p = g.pack(W, b_max=BMAX)
                 del W
                 x = wl.activations_outlier(K, 1, key=(1, c, li, 2 + ti), chan_key=(1, 0, li))[0]
                 x_d = torch.from_numpy(x.view(np.int16)).to(dev)
@@ -195,7 +200,7 @@ def run_gpu(args):
 
     def step_pairs(c):
         for pr in groups[c]:
-            g.select(pr["x"], pr["th"], wl.CLASSES, out=pr["sel"], stream=stream)
+            g.select(pr["x"], pr["th"], CLASSES, out=pr["sel"], stream=stream)
             g.vmm(pr["packed"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
 
     def vmm_only(c):
@@ -206,7 +211,7 @@ def run_gpu(args):
     # the VMM kernel, no channel lists): reported beside the headline
     def fused_pairs(c):
         for pr in groups[c]:
-            g.select_vmm(pr["packed"], pr["x"], pr["th"], wl.CLASSES, pr["ws"], y=pr["y"], stream=stream)
+            g.select_vmm(pr["packed"], pr["x"], pr["th"], CLASSES, pr["ws"], y=pr["y"], stream=stream)
 
     # e2e: a step's inputs come from pinned host memory in one copy and its
     # outputs go back in one copy: every pair's x and y are views into one
@@ -233,7 +238,7 @@ def run_gpu(args):
         xs_dev, ys_dev, xs_pin, ys_pin = io[c]
         xs_dev.copy_(xs_pin, non_blocking=True)
         for pr in groups[c]:
-            g.select(pr["x"], pr["th"], wl.CLASSES, out=pr["sel"], stream=stream)
+            g.select(pr["x"], pr["th"], CLASSES, out=pr["sel"], stream=stream)
             g.vmm(pr["packed"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
         ys_pin.copy_(ys_dev, non_blocking=True)
 
@@ -335,7 +340,7 @@ def run_gpu(args):
             "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step / args.steps, 6), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "u8 planes, fp32 accumulate", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "pairs_per_step": n_pairs, "classes": list(wl.CLASSES),
+            "config": {"workload": WORKLOAD, "pairs_per_step": n_pairs, "classes": list(CLASSES), "b_max": BMAX,
                        "l2": "inputs larger than L2: every pair of a step reads its own packed copy; "
                              "%d copies of the layer set (%.2f GB) rotate" % (
                                  len(pairs), sum(pr["packed"].packed.numel() for pr in pairs) / 1e9),
@@ -370,7 +375,7 @@ def _oracle_sample(budget_s, nthreads):
     """Time oracle select + vmm on a bounded sample of the workload's pairs."""
     import oracle
     from activation_graded_bit_b200 import workloads as wl
-    classes = np.array(wl.CLASSES, np.uint8)
+    classes = np.array(CLASSES, np.uint8)
     done = 0
     secs = 0.0
     names = []
@@ -380,7 +385,7 @@ def _oracle_sample(budget_s, nthreads):
             break
         # untimed setup: weights, RTN codes, thresholds of this linear
         W = wl.weights_gaussian(K, N, key=(1, 9, li, 0))
-        q, s, z = oracle.rtn_quantize(W)
+        q, s, z = oracle.rtn_quantize(W, BMAX)
         del W
         Xc = wl.activations_outlier(K, 32, key=(1, 0, li, 1), chan_key=(1, 0, li))
         for ti, t in enumerate(TARGETS):
@@ -388,7 +393,7 @@ def _oracle_sample(budget_s, nthreads):
             x = wl.activations_outlier(K, 1, key=(1, 0, li, 2 + ti), chan_key=(1, 0, li))[0]
             t0 = time.perf_counter()
             bits, idx, off = oracle.select(x, th, classes)
-            oracle.vmm(x, q, s, z, bits, nthreads=nthreads)
+            oracle.vmm(x, q, s, z, bits, nthreads=nthreads, bmax=BMAX)
             secs += time.perf_counter() - t0
             done += 1
             names.append("%s@%g" % (name, t))
@@ -635,7 +640,15 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="average-bit sweep on a 14336x4096 layer (one JSON line)")
     ap.add_argument("--stack", action="store_true", help="32-layer linear stack tokens/s (one JSON line)")
     ap.add_argument("--stack-steps", type=int, default=256)
+    ap.add_argument("--bmax", type=int, default=8, choices=(4, 6, 8),
+                    help="stored code width; 4 or 6 grade into the classes {0, 2, ..., b_max}")
     args = ap.parse_args()
+    global BMAX, CLASSES, WORKLOAD
+    from activation_graded_bit_b200 import workloads as wl
+    BMAX = args.bmax
+    CLASSES = tuple(wl.CLASSES) if BMAX == 8 else tuple(range(0, BMAX + 1, 2))
+    if BMAX != 8:
+        WORKLOAD = WORKLOAD + ", b_max %d codes, classes %s" % (BMAX, "/".join(map(str, CLASSES)))
     if args.warmup < 3:
         args.warmup = 3
     if args.sweep:
