@@ -2,8 +2,8 @@
 
 GRINQH ("Graded Input-based Quantization Hierarchy", arXiv 2606.23419) grades
 every input channel of a linear layer per token by |x| against calibrated
-thresholds and reads only the top b bits of that channel's 8-bit weights from
-nested MSB-first bit planes.
+thresholds and reads only the top b bits of that channel's b_max-bit weights
+(8 by default; 2, 4 or 6 on request) from nested MSB-first bit planes.
 
 Modules:
   grinqh     ctypes binding of the C ABI (include/grinqh.h) in libgrinqh.so
