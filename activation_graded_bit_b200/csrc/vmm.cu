@@ -123,11 +123,6 @@ __device__ __forceinline__ RowAddr row_addr(const VmmArgs& a, int t, int w) {
   return ra;
 }
 
-// Ask L2 to fetch the cache line holding ptr (no register, no completion).
-__device__ __forceinline__ void prefetch_l2(const void* ptr) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
-}
-
 // Read-only load that skips L1 allocation (every weight word is read once).
 __device__ __forceinline__ uint32_t ld_stream(const void* ptr) {
   uint32_t v;
