@@ -59,6 +59,7 @@
 // y directly and no second kernel runs.
 #include <cstdint>
 #include <cuda_fp16.h>
+#include <atomic>
 #include <mutex>
 
 #include "async.cuh"
@@ -528,19 +529,28 @@ static cudaError_t launch_one(const cudaLaunchConfig_t& cfg, const VmmArgs& a, b
   return fused ? cudaLaunchKernelEx(&cfg, vmm_kernel<true, kBmax>, a) : cudaLaunchKernelEx(&cfg, vmm_kernel<false, kBmax>, a);
 }
 
-cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused) {
-  static bool attr_set[64] = {};
+// The kernels' shared-memory limit is raised once per device (with that device
+// current); calls from several host threads may race here, so the flag is atomic
+// and setting the attribute twice is harmless.
+static cudaError_t ensure_smem_attrs() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<bool> done[kMaxDevices];
   int dev = 0;
-  cudaGetDevice(&dev);
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = set_smem_attr<8>();
+  if (e == cudaSuccess) e = set_smem_attr<6>();
+  if (e == cudaSuccess) e = set_smem_attr<4>();
+  if (e == cudaSuccess) e = set_smem_attr<2>();
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev].store(true, std::memory_order_release);
+  return e;
+}
+
+cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused) {
   const int smem = (int)sizeof(VmmSmem);
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    cudaError_t e = set_smem_attr<8>();
-    if (e == cudaSuccess) e = set_smem_attr<6>();
-    if (e == cudaSuccess) e = set_smem_attr<4>();
-    if (e == cudaSuccess) e = set_smem_attr<2>();
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
+  cudaError_t ea = ensure_smem_attrs();
+  if (ea != cudaSuccess) return ea;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
