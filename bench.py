@@ -256,8 +256,19 @@ def run_gpu(args):
         torch.cuda.synchronize()
         return graphs
 
+    # the layers the 75%-of-HBM target is stated for: at least 4096 x 4096, 3-4
+    # average bits (q, o, gate, up, down at targets 4 and 3)
+    def big(pr):
+        return pr["K"] >= 4096 and pr["N"] >= 4096 and pr["target"] >= 3.0
+
+    def vmm_big(c):
+        for pr in groups[c]:
+            if big(pr):
+                g.vmm(pr["packed"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
+
     g_step = capture(step_pairs)
     g_vmm = capture(vmm_only)
+    g_big = capture(vmm_big)
     g_e2e = capture(e2e_pairs)
     g_fused = capture(fused_pairs)
 
@@ -290,6 +301,7 @@ def run_gpu(args):
     ms_vmm = timed(g_vmm, args.steps, args.warmup)
     ms_e2e = timed(g_e2e, args.steps, args.warmup)
     ms_fused = timed(g_fused, args.steps, args.warmup)
+    ms_big = timed(g_big, args.steps, args.warmup)
 
     # correctness spot check of the timed path (one pair) before reporting
     torch.cuda.synchronize()
@@ -307,6 +319,9 @@ def run_gpu(args):
                            mean_bits=round(mean_bits, 4), active_frac=round(active, 4),
                            planes_bytes=int(planes), alg_bytes=int(total)))
     peak, peak_kind = _peaks()
+    big_pairs = [pr for pr in groups[copies[0]] if big(pr)]
+    big_alg = sum(algorithmic_bytes(pr)[1] for pr in big_pairs)
+    achieved_big = big_alg * args.steps / (ms_big * 1e-3) / 1e9
     us_pair = ms_step * 1e3 / (args.steps * n_pairs)
     us_vmm = ms_vmm * 1e3 / (args.steps * n_pairs)
     achieved = tot_alg * args.steps / (ms_vmm * 1e-3) / 1e9
@@ -353,6 +368,12 @@ def run_gpu(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
                          "kernel": "grinqh vmm_kernel"},
+            "roofline_target_layers": {
+                "what": "grinqh_vmm on the layers of at least 4096 x 4096 at 3-4 average bits (q, o, gate, up, "
+                        "down at targets 4 and 3): algorithmic bytes / time of a graph of those %d calls" % len(big_pairs),
+                "us_per_vmm": round(ms_big * 1e3 / (args.steps * len(big_pairs)), 4),
+                "achieved": round(achieved_big, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved_big / peak, 4), "peak_kind": peak_kind},
             "points": points,
             "e2e": {"value": round(e2e_us, 4), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
@@ -363,7 +384,7 @@ def run_gpu(args):
             out["cpu_baseline"] = cpu
         print(json.dumps(out))
     # release graphs before tearing down the process group
-    del g_step, g_vmm, g_e2e
+    del g_step, g_vmm, g_e2e, g_big
     if world > 1:
         dist.destroy_process_group()
 
