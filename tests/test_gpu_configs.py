@@ -103,3 +103,30 @@ def test_linear_stack_slice(g, orc):
                 bits, _, _ = orc.select(x, d["th_ref"], cl)
                 yr, bound = orc.vmm(x, d["q"], d["s"], d["z"], bits)
                 assert_close(y.cpu().numpy()[d["cols"]], yr, bound, "layer %d %s step %d" % (layer, d["name"], step))
+
+
+@pytest.mark.parametrize("N", [6144, 28672])
+def test_grouped_linears_sampled_columns(g, orc, N):
+    # the stack's grouped shapes: [q|k|v] 4096 x 6144 and [gate|up] 4096 x 28672
+    # (28 column tiles, 5 row splits), one set of thresholds for the shared x
+    K = 4096
+    W = wl.weights_gaussian(K, N, key=(5, N, 0))
+    Xc = wl.activations_outlier(K, 128, key=(5, N, 1), chan_key=(5, N))
+    x = wl.activations_outlier(K, 1, key=(5, N, 2), chan_key=(5, N))[0]
+    p = g.pack(torch.from_numpy(W).cuda())
+    cl = np.array(CL, np.uint8)
+    P = orc.maxent_distribution(cl, 3.0)
+    th = g.calibrate(dev_u16(Xc), CL, P=P)
+    th_ref = orc.thresholds(Xc, P)
+    assert np.array_equal(th.cpu().numpy(), th_ref)
+    xd = dev_u16(x)
+    sel = g.select(xd, th, CL)
+    y = g.vmm(p, xd, sel, g.vmm_workspace(p.layout)).cpu().numpy()
+    yf = g.select_vmm(p, xd, th, CL, g.vmm_workspace(p.layout)).cpu().numpy()
+    bits, idx, off = orc.select(x, th_ref, cl)
+    assert np.array_equal(sel.bits.cpu().numpy(), bits)
+    cols = _cols(N, np.random.default_rng(N))
+    q, s, z = orc.rtn_quantize(W[:, cols])
+    yr, bound = orc.vmm(x, q, s, z, bits)
+    assert_close(y[cols], yr, bound, "grouped N=%d" % N)
+    assert_close(yf[cols], yr, bound, "grouped fused N=%d" % N)
