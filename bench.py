@@ -641,6 +641,10 @@ def run_stack(args):
             g.select(x, d["th"], classes, out=d["sel"], stream=st)
             g.vmm(d["p"], x, d["sel"], d["ws"], y=d["y"], stream=st)
 
+    def step_grp_fused(st, k):
+        for d in grp:
+            g.select_vmm(d["p"], xs[k][d["layer"]][d["src"]], d["th"], classes, d["ws"], y=d["y"], stream=st)
+
     def tokens_per_s(step):
         graphs = []
         with torch.cuda.stream(stream):
@@ -668,6 +672,7 @@ def run_stack(args):
 
     ms = tokens_per_s(step_sep)
     ms_g = tokens_per_s(step_grp)
+    ms_gf = tokens_per_s(step_grp_fused)
     assert all(bool(torch.isfinite(d["y"]).all()) for d in lin[:7] + grp[:4])
     packed_gb = sum(d["p"].packed.numel() for d in lin) / 1e9
     print(json.dumps({"metric": "linear-stack tokens/s (32 x 7 Llama3-8B linears, batch 1, 3 average bits)",
@@ -680,7 +685,12 @@ def run_stack(args):
                                   "ms_per_token": round(ms_g / args.stack_steps, 4),
                                   "what": "same weights, [q|k|v] and [gate|up] concatenated along N, thresholds "
                                           "per input vector: 4 select + VMM pairs per layer",
-                                  "gpu_launches_per_token": 2 * len(grp) + sum(1 for d in grp if d["ws"].numel() > 16)}}))
+                                  "gpu_launches_per_token": 2 * len(grp) + sum(1 for d in grp if d["ws"].numel() > 16)},
+                      "grouped_fused": {"value": round(args.stack_steps / (ms_gf * 1e-3), 2), "unit": "tokens/s",
+                                        "ms_per_token": round(ms_gf / args.stack_steps, 4),
+                                        "what": "the grouped stack through grinqh_select_vmm (grading inside the "
+                                                "VMM kernel, no channel lists): 4 calls per layer",
+                                        "gpu_launches_per_token": len(grp) + sum(1 for d in grp if d["ws"].numel() > 16)}}))
 
 def main():
     ap = argparse.ArgumentParser()
