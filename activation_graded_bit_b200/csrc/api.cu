@@ -16,6 +16,7 @@ namespace {
 
 constexpr int64_t kMaxDim = int64_t(1) << 24;
 constexpr int64_t kMaxElems = int64_t(1) << 34;
+constexpr int32_t kMaxTokens = 65535;   // tokens of a batched call: one grid dimension
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -315,6 +316,43 @@ grinqh_status grinqh_select_vmm(const grinqh_layout* layout, const void* packed,
   a.status = (uint32_t*)workspace;
   a.partial = (float*)((char*)workspace + 16);
   a.ct = table(classes, n_classes);
+  return cuda_status(launch_vmm(a, (cudaStream_t)stream, true));
+}
+
+grinqh_status grinqh_vmm_batch_workspace_bytes(const grinqh_layout* layout, int32_t tokens, size_t* bytes) {
+  if (!layout_ok(layout) || !bytes || tokens < 1 || tokens > kMaxTokens) return GRINQH_ERR_INVALID_ARG;
+  *bytes = vmm_workspace_bytes_batch(layout->n_tiles, tokens);
+  return GRINQH_OK;
+}
+
+grinqh_status grinqh_select_vmm_batch(const grinqh_layout* layout, const void* packed, const uint16_t* X,
+                                      int32_t tokens, const float* thresholds, const uint8_t* classes,
+                                      int32_t n_classes, float* Y, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  if (!layout_ok(layout) || !valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
+  if (!classes_fit(classes, n_classes, layout->b_max)) return GRINQH_ERR_INVALID_ARG;
+  if (tokens < 1 || tokens > kMaxTokens) return GRINQH_ERR_INVALID_ARG;
+  if (!packed || !X || !Y || (n_classes > 1 && !thresholds)) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(X, 2) || !aligned(Y, 4) || (thresholds && !aligned(thresholds, 4)))
+    return GRINQH_ERR_ALIGNMENT;
+  const grinqh_layout& L = *layout;
+  if (L.K > vmm_fused_max_k()) return GRINQH_ERR_UNSUPPORTED;
+  const size_t need = vmm_workspace_bytes_batch(L.n_tiles, tokens);
+  if (!workspace || workspace_bytes < need) return GRINQH_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return GRINQH_ERR_ALIGNMENT;
+  VmmArgs a{};
+  a.K = L.K;
+  a.N = L.N;
+  a.n_tiles = L.n_tiles;
+  a.b_max = L.b_max;
+  a.packed = (const uint8_t*)packed;
+  a.x = X;
+  a.thresholds = thresholds;
+  a.y = Y;
+  a.status = (uint32_t*)workspace;
+  a.partial = (float*)((char*)workspace + 16);
+  a.ct = table(classes, n_classes);
+  a.tokens = tokens;
   return cuda_status(launch_vmm(a, (cudaStream_t)stream, true));
 }
 

@@ -31,11 +31,14 @@ struct VmmArgs {
   const float* thresholds;   // fused grading only: the n_classes - 1 thresholds
   float* y;
   uint32_t* status;     // workspace: sticky error word (bit 0: a bounded wait timed out)
-  float* partial;       // workspace: per-row-split partial sums [R][n_tiles * 1024]
+  float* partial;       // workspace: per-row-split partial sums [tokens][R][n_tiles * 1024]
   ClassTable ct;
+  int tokens;           // batch: token t reads x + t K and writes y + t N (1 for a single vector)
 };
 
 size_t vmm_workspace_bytes(int n_tiles, int tile_n);
+// Workspace of a batch of T tokens: the status word, then T sets of partials.
+size_t vmm_workspace_bytes_batch(int n_tiles, int tokens);
 // fused = true: the kernel grades x itself (a.thresholds) instead of reading
 // a.idx / a.offsets; K <= vmm_fused_max_k().
 cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused = false);

@@ -104,6 +104,7 @@ struct RowRegs {
 // layout has K * N <= 2^34, so K * n_tiles <= 2^25) and one wide multiply-add
 // each of this lane's addresses in it.
 struct RowAddr {
+  const uint16_t* x;      // this CTA's token's activation vector
   const uint8_t* meta;    // packed + this lane's scale/zero word within a record
   const uint8_t* pairs;   // packed + this lane's two words of pair 0 within a record
   const uint8_t* lines;   // packed + 128 * lane (the lane's L2 line within a record prefix)
@@ -115,6 +116,7 @@ __device__ __forceinline__ RowAddr row_addr(const VmmArgs& a, int t, int w) {
   const uint32_t kSectors = (uint32_t)record_bytes_for(a.b_max) / 32u;   // 9, 17, 25 or 33
   static_assert(kMetaBytes % 32 == 0 && kPlaneBytes % 16 == 0, "records are whole 32-byte sectors");
   RowAddr ra;
+  ra.x = a.x + (size_t)blockIdx.z * a.K;
   ra.meta = a.packed + 4 * (w >> 2);
   ra.pairs = a.packed + kMetaBytes + 8 * w;
   ra.lines = a.packed + 128 * w;
@@ -199,7 +201,7 @@ __device__ __forceinline__ void load_row(const VmmArgs& a, const RowAddr& ra, ui
   const uint32_t sec = k * ra.nt33 + ra.t33;                  // record offset in 32-byte sectors
   r.b = b;
   r.m = ld_stream(ra.meta + 32ull * sec);
-  r.xh = __ldg(a.x + k);
+  r.xh = __ldg(ra.x + k);
   const uint8_t* pw = ra.pairs + 32ull * sec;                  // this lane's two words of pair 0
   ld_stream2_at<0>(pw, r.p[0], r.p[1]);
   ld_stream2_at_if<1 * kPairBytes>(b > 2, pw, r.p[2], r.p[3]);
@@ -282,6 +284,7 @@ __device__ __forceinline__ int stage_fused(const VmmArgs& a, VmmSmem& s, int r, 
   for (int q = 0; q < 8; ++q) th[q] = (q < nt) ? __ldg(a.thresholds + q) : 0.0f;
   const int nk = (a.K > r) ? (a.K - r + R - 1) / R : 0;
   const uint32_t lt = (1u << lane) - 1u;
+  const uint16_t* xt = a.x + (size_t)blockIdx.z * a.K;   // this CTA's token
   int base = 0;
 #pragma unroll 1
   for (int i0 = 0, rnd = 0; i0 < nk; i0 += kThreads, rnd ^= 1) {
@@ -290,7 +293,7 @@ __device__ __forceinline__ int stage_fused(const VmmArgs& a, VmmSmem& s, int r, 
     bool keep = false;
     if (i < nk) {
       const int k = r + R * i;
-      const float ax = fabsf(__half2float(__ushort_as_half(__ldg(a.x + k))));
+      const float ax = fabsf(__half2float(__ushort_as_half(__ldg(xt + k))));
       int c = 0;
 #pragma unroll
       for (int q = 0; q < 8; ++q) c += (q < nt && ax >= th[q]) ? 1 : 0;
@@ -442,7 +445,9 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
   __syncthreads();
   // partial[r][column], or y itself when there is a single row split; every
   // column of the tile is written, zeros included, so no clearing is needed
-  float* out = (R == 1) ? a.y : a.partial + (size_t)r * a.n_tiles * kTileN;
+  // (token blockIdx.z: its y row and its set of partials)
+  const size_t tok = blockIdx.z;
+  float* out = (R == 1) ? a.y + tok * a.N : a.partial + (tok * R + r) * a.n_tiles * kTileN;
   const int limit = (R == 1) ? a.N : a.n_tiles * kTileN;
 #pragma unroll
   for (int e = tid; e < kTileN; e += kThreads) {
@@ -469,6 +474,8 @@ __global__ void __launch_bounds__(32 * kRedChains) reduce_partials_kernel(const 
   pdl_wait();   // the partials come from the VMM kernel just before
   const int lane = threadIdx.x & 31, chain = threadIdx.x >> 5;
   const int col = blockIdx.x * 32 + lane;
+  partial += (size_t)blockIdx.y * R * stride;   // token blockIdx.y
+  y += (size_t)blockIdx.y * N;
   float v = 0.0f;
   if (col < N) {
     for (int r0 = chain; r0 < R; r0 += kRedChains * kRedLoads) {
@@ -509,11 +516,13 @@ static int row_splits(int n_tiles) {
   return R < 1 ? 1 : R;
 }
 
-// status word (16 B), then partial[R][n_tiles * 1024] floats when R > 1
-size_t vmm_workspace_bytes(int n_tiles, int /*tile_n*/) {
+// status word (16 B), then partial[tokens][R][n_tiles * 1024] floats when R > 1
+size_t vmm_workspace_bytes_batch(int n_tiles, int tokens) {
   const int R = row_splits(n_tiles);
-  return 16 + (R > 1 ? (size_t)R * n_tiles * kTileN * sizeof(float) : 0);
+  return 16 + (R > 1 ? (size_t)tokens * R * n_tiles * kTileN * sizeof(float) : 0);
 }
+
+size_t vmm_workspace_bytes(int n_tiles, int /*tile_n*/) { return vmm_workspace_bytes_batch(n_tiles, 1); }
 
 template <int kBmax>
 static cudaError_t set_smem_attr() {
@@ -557,7 +566,7 @@ cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused) {
 
   const int R = row_splits(a.n_tiles);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.n_tiles, R, 1);
+  cfg.gridDim = dim3(a.n_tiles, R, a.tokens > 1 ? a.tokens : 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -574,7 +583,7 @@ cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused) {
   if (e != cudaSuccess || R == 1) return e;
 
   cudaLaunchConfig_t rc = {};
-  rc.gridDim = dim3((a.N + 31) / 32, 1, 1);
+  rc.gridDim = dim3((a.N + 31) / 32, a.tokens > 1 ? a.tokens : 1, 1);
   rc.blockDim = dim3(32 * kRedChains, 1, 1);
   rc.stream = st;
   rc.attrs = attr;

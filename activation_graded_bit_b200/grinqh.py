@@ -67,12 +67,15 @@ _vmm_ws = _sig("grinqh_vmm_workspace_bytes", [_LP, ctypes.POINTER(ctypes.c_size_
 _vmm = _sig("grinqh_vmm", [_LP, _P, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
 _vmm_noalloc = _sig("grinqh_vmm_noalloc", [_LP, _P, _P, _P, _P, _P, _I, _P, _P])
 _select_vmm = _sig("grinqh_select_vmm", [_LP, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
+_batch_ws = _sig("grinqh_vmm_batch_workspace_bytes", [_LP, _I, ctypes.POINTER(ctypes.c_size_t)])
+_select_vmm_batch = _sig("grinqh_select_vmm_batch", [_LP, _P, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
 
 # Every exported symbol of the C ABI, for the export check in the tests.
 EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grinqh_layout_init_bmax", "grinqh_pack",
            "grinqh_unpack_codes", "grinqh_maxent_distribution", "grinqh_calibrate_workspace_bytes",
            "grinqh_calibrate", "grinqh_select", "grinqh_vmm_workspace_bytes", "grinqh_vmm",
-           "grinqh_vmm_noalloc", "grinqh_select_vmm")
+           "grinqh_vmm_noalloc", "grinqh_select_vmm", "grinqh_vmm_batch_workspace_bytes",
+           "grinqh_select_vmm_batch")
 
 
 def version() -> str:
@@ -246,6 +249,29 @@ def select_vmm(p: PackedLayer, x: torch.Tensor, thresholds: Optional[torch.Tenso
                        _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
            "grinqh_select_vmm")
     return y
+
+
+def vmm_batch_workspace(L: Layout, tokens: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace for grinqh_select_vmm_batch with this many tokens."""
+    v = ctypes.c_size_t()
+    _check(_batch_ws(ctypes.byref(L), int(tokens), ctypes.byref(v)), "grinqh_vmm_batch_workspace_bytes")
+    return torch.zeros(v.value, dtype=torch.uint8, device=device)
+
+
+def select_vmm_batch(p: PackedLayer, X: torch.Tensor, thresholds: Optional[torch.Tensor], classes: Sequence[int],
+                     workspace: torch.Tensor, Y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """grinqh_select_vmm_batch: X is a contiguous [T, K] CUDA tensor of fp16 (or its
+    16-bit bit view); returns Y fp32 [T, N], row t as grinqh_select_vmm gives for X[t]."""
+    assert X.is_cuda and X.dim() == 2 and X.is_contiguous() and X.element_size() == 2 and X.shape[1] == p.K
+    T = X.shape[0]
+    if Y is None:
+        Y = torch.empty((T, p.N), dtype=torch.float32, device=X.device)
+    cb, n = _classes_buf(classes)
+    _check(_select_vmm_batch(ctypes.byref(p.layout), _ptr(p.packed), _ptr(X), T, _ptr(thresholds),
+                             ctypes.addressof(cb), n, _ptr(Y), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)),
+           "grinqh_select_vmm_batch")
+    return Y
 
 
 def vmm_noalloc(p: PackedLayer, x: torch.Tensor, sel: Selection, y: torch.Tensor, stream=None) -> torch.Tensor:

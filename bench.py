@@ -692,6 +692,66 @@ def run_stack(args):
                                                 "VMM kernel, no channel lists): 4 calls per layer",
                                         "gpu_launches_per_token": len(grp) + sum(1 for d in grp if d["ws"].numel() > 16)}}))
 
+def run_batch(args):
+    """Batch > 1 through grinqh_select_vmm_batch on the Llama3-8B step (21
+    (linear, width) pairs, two packed copies rotated): for T tokens per call,
+    microseconds per call and per token, graph-replayed; the T activation
+    vectors of a pair are drawn like the batch-1 ones."""
+    import torch
+    from activation_graded_bit_b200 import grinqh as g
+    from activation_graded_bit_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    pairs = build_workload(g, wl, torch, dev, copies=2)
+    groups = {}
+    for pr in pairs:
+        groups.setdefault(pr["copy"], []).append(pr)
+    copies = sorted(groups)
+    stream = torch.cuda.Stream(device=dev)
+    out = []
+    for T in (1, 2, 4, 8, 16):
+        for pr in pairs:
+            X = wl.activations_outlier(pr["K"], T, key=(7, pr["copy"], T, pr["K"], pr["N"], int(pr["target"])),
+                                       chan_key=(1, 0, 0))
+            pr["X"] = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).to(dev)
+            pr["Y"] = torch.empty((T, pr["N"]), dtype=torch.float32, device=dev)
+            pr["wsT"] = g.vmm_batch_workspace(pr["packed"].layout, T, dev)
+
+        def step(c):
+            for pr in groups[c]:
+                g.select_vmm_batch(pr["packed"], pr["X"], pr["th"], CLASSES, pr["wsT"], Y=pr["Y"], stream=stream)
+        graphs = {}
+        with torch.cuda.stream(stream):
+            for c in copies:
+                step(c)
+            torch.cuda.synchronize()
+            for c in copies:
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=stream):
+                    step(c)
+                graphs[c] = gr
+            for i in range(args.warmup):
+                graphs[copies[i % len(copies)]].replay()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            steps = max(args.steps // 10, 20)
+            e0.record(stream)
+            for i in range(steps):
+                graphs[copies[i % len(copies)]].replay()
+            e1.record(stream)
+        stream.synchronize()
+        us_call = e0.elapsed_time(e1) * 1e3 / (steps * len(groups[copies[0]]))
+        out.append({"tokens": T, "us_per_call": round(us_call, 3), "us_per_token": round(us_call / T, 3)})
+        del graphs
+        assert all(bool(torch.isfinite(pr["Y"]).all()) for pr in groups[copies[0]])
+    print(json.dumps({"metric": "grinqh_select_vmm_batch: us per (linear, width) call and per token vs batch size",
+                      "unit": "µs", "higher_is_better": False, "data": "synthetic",
+                      "config": {"workload": WORKLOAD.replace("batch 1", "batch 1..16"), "classes": list(CLASSES),
+                                 "b_max": BMAX, "l2": "two packed copies of the layer set rotate"},
+                      "points": out}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -707,6 +767,7 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="average-bit sweep on a 14336x4096 layer (one JSON line)")
     ap.add_argument("--stack", action="store_true", help="32-layer linear stack tokens/s (one JSON line)")
     ap.add_argument("--stack-steps", type=int, default=256)
+    ap.add_argument("--batch", action="store_true", help="batch 1..16 through the batched fused call (one JSON line)")
     ap.add_argument("--bmax", type=int, default=8, choices=(4, 6, 8),
                     help="stored code width; 4 or 6 grade into the classes {0, 2, ..., b_max}")
     args = ap.parse_args()
@@ -723,6 +784,9 @@ def main():
         return
     if args.stack:
         run_stack(args)
+        return
+    if args.batch:
+        run_batch(args)
         return
     if args.profile:
         run_profile_case(args)

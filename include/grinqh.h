@@ -265,6 +265,32 @@ grinqh_status grinqh_select_vmm(const grinqh_layout* layout, const void* packed,
                                 const float* thresholds, const uint8_t* classes, int32_t n_classes,
                                 float* y, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Workspace bytes grinqh_select_vmm_batch needs for a layout and a token count. */
+grinqh_status grinqh_vmm_batch_workspace_bytes(const grinqh_layout* layout, int32_t tokens, size_t* bytes);
+
+/*
+ * grinqh_select_vmm for a batch of tokens in one launch: row t of Y is exactly
+ * what grinqh_select_vmm gives for row t of X (the same bits). Paper: Section
+ * 3.1 (every token grades every channel from its own |x|) and Section 6, which
+ * states that the method targets batch size one; this library's reading for a
+ * batch keeps every token's grading and reconstruction as at batch one. The
+ * tokens' CTAs run one token after another on the same weights, so a row that
+ * several tokens need is read from DRAM about once (the union of the tokens'
+ * widths) and from L2 after that, as long as the layer's graded bytes fit in L2.
+ *   X            device fp16 [tokens][K] row-major, 2-byte aligned.
+ *   tokens       1..65535.
+ *   Y            device fp32 [tokens][N] row-major, output (overwritten).
+ *   thresholds   as grinqh_select_vmm (shared by every token).
+ *   workspace    device, >= grinqh_vmm_batch_workspace_bytes(layout, tokens),
+ *                16-byte aligned, first 16 bytes zero-filled once before first use.
+ * Limit: K <= 16384 (GRINQH_ERR_UNSUPPORTED above).
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+grinqh_status grinqh_select_vmm_batch(const grinqh_layout* layout, const void* packed, const uint16_t* X,
+                                      int32_t tokens, const float* thresholds, const uint8_t* classes,
+                                      int32_t n_classes, float* Y, void* workspace, size_t workspace_bytes,
+                                      void* stream);
+
 /*
  * grinqh_vmm without a caller-provided workspace. The paper has no counterpart:
  * this is a calling convention of the library, not a step of the method.

@@ -158,3 +158,26 @@ def test_bmax_validation_rejects_before_launch(g):
     L3 = g.layout(64, 1024, 4)
     L3.reserved = 1
     assert g._pack(ctypes.byref(L3), P(0x1000), P(0x1000), None) == 1
+
+
+def test_batch_validation_rejects_before_launch(g):
+    P = ctypes.c_void_p
+    cl = (ctypes.c_uint8 * 5)(0, 2, 3, 4, 8)
+    L = g.layout(64, 1024)
+    ws = ctypes.c_size_t()
+    assert g._batch_ws(ctypes.byref(L), 0, ctypes.byref(ws)) == 1
+    assert g._batch_ws(ctypes.byref(L), 65536, ctypes.byref(ws)) == 1
+    assert g._batch_ws(ctypes.byref(L), 3, ctypes.byref(ws)) == 0
+    need3 = ws.value
+    assert g._batch_ws(ctypes.byref(L), 1, ctypes.byref(ws)) == 0
+    assert ws.value == g.vmm_workspace_bytes(L)
+    assert need3 - 16 == 3 * (ws.value - 16)          # one set of partials per token
+    base = [ctypes.byref(L), P(0x1000), P(0x1000)]
+    rest = [P(0x1000), ctypes.addressof(cl), 5, P(0x1000)]
+    assert g._select_vmm_batch(*base, 0, *rest, P(0x1000), need3, None) == 1            # no tokens
+    assert g._select_vmm_batch(*base, 3, *rest, P(0x1000), need3 - 1, None) == 4        # workspace short
+    assert g._select_vmm_batch(*base, 3, P(0x1000), ctypes.addressof(cl), 5, P(0x1002), P(0x1000), need3,
+                               None) == 2                                                # Y misaligned
+    Lbig = g.layout(20000, 64)
+    assert g._select_vmm_batch(ctypes.byref(Lbig), P(0x1000), P(0x1000), 2, *rest, P(0x1000), 1 << 30,
+                               None) == 3                                                # K above the fused limit
