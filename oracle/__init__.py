@@ -37,10 +37,11 @@ def lib():
         L.orc_compact.argtypes = [P, i32, P, i32, P, P]
         L.orc_vmm.argtypes = [P, P, P, P, P, i32, i32, P, P, i32]
         L.orc_vmm_bmax.argtypes = [P, P, P, P, P, i32, i32, i32, P, P, i32]
+        L.orc_dequant_f16.argtypes = [P, P, P, i32, i32, P]
         L.orc_maxent_distribution.argtypes = [P, i32, ctypes.c_double, P]
         L.orc_thresholds.argtypes = [P, i32, i32, P, i32, P]
         for f in ("orc_rtn_quantize", "orc_rtn_quantize_bmax", "orc_code", "orc_code_bmax", "orc_grade",
-                  "orc_compact", "orc_vmm", "orc_vmm_bmax",
+                  "orc_compact", "orc_vmm", "orc_vmm_bmax", "orc_dequant_f16",
                   "orc_maxent_distribution", "orc_thresholds"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -164,3 +165,25 @@ def select(x_bits, theta, classes):
     bits = grade(x_bits, theta, classes)
     idx, off = compact(bits, classes)
     return bits, idx, off
+
+
+def dequant_f16(q, scale, zero):
+    """Full-width weights rounded once to binary16, w_hat = s (q - z) (Section 4,
+    prefill at b_max; Section 3.3): uint16 bit patterns [K, N]."""
+    q = _c(q, np.uint8)
+    scale = _c(scale, np.uint16)
+    zero = _c(zero, np.uint16)
+    K, N = q.shape
+    out = np.empty((K, N), np.uint16)
+    if lib().orc_dequant_f16(_p(q), _p(scale), _p(zero), K, N, _p(out)) != 0:
+        raise ValueError("bad sizes")
+    return out
+
+
+def prefill(X_bits, w16):
+    """Dense prefill product in fp64: Y[t, n] = sum_k x[t, k] * w16[k, n] over the
+    binary16 operands (a library matmul on their exact fp64 values), and the
+    tolerance scale bound[t, n] = sum_k |x[t, k] * w16[k, n]|."""
+    Xf = np.ascontiguousarray(X_bits, np.uint16).view(np.float16).astype(np.float64)
+    Wf = np.ascontiguousarray(w16, np.uint16).view(np.float16).astype(np.float64)
+    return Xf @ Wf, np.abs(Xf) @ np.abs(Wf)

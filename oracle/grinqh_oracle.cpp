@@ -148,6 +148,29 @@ int orc_code_bmax(int q, int b, int bmax) {
 int orc_code(int q, int b) { return orc_code_bmax(q, b, 8); }
 
 // ---------------------------------------------------------------------------
+// Full-width dequantisation for the prefill product.
+// Paper: Section 4 ("Prefill vs. Decoding Evaluation": prefill unpacks the
+// weights at full b_max precision and runs a dense matrix-matrix product) and
+// Section 3.3 (w_hat = s * (q - z) at b = b_max). Library reading: the dense
+// operand is w_hat rounded once to binary16 (round to nearest even), computed
+// as the exact fp64 product s * (q - z) (an 11-bit by 9-bit product).
+// q[K*N] codes of b_max bits, scale/zero [K*n_g] fp16 bit patterns; out[K*N]
+// binary16 bit patterns. Returns 0, or -1 on bad sizes.
+// ---------------------------------------------------------------------------
+int orc_dequant_f16(const uint8_t* q, const uint16_t* scale, const uint16_t* zero, int K, int N,
+                    uint16_t* out) {
+  if (K <= 0 || N <= 0) return -1;
+  const int ng = (N + 127) / 128;
+  for (int k = 0; k < K; ++k)
+    for (int n = 0; n < N; ++n) {
+      const double s = orc_f16_to_f64(scale[(size_t)k * ng + n / 128]);
+      const double z = orc_f16_to_f64(zero[(size_t)k * ng + n / 128]);
+      out[(size_t)k * N + n] = orc_f64_to_f16(s * ((double)q[(size_t)k * N + n] - z));
+    }
+  return 0;
+}
+
+// ---------------------------------------------------------------------------
 // Grading. Paper: Section 3.1 "Dynamic Precision Assignment": b_i = b_k when
 // |x_i| lies in [theta_k, theta_{k+1}) with theta_0 = 0 and theta_{n+1} = inf.
 // Written as a count: class j = #{ i in 1..n : |x| >= theta_i }, which equals
