@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libgrinqh.so")
-SOURCES = ["api.cu", "pack.cu", "select.cu", "vmm.cu", "calibrate.cu"]
+SOURCES = ["api.cu", "pack.cu", "select.cu", "vmm.cu", "calibrate.cu", "prefill.cu"]
 HEADERS = ["common.cuh", "kernels.h", "async.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -43,7 +43,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
             sys.stderr.write(r.stderr)
         objs.append(obj)
     cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", LIB + ".tmp",
-           "-lcudart"]
+           "-lcudart", "-lcublas"]
     subprocess.check_call(cmd)
     os.replace(LIB + ".tmp", LIB)
     return LIB

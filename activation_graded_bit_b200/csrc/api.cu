@@ -126,6 +126,24 @@ grinqh_status grinqh_unpack_codes(const grinqh_layout* layout, const void* packe
   return cuda_status(launch_unpack(packed, bits, L.K, L.N, L.n_tiles, L.b_max, codes, (cudaStream_t)stream));
 }
 
+grinqh_status grinqh_dequant(const grinqh_layout* layout, const void* packed, uint16_t* W16, void* stream) {
+  if (!layout_ok(layout) || !packed || !W16) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(W16, 16)) return GRINQH_ERR_ALIGNMENT;
+  const grinqh_layout& L = *layout;
+  return cuda_status(launch_dequant(packed, L.K, L.N, L.n_tiles, L.b_max, W16, (cudaStream_t)stream));
+}
+
+grinqh_status grinqh_prefill(const grinqh_layout* layout, const void* packed, const uint16_t* X, int32_t T,
+                             float* Y, uint16_t* W16, void* stream) {
+  if (!layout_ok(layout) || !packed || !X || !Y || !W16) return GRINQH_ERR_INVALID_ARG;
+  if (T < 1 || T > kMaxDim) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(W16, 16) || !aligned(X, 2) || !aligned(Y, 4)) return GRINQH_ERR_ALIGNMENT;
+  const grinqh_layout& L = *layout;
+  cudaError_t e = launch_dequant(packed, L.K, L.N, L.n_tiles, L.b_max, W16, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = launch_prefill_gemm(X, W16, Y, T, L.K, L.N, (cudaStream_t)stream);
+  return cuda_status(e);
+}
+
 grinqh_status grinqh_maxent_distribution(const uint8_t* classes, int32_t n_classes, double target_bits,
                                          double* P) {
   if (!valid_classes(classes, n_classes) || !P) return GRINQH_ERR_INVALID_ARG;

@@ -13,6 +13,15 @@ cudaError_t launch_pack(const float* W, int K, int N, int n_tiles, int n_groups,
 cudaError_t launch_unpack(const void* packed, const uint8_t* bits, int K, int N, int n_tiles, int b_max,
                           uint8_t* codes, cudaStream_t st);
 
+// Full-width w_hat = s (q - z) as binary16, [K][N] row-major.
+cudaError_t launch_dequant(const void* packed, int K, int N, int n_tiles, int b_max, uint16_t* out,
+                           cudaStream_t st);
+
+// Y[T][N] (fp32) = X[T][K] (fp16) . W16[K][N] (fp16), fp32 accumulation, on the
+// stream (a plain library GEMM).
+cudaError_t launch_prefill_gemm(const uint16_t* X, const uint16_t* W16, float* Y, int T, int K, int N,
+                                cudaStream_t st);
+
 struct ClassTable {
   int n;              // number of classes (1..9)
   uint8_t width[9];   // bit width of class j

@@ -152,6 +152,65 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
     }
 }
 
+// Full-width dequantisation for the prefill product: one warp per (row, tile)
+// record, 8 records per CTA; lane w rebuilds its 32 columns at b_max and writes
+// w_hat = s (q - z) rounded once to binary16 (the fp32 product of an 11-bit
+// scale and a 9-bit code difference is exact). A lane's 32 columns are 64
+// contiguous bytes, written as four 16-byte stores when the row allows it.
+template <int B>
+__device__ __forceinline__ void dequant_record(const uint8_t* rec, int w, int k, int N, int n0,
+                                               __half* __restrict__ out) {
+  uint32_t R[8];
+  decode_word<B>(rec, w, B, R);
+  const uint32_t m = reinterpret_cast<const uint32_t*>(rec)[w >> 2];   // this lane's group's scale | zero
+  const float s = __half2float(__ushort_as_half((unsigned short)(m & 0xFFFFu)));
+  const float z = __half2float(__ushort_as_half((unsigned short)(m >> 16)));
+  __half2 h[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float c0 = (float)(R[j] & 0xFFu), c1 = (float)((R[j] >> 8) & 0xFFu);
+    const float c2 = (float)((R[j] >> 16) & 0xFFu), c3 = (float)(R[j] >> 24);
+    h[2 * j] = __floats2half2_rn(s * (c0 - z), s * (c1 - z));
+    h[2 * j + 1] = __floats2half2_rn(s * (c2 - z), s * (c3 - z));
+  }
+  __half* row = out + (size_t)k * N;
+  if (n0 + 32 <= N && (N & 7) == 0) {
+    uint4* dst = reinterpret_cast<uint4*>(row + n0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      dst[q] = make_uint4(*reinterpret_cast<const uint32_t*>(&h[4 * q]), *reinterpret_cast<const uint32_t*>(&h[4 * q + 1]),
+                          *reinterpret_cast<const uint32_t*>(&h[4 * q + 2]), *reinterpret_cast<const uint32_t*>(&h[4 * q + 3]));
+  } else {
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+      if (n0 + c < N) row[n0 + c] = (c & 1) ? __high2half(h[c >> 1]) : __low2half(h[c >> 1]);
+  }
+}
+
+__global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict__ packed, int K, int N, int n_tiles,
+                                                      int b_max, __half* __restrict__ out) {
+  const int t = blockIdx.y;
+  const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int w = threadIdx.x & 31;
+  if (k >= K) return;
+  const uint8_t* rec = packed + ((size_t)k * n_tiles + t) * record_bytes_for(b_max);
+  const int n0 = t * kTileN + 32 * w;
+  if (n0 >= N) return;
+  switch (b_max) {
+    case 2: dequant_record<2>(rec, w, k, N, n0, out); break;
+    case 4: dequant_record<4>(rec, w, k, N, n0, out); break;
+    case 6: dequant_record<6>(rec, w, k, N, n0, out); break;
+    default: dequant_record<8>(rec, w, k, N, n0, out); break;
+  }
+}
+
+cudaError_t launch_dequant(const void* packed, int K, int N, int n_tiles, int b_max, uint16_t* out,
+                           cudaStream_t st) {
+  dim3 grid((K + 7) / 8, n_tiles);
+  dequant_kernel<<<grid, 256, 0, st>>>((const uint8_t*)packed, K, N, n_tiles, b_max, reinterpret_cast<__half*>(out));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_pack(const float* W, int K, int N, int n_tiles, int n_groups, int b_max, void* packed,
                         cudaStream_t st) {
   dim3 grid(K, n_tiles);

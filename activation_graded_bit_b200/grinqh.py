@@ -69,13 +69,15 @@ _vmm_noalloc = _sig("grinqh_vmm_noalloc", [_LP, _P, _P, _P, _P, _P, _I, _P, _P])
 _select_vmm = _sig("grinqh_select_vmm", [_LP, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
 _batch_ws = _sig("grinqh_vmm_batch_workspace_bytes", [_LP, _I, ctypes.POINTER(ctypes.c_size_t)])
 _select_vmm_batch = _sig("grinqh_select_vmm_batch", [_LP, _P, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
+_dequant = _sig("grinqh_dequant", [_LP, _P, _P, _P])
+_prefill = _sig("grinqh_prefill", [_LP, _P, _P, _I, _P, _P, _P])
 
 # Every exported symbol of the C ABI, for the export check in the tests.
 EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grinqh_layout_init_bmax", "grinqh_pack",
            "grinqh_unpack_codes", "grinqh_maxent_distribution", "grinqh_calibrate_workspace_bytes",
            "grinqh_calibrate", "grinqh_select", "grinqh_vmm_workspace_bytes", "grinqh_vmm",
            "grinqh_vmm_noalloc", "grinqh_select_vmm", "grinqh_vmm_batch_workspace_bytes",
-           "grinqh_select_vmm_batch")
+           "grinqh_select_vmm_batch", "grinqh_dequant", "grinqh_prefill")
 
 
 def version() -> str:
@@ -270,7 +272,28 @@ def select_vmm_batch(p: PackedLayer, X: torch.Tensor, thresholds: Optional[torch
     _check(_select_vmm_batch(ctypes.byref(p.layout), _ptr(p.packed), _ptr(X), T, _ptr(thresholds),
                              ctypes.addressof(cb), n, _ptr(Y), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)),
-           "grinqh_select_vmm_batch")
+           "grinqh_select_vmm_batch", "grinqh_dequant", "grinqh_prefill")
+    return Y
+
+
+def dequant(p: PackedLayer, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """grinqh_dequant: full-width w_hat as binary16 [K, N] (returned as float16)."""
+    W16 = out if out is not None else torch.empty((p.K, p.N), dtype=torch.float16, device=p.packed.device)
+    _check(_dequant(ctypes.byref(p.layout), _ptr(p.packed), _ptr(W16), _stream(stream)), "grinqh_dequant")
+    return W16
+
+
+def prefill(p: PackedLayer, X: torch.Tensor, Y: Optional[torch.Tensor] = None, W16: Optional[torch.Tensor] = None,
+            stream=None) -> torch.Tensor:
+    """grinqh_prefill: Y fp32 [T, N] = X [T, K] (fp16 or its bit view) . w_hat at full width."""
+    assert X.is_cuda and X.dim() == 2 and X.is_contiguous() and X.element_size() == 2 and X.shape[1] == p.K
+    T = X.shape[0]
+    if Y is None:
+        Y = torch.empty((T, p.N), dtype=torch.float32, device=X.device)
+    if W16 is None:
+        W16 = torch.empty((p.K, p.N), dtype=torch.float16, device=X.device)
+    _check(_prefill(ctypes.byref(p.layout), _ptr(p.packed), _ptr(X), T, _ptr(Y), _ptr(W16), _stream(stream)),
+           "grinqh_prefill")
     return Y
 
 

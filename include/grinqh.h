@@ -24,7 +24,8 @@
  *   - fp16 values are IEEE binary16 bit patterns passed as uint16_t.
  *   - "device" pointers are CUDA global-memory addresses of the current device;
  *     "host" pointers are ordinary CPU memory. The caller allocates and owns
- *     every buffer; the library never allocates, frees or synchronises.
+ *     every buffer; the library never allocates, frees or synchronises
+ *     (grinqh_prefill's cuBLAS handle is the one exception, see there).
  *   - stream is a cudaStream_t passed as void*; NULL means the legacy default
  *     stream. Every device call is asynchronous on that stream.
  *   - Arguments are checked on the host before anything is launched; a failed
@@ -144,6 +145,34 @@ grinqh_status grinqh_pack(const grinqh_layout* layout, const float* W, void* pac
  */
 grinqh_status grinqh_unpack_codes(const grinqh_layout* layout, const void* packed,
                                   const uint8_t* bits, uint8_t* codes, void* stream);
+
+/*
+ * Full-width dequantisation (the first step of the prefill path).
+ * Paper: Section 4, "Prefill vs. Decoding Evaluation" (prefill unpacks the
+ * weights at full b_max precision for a dense product) and Section 3.3
+ * (w_hat = s * (q - z) at b = b_max). W16[k][n] = w_hat rounded once to binary16
+ * (round to nearest even; the product itself is exact).
+ *   packed  device, from grinqh_pack with this layout, 16-byte aligned.
+ *   W16     device binary16 [K][N] row-major, 16-byte aligned; fully overwritten.
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ */
+grinqh_status grinqh_dequant(const grinqh_layout* layout, const void* packed, uint16_t* W16, void* stream);
+
+/*
+ * The prefill product: Y = X . W_hat for T tokens at full width (no grading),
+ * as grinqh_dequant into W16 followed by a dense binary16 GEMM with fp32
+ * accumulation (cuBLAS, on the same stream). Paper: Section 4, "Prefill vs.
+ * Decoding Evaluation". This call links cuBLAS, which allocates its handle's
+ * resources the first time a device uses it; call it once before any stream
+ * capture.
+ *   X     device fp16 [T][K] row-major, 2-byte aligned; 1 <= T <= 2^24.
+ *   Y     device fp32 [T][N] row-major, output (overwritten), 4-byte aligned.
+ *   W16   device binary16 [K][N], 16-byte aligned: scratch that receives the
+ *         dequantised weights (and keeps them after the call).
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ */
+grinqh_status grinqh_prefill(const grinqh_layout* layout, const void* packed, const uint16_t* X, int32_t T,
+                             float* Y, uint16_t* W16, void* stream);
 
 /*
  * Maximum-entropy precision distribution P over a class set for a requested

@@ -181,3 +181,14 @@ def test_batch_validation_rejects_before_launch(g):
     Lbig = g.layout(20000, 64)
     assert g._select_vmm_batch(ctypes.byref(Lbig), P(0x1000), P(0x1000), 2, *rest, P(0x1000), 1 << 30,
                                None) == 3                                                # K above the fused limit
+
+
+def test_prefill_validation_rejects_before_launch(g):
+    P = ctypes.c_void_p
+    L = g.layout(64, 1024)
+    assert g._dequant(ctypes.byref(L), P(0x1000), None, None) == 1
+    assert g._dequant(ctypes.byref(L), P(0x1000), P(0x1008), None) == 2        # W16 not 16-byte aligned
+    assert g._prefill(ctypes.byref(L), P(0x1000), P(0x1000), 0, P(0x1000), P(0x1000), None) == 1   # T = 0
+    assert g._prefill(ctypes.byref(L), P(0x1000), P(0x1001), 4, P(0x1000), P(0x1000), None) == 2  # X odd
+    assert g._prefill(ctypes.byref(L), P(0x1000), P(0x1000), 4, P(0x1002), P(0x1000), None) == 2  # Y
+    assert g._prefill(None, P(0x1000), P(0x1000), 4, P(0x1000), P(0x1000), None) == 1
