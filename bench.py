@@ -752,6 +752,81 @@ def run_batch(args):
                       "points": out}))
 
 
+def run_prefill(args):
+    """The prefill path on the Llama3-8B linears (Section 4 of the paper: unpack at
+    full b_max precision, then a dense product): for T tokens, microseconds of
+    grinqh_dequant alone, of the GEMM alone and of grinqh_prefill, TFLOP/s of the
+    whole call (2 T K N flops) against the measured bf16 GEMM peak (binary16 runs
+    at the bf16 rate), and the dequant's GB/s (record bytes read + 2 K N written)
+    against the measured copy bandwidth. Graph-replayed over two packed copies."""
+    import torch
+    from activation_graded_bit_b200 import grinqh as g
+    from activation_graded_bit_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device=dev)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        pass
+    tflops_peak = float(peaks.get("bf16_tflops", 1590.0))
+    hbm_peak, hbm_kind = _peaks()
+    lin = []
+    for li, (name, K, N) in enumerate(wl.LLAMA3_8B):
+        ps = []
+        for c in range(2):
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(6_000_011 * (li + 1) + c)
+            ps.append(g.pack(torch.randn(K, N, generator=gen, device=dev, dtype=torch.float32) * 0.02))
+        lin.append(dict(name=name, K=K, N=N, p=ps, W16=[torch.empty((K, N), dtype=torch.float16, device=dev)
+                                                         for _ in range(2)]))
+    out = []
+    for T in (512, 2048):
+        for d in lin:
+            X = wl.activations_outlier(d["K"], T, key=(6, T, d["K"], d["N"]), chan_key=(6, d["K"]))
+            d["X"] = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).to(dev)
+            d["Y"] = torch.empty((T, d["N"]), dtype=torch.float32, device=dev)
+
+        def timed(fn, reps=20):
+            with torch.cuda.stream(stream):
+                fn(0)
+                fn(1)
+                torch.cuda.synchronize()
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=stream):
+                    for r in range(reps):
+                        fn(r % 2)
+                gr.replay()
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                gr.replay()
+                e1.record(stream)
+            stream.synchronize()
+            del gr
+            return e0.elapsed_time(e1) * 1e3 / reps
+
+        for d in lin:
+            K, N = d["K"], d["N"]
+            us_deq = timed(lambda c: g.dequant(d["p"][c], out=d["W16"][c], stream=stream))
+            us_all = timed(lambda c: g.prefill(d["p"][c], d["X"], Y=d["Y"], W16=d["W16"][c], stream=stream))
+            flops = 2.0 * T * K * N
+            deq_bytes = d["p"][0].packed.numel() + 2.0 * K * N
+            out.append({"linear": d["name"], "K": K, "N": N, "tokens": T, "prefill_us": round(us_all, 2),
+                        "dequant_us": round(us_deq, 2), "tflops": round(flops / (us_all * 1e-6) / 1e12, 1),
+                        "tflops_frac": round(flops / (us_all * 1e-6) / 1e12 / tflops_peak, 4),
+                        "dequant_gbs": round(deq_bytes / (us_deq * 1e-6) / 1e9, 1),
+                        "dequant_frac": round(deq_bytes / (us_deq * 1e-6) / 1e9 / hbm_peak, 4)})
+    print(json.dumps({"metric": "prefill: us per linear, TFLOP/s of dequant + fp16 GEMM, dequant GB/s",
+                      "unit": "µs", "higher_is_better": False, "data": "synthetic",
+                      "peak_tflops": tflops_peak, "peak_gbs": hbm_peak, "peak_kind": hbm_kind,
+                      "config": {"workload": "llama3-8b linears, prefill of 512 and 2048 tokens, b_max 8 codes, "
+                                             "two packed copies rotated"},
+                      "points": out}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -768,6 +843,7 @@ def main():
     ap.add_argument("--stack", action="store_true", help="32-layer linear stack tokens/s (one JSON line)")
     ap.add_argument("--stack-steps", type=int, default=256)
     ap.add_argument("--batch", action="store_true", help="batch 1..16 through the batched fused call (one JSON line)")
+    ap.add_argument("--prefill", action="store_true", help="prefill path: dequant + GEMM on the linears (one JSON line)")
     ap.add_argument("--bmax", type=int, default=8, choices=(4, 6, 8),
                     help="stored code width; 4 or 6 grade into the classes {0, 2, ..., b_max}")
     args = ap.parse_args()
@@ -787,6 +863,9 @@ def main():
         return
     if args.batch:
         run_batch(args)
+        return
+    if args.prefill:
+        run_prefill(args)
         return
     if args.profile:
         run_profile_case(args)
