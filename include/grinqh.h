@@ -2,7 +2,7 @@
  * grinqh.h - C ABI of the GRINQH graded bit-plane VMM library (sm_100a).
  *
  * GRINQH ("GRINQH: Graded Input-based Quantization Hierarchy for Efficient LLM
- * Generation", arXiv 2606.23419) speeds up batch-1 decoding by reading, for each
+ * Generation", arXiv 2606.23419) speeds up decoding by reading, for each
  * input channel k of a linear layer, only the b_k most significant bits of that
  * channel's b_max-bit weights (b_max = 8 by default; 2, 4 or 6 on request),
  * where b_k is chosen per token from |x_k| against calibrated thresholds
@@ -18,6 +18,12 @@
  *   grinqh_maxent_distribution / grinqh_calibrate   thresholds for a target width
  *   grinqh_select            per-token grading + per-class channel lists
  *   grinqh_vmm               y = x . W_hat over the graded bit planes
+ * and, for the same packed layer:
+ *   grinqh_select_vmm        grading and the graded product in one launch
+ *   grinqh_select_vmm_batch  the same for T tokens in one launch
+ *   grinqh_vmm_noalloc       grinqh_vmm on the library's own static scratch
+ *   grinqh_dequant / grinqh_prefill   full-width weights and the dense prefill
+ *                            product for many tokens
  *
  * Conventions for every call:
  *   - W is K x N: K input channels (rows), N output channels (columns).
