@@ -49,14 +49,19 @@
 // that matter). The per-row constant a * (mid_b - z) goes to one scalar per
 // thread, since all 32 columns of a thread share one 128-column group.
 //
-// Reduction. The 16 warps of a CTA are summed in shared memory into one
-// 1024-column partial, stored with plain coalesced stores into the workspace
-// as partial[r][column]. A second kernel, chained with programmatic dependent
-// launch, sums the R partials of every column in a fixed order and overwrites
-// y. (Adding partials into y with L2 atomics instead costs far more: up to 148
-// CTAs would add into the same 1024..16384 addresses, and same-address
-// reductions serialise in L2.) With a single row split (R = 1) the CTA writes
-// y directly and no second kernel runs.
+// Reduction. Each warp stores its 1024 column sums into shared memory as soon
+// as its own rows are done (the buffer is not shared with the row list); after
+// one barrier the CTA sums the 16 warps into one 1024-column partial, stored
+// with plain coalesced stores into the workspace as partial[r][column]. A
+// second kernel, chained with programmatic dependent launch, sums the R
+// partials of every column in a fixed order (every load of a column in flight
+// at once) and overwrites y, so repeated calls give the same bits. (Finishing
+// the sum inside this kernel, with vector L2 reductions into a per-tile
+// accumulator and the last CTA to arrive writing y, measured no faster, and
+// its order of additions varies from call to call.) With a single row split
+// (R = 1) the CTA writes y directly and no second kernel runs. A batch of
+// tokens (grinqh_select_vmm_batch) adds a grid dimension: token z reads
+// x + z K and has its own set of partials and its own y row.
 #include <cstdint>
 #include <cuda_fp16.h>
 #include <atomic>
