@@ -43,6 +43,27 @@ WORKLOAD = "llama3-8b decode linears (q,k,v,o,gate,up,down), batch 1, avg bits 4
 # the paper's even classes {0, 2, ..., b_max} (Section 3.3, b_max in {4, 6, 8}).
 BMAX = 8
 CLASSES = None   # set in main()
+# Layer family: "llama3" (Llama3-8B shapes, weights N(0, 0.02), outlier
+# activations, average bits 4/3/2) or "qwen3" (Qwen3-8B shapes, weights with a
+# log-uniform per-row std in [0.005, 0.05], Student-t(3) activations, 4/3).
+FAMILY = "llama3"
+
+
+def _family(wl):
+    """(shapes, activation draw (K, count, key) -> uint16 bits) of FAMILY."""
+    if FAMILY == "qwen3":
+        return wl.QWEN3_8B, (lambda K, count, key, li: wl.activations_student_t(K, count, key=key))
+    return wl.LLAMA3_8B, (lambda K, count, key, li: wl.activations_outlier(K, count, key=key, chan_key=(1, 0, li)))
+
+
+def _weights(torch, gen, K, N, dev):
+    """Weights of one linear on the GPU from the seeded generator `gen`."""
+    W = torch.randn(K, N, generator=gen, device=dev, dtype=torch.float32)
+    if FAMILY == "qwen3":
+        u = torch.rand(K, 1, generator=gen, device=dev, dtype=torch.float64)
+        sig = torch.exp(np.log(0.005) + u * (np.log(0.05) - np.log(0.005))).float()
+        return W * sig
+    return W * 0.02
 
 
 def _peaks():
@@ -140,8 +161,9 @@ def build_workload(g, wl, torch, dev, copies=2):
     classes = CLASSES
     pairs = []
     gen = torch.Generator(device=dev)
-    for li, (name, K, N) in enumerate(wl.LLAMA3_8B):
-        Xc = wl.activations_outlier(K, 128, key=(1, 0, li, 1), chan_key=(1, 0, li))
+    shapes, draw = _family(wl)
+    for li, (name, K, N) in enumerate(shapes):
+        Xc = draw(K, 128, (1, 0, li, 1), li)
         Xc_d = torch.from_numpy(Xc.view(np.int16)).to(dev)
         th = {}
         for t in TARGETS:
@@ -149,10 +171,10 @@ def build_workload(g, wl, torch, dev, copies=2):
         for c in range(copies):
             for ti, t in enumerate(TARGETS):
                 gen.manual_seed(1_000_003 * (li + 1) + 7919 * c + 31 * ti)
-                W = torch.randn(K, N, generator=gen, device=dev, dtype=torch.float32) * 0.02
+                W = _weights(torch, gen, K, N, dev)
                 p = g.pack(W, b_max=BMAX)
                 del W
-                x = wl.activations_outlier(K, 1, key=(1, c, li, 2 + ti), chan_key=(1, 0, li))[0]
+                x = draw(K, 1, (1, c, li, 2 + ti), li)[0]
                 x_d = torch.from_numpy(x.view(np.int16)).to(dev)
                 sel = g.select(x_d, th[t], classes)
                 pairs.append(dict(name=name, K=K, N=N, target=t, copy=c, packed=p, x=x_d, x_host=x,
@@ -339,9 +361,11 @@ def run_gpu(args):
         L = pr["packed"].layout
         launches_per_step += 2 + (1 if pr["ws"].numel() > 16 + L.n_tiles * 4096 else 0)
 
+    # DRAM traffic comes from an ncu capture of the default workload (Llama3-8B
+    # linears, b_max 8); for any other workload it was not measured
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "vmm_traffic.json")
-    if os.path.exists(tpath):
+    if os.path.exists(tpath) and FAMILY == "llama3" and BMAX == 8:
         try:
             traffic = json.load(open(tpath)).get("bytes_per_launch_scaled")
         except Exception:
@@ -357,7 +381,7 @@ def run_gpu(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "u8 planes, fp32 accumulate", "data": "synthetic",
             "config": {"workload": WORKLOAD, "pairs_per_step": n_pairs, "classes": list(CLASSES), "b_max": BMAX,
                        "l2": "inputs larger than L2: every pair of a step reads its own packed copy; "
-                             "%d copies of the layer set (%.2f GB) rotate" % (
+                             "%d packed layers (%.2f GB) rotate" % (
                                  len(pairs), sum(pr["packed"].packed.numel() for pr in pairs) / 1e9),
                        "parallelism": "replicas only" if world > 1 else "single GPU"},
             "vmm_us": round(us_vmm, 4), "select_plus_vmm_us": round(us_pair, 4),
@@ -401,17 +425,19 @@ def _oracle_sample(budget_s, nthreads):
     secs = 0.0
     names = []
     t_start = time.time()
-    for li, (name, K, N) in enumerate(wl.LLAMA3_8B):
+    shapes, draw = _family(wl)
+    for li, (name, K, N) in enumerate(shapes):
         if time.time() - t_start > budget_s:
             break
         # untimed setup: weights, RTN codes, thresholds of this linear
-        W = wl.weights_gaussian(K, N, key=(1, 9, li, 0))
+        W = (wl.weights_rowstd_loguniform(K, N, key=(1, 9, li, 0)) if FAMILY == "qwen3"
+             else wl.weights_gaussian(K, N, key=(1, 9, li, 0)))
         q, s, z = oracle.rtn_quantize(W, BMAX)
         del W
-        Xc = wl.activations_outlier(K, 32, key=(1, 0, li, 1), chan_key=(1, 0, li))
+        Xc = draw(K, 32, (1, 0, li, 1), li)
         for ti, t in enumerate(TARGETS):
             th = oracle.thresholds(Xc, oracle.maxent_distribution(classes, t))
-            x = wl.activations_outlier(K, 1, key=(1, 0, li, 2 + ti), chan_key=(1, 0, li))[0]
+            x = draw(K, 1, (1, 0, li, 2 + ti), li)[0]
             t0 = time.perf_counter()
             bits, idx, off = oracle.select(x, th, classes)
             oracle.vmm(x, q, s, z, bits, nthreads=nthreads, bmax=BMAX)
@@ -427,7 +453,8 @@ def cpu_baseline(args):
     nthreads = os.cpu_count() or 1
     done, secs, names = _oracle_sample(args.cpu_budget, nthreads)
     return {"value": round(secs * 1e6 / max(done, 1), 1), "unit": UNIT, "cores": nthreads, "kind": "oracle",
-            "sample": "fp64 oracle select+vmm on %d of the 21 (linear, width) pairs: %s" % (done, ", ".join(names))}
+            "sample": "fp64 oracle select+vmm on %d of the %d (linear, width) pairs: %s" % (
+                done, 7 * len(TARGETS), ", ".join(names))}
 
 
 def run_reference(args):
@@ -846,8 +873,15 @@ def main():
     ap.add_argument("--prefill", action="store_true", help="prefill path: dequant + GEMM on the linears (one JSON line)")
     ap.add_argument("--bmax", type=int, default=8, choices=(4, 6, 8),
                     help="stored code width; 4 or 6 grade into the classes {0, 2, ..., b_max}")
+    ap.add_argument("--family", default="llama3", choices=("llama3", "qwen3"),
+                    help="layer family of the main run: Llama3-8B (default) or Qwen3-8B shapes and distributions")
     args = ap.parse_args()
-    global BMAX, CLASSES, WORKLOAD
+    global BMAX, CLASSES, WORKLOAD, FAMILY, TARGETS
+    FAMILY = args.family
+    if FAMILY == "qwen3":
+        TARGETS = (4.0, 3.0)
+        WORKLOAD = ("qwen3-8b decode linears (q,k,v,o,gate,up,down), batch 1, avg bits 4/3, row-std log-uniform "
+                    "weights, student-t activations")
     from activation_graded_bit_b200 import workloads as wl
     BMAX = args.bmax
     CLASSES = tuple(wl.CLASSES) if BMAX == 8 else tuple(range(0, BMAX + 1, 2))
