@@ -109,7 +109,6 @@ struct RowRegs {
 // layout has K * N <= 2^34, so K * n_tiles <= 2^25) and one wide multiply-add
 // each of this lane's addresses in it.
 struct RowAddr {
-  const uint16_t* x;      // this CTA's token's activation vector
   const uint8_t* meta;    // packed + this lane's scale/zero word within a record
   const uint8_t* pairs;   // packed + this lane's two words of pair 0 within a record
   const uint8_t* lines;   // packed + 128 * lane (the lane's L2 line within a record prefix)
@@ -121,7 +120,6 @@ __device__ __forceinline__ RowAddr row_addr(const VmmArgs& a, int t, int w) {
   const uint32_t kSectors = (uint32_t)record_bytes_for(a.b_max) / 32u;   // 9, 17, 25 or 33
   static_assert(kMetaBytes % 32 == 0 && kPlaneBytes % 16 == 0, "records are whole 32-byte sectors");
   RowAddr ra;
-  ra.x = a.x + (size_t)blockIdx.z * a.K;
   ra.meta = a.packed + 4 * (w >> 2);
   ra.pairs = a.packed + kMetaBytes + 8 * w;
   ra.lines = a.packed + 128 * w;
@@ -201,12 +199,13 @@ __device__ __forceinline__ void fma_codes(const uint32_t (&R)[8], float A0s, flo
 // coalesced 256-byte request across the warp). Pairs 1..3 are loaded under a
 // predicate: a narrow row reads no pair it does not use, and no branch is taken.
 // Every row that reaches the loop has b >= 1 (the width-0 class is never staged).
-__device__ __forceinline__ void load_row(const VmmArgs& a, const RowAddr& ra, uint32_t info, RowRegs& r) {
+__device__ __forceinline__ void load_row(const uint16_t* __restrict__ x, const RowAddr& ra, uint32_t info,
+                                         RowRegs& r) {
   const uint32_t k = info & 0xFFFFFFu, b = info >> 24;
   const uint32_t sec = k * ra.nt33 + ra.t33;                  // record offset in 32-byte sectors
   r.b = b;
   r.m = ld_stream(ra.meta + 32ull * sec);
-  r.xh = __ldg(ra.x + k);
+  r.xh = __ldg(x + k);
   const uint8_t* pw = ra.pairs + 32ull * sec;                  // this lane's two words of pair 0
   ld_stream2_at<0>(pw, r.p[0], r.p[1]);
   ld_stream2_at_if<1 * kPairBytes>(b > 2, pw, r.p[2], r.p[3]);
@@ -281,7 +280,8 @@ __device__ __forceinline__ void row_fma(const RowRegs& r, float2 (&acc)[16], flo
 // grades only its own K/R channels: no selection kernel, no kernel boundary, no
 // channel list and no grading repeated across CTAs. s.width must be filled.
 // Returns the number of rows staged (K <= kFusedMaxK = kIdxCap: one pass).
-__device__ __forceinline__ int stage_fused(const VmmArgs& a, VmmSmem& s, int r, int R) {
+__device__ __forceinline__ int stage_fused(const VmmArgs& a, const uint16_t* __restrict__ xt, VmmSmem& s, int r,
+                                           int R) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nt = a.ct.n - 1;
   float th[8];
@@ -289,7 +289,6 @@ __device__ __forceinline__ int stage_fused(const VmmArgs& a, VmmSmem& s, int r, 
   for (int q = 0; q < 8; ++q) th[q] = (q < nt) ? __ldg(a.thresholds + q) : 0.0f;
   const int nk = (a.K > r) ? (a.K - r + R - 1) / R : 0;
   const uint32_t lt = (1u << lane) - 1u;
-  const uint16_t* xt = a.x + (size_t)blockIdx.z * a.K;   // this CTA's token
   int base = 0;
 #pragma unroll 1
   for (int i0 = 0, rnd = 0; i0 < nk; i0 += kThreads, rnd ^= 1) {
@@ -324,12 +323,16 @@ __device__ __forceinline__ int stage_fused(const VmmArgs& a, VmmSmem& s, int r, 
 }
 
 
-template <bool kFused, int kBmax>
+// kBatch: the grid has a token dimension (grinqh_select_vmm_batch): token z
+// reads x + z K, has its own set of partials and its own y row. The
+// single-vector kernels are compiled without it.
+template <bool kFused, int kBmax, bool kBatch>
 __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   VmmSmem& s = *reinterpret_cast<VmmSmem*>(smem_raw);
   const int tid = threadIdx.x, h = tid >> 5, w = tid & 31;   // warp h, word w = lane
   const int t = blockIdx.x, r = blockIdx.y, R = gridDim.y;
+  const uint16_t* xv = kBatch ? a.x + (size_t)blockIdx.z * a.K : a.x;   // this CTA's activation vector
 
   // This CTA takes list positions r + R e (e = 0, 1, ...); the width-0 class,
   // when there is one, is the first class of the list, so its positions are a
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
   for (int c = 0; c < 16; ++c) acc[c] = make_float2(0.0f, 0.0f);
   float cacc = 0.0f;
 
-  const int nq_fused = kFused ? stage_fused(a, s, r, R) : 0;   // one pass: K <= kFusedMaxK rows fit
+  const int nq_fused = kFused ? stage_fused(a, xv, s, r, R) : 0;   // one pass: K <= kFusedMaxK rows fit
   const int passes_total = kFused ? nq_fused : nq_total;
   for (int qb = 0; qb < passes_total; qb += kIdxCap) {
     const int nq = kFused ? nq_fused : min(kIdxCap, nq_total - qb);
@@ -399,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
     RowRegs S[kDepth];
 #pragma unroll
     for (int d = 0; d < kDepth; ++d)
-      if (d < nrow) load_row(a, ra, s.u.rows[h + kWarps * d], S[d]);
+      if (d < nrow) load_row(xv, ra, s.u.rows[h + kWarps * d], S[d]);
 #pragma unroll 1
     for (int m = kDepth; m < min(nrow, kDepth + kL2Ahead); ++m) prefetch_row_l2(ra, s.u.rows[h + kWarps * m]);
     int m0 = 0;
@@ -410,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
       for (int d = 0; d < kDepth; ++d) {
         const int m = m0 + d;
         row_fma<kBmax>(S[d], acc, cacc);
-        load_row(a, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
+        load_row(xv, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
         // the record prefix of the row kL2Ahead rows further on goes to L2 now,
         // one 128-byte line per lane, so its register loads later hit L2
         prefetch_row_l2(ra, s.u.rows[h + kWarps * (m + kDepth + kL2Ahead)]);
@@ -427,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
         const int m = m0 + d;
         if (m < nrow) {
           row_fma<kBmax>(S[d], acc, cacc);
-          if (m + kDepth < nrow) load_row(a, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
+          if (m + kDepth < nrow) load_row(xv, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
         }
       }
     }
@@ -450,8 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
   __syncthreads();
   // partial[r][column], or y itself when there is a single row split; every
   // column of the tile is written, zeros included, so no clearing is needed
-  // (token blockIdx.z: its y row and its set of partials)
-  const size_t tok = blockIdx.z;
+  // (a batch's token blockIdx.z: its y row and its set of partials)
+  const size_t tok = kBatch ? blockIdx.z : 0;
   float* out = (R == 1) ? a.y + tok * a.N : a.partial + (tok * R + r) * a.n_tiles * kTileN;
   const int limit = (R == 1) ? a.N : a.n_tiles * kTileN;
 #pragma unroll
@@ -472,6 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
 // column arrive in one memory round trip.
 constexpr int kRedChains = 16;
 constexpr int kRedLoads = 8;   // R <= 128 in one round trip; larger R loops
+template <bool kBatch>
 __global__ void __launch_bounds__(32 * kRedChains) reduce_partials_kernel(const float* __restrict__ partial, int R,
                                                                          int stride, float* __restrict__ y, int N) {
   __shared__ float s_part[kRedChains][33];
@@ -479,8 +483,10 @@ __global__ void __launch_bounds__(32 * kRedChains) reduce_partials_kernel(const 
   pdl_wait();   // the partials come from the VMM kernel just before
   const int lane = threadIdx.x & 31, chain = threadIdx.x >> 5;
   const int col = blockIdx.x * 32 + lane;
-  partial += (size_t)blockIdx.y * R * stride;   // token blockIdx.y
-  y += (size_t)blockIdx.y * N;
+  if (kBatch) {   // token blockIdx.y of a batch
+    partial += (size_t)blockIdx.y * R * stride;
+    y += (size_t)blockIdx.y * N;
+  }
   float v = 0.0f;
   if (col < N) {
     for (int r0 = chain; r0 < R; r0 += kRedChains * kRedLoads) {
@@ -532,15 +538,18 @@ size_t vmm_workspace_bytes(int n_tiles, int /*tile_n*/) { return vmm_workspace_b
 template <int kBmax>
 static cudaError_t set_smem_attr() {
   const int smem = (int)sizeof(VmmSmem);
-  cudaError_t e = cudaFuncSetAttribute(vmm_kernel<false, kBmax>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(vmm_kernel<true, kBmax>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const cudaFuncAttribute at = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaError_t e = cudaFuncSetAttribute(vmm_kernel<false, kBmax, false>, at, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(vmm_kernel<true, kBmax, false>, at, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(vmm_kernel<true, kBmax, true>, at, smem);
   return e;
 }
 
 template <int kBmax>
 static cudaError_t launch_one(const cudaLaunchConfig_t& cfg, const VmmArgs& a, bool fused) {
-  return fused ? cudaLaunchKernelEx(&cfg, vmm_kernel<true, kBmax>, a) : cudaLaunchKernelEx(&cfg, vmm_kernel<false, kBmax>, a);
+  if (a.tokens > 1) return cudaLaunchKernelEx(&cfg, vmm_kernel<true, kBmax, true>, a);   // only the fused call batches
+  return fused ? cudaLaunchKernelEx(&cfg, vmm_kernel<true, kBmax, false>, a)
+               : cudaLaunchKernelEx(&cfg, vmm_kernel<false, kBmax, false>, a);
 }
 
 // The kernels' shared-memory limit is raised once per device (with that device
@@ -593,7 +602,10 @@ cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused) {
   rc.stream = st;
   rc.attrs = attr;
   rc.numAttrs = 1;
-  return cudaLaunchKernelEx(&rc, reduce_partials_kernel, (const float*)a.partial, R, a.n_tiles * kTileN, a.y,
+  if (a.tokens > 1)
+    return cudaLaunchKernelEx(&rc, reduce_partials_kernel<true>, (const float*)a.partial, R, a.n_tiles * kTileN,
+                              a.y, a.N);
+  return cudaLaunchKernelEx(&rc, reduce_partials_kernel<false>, (const float*)a.partial, R, a.n_tiles * kTileN, a.y,
                             a.N);
 }
 

@@ -272,7 +272,7 @@ def select_vmm_batch(p: PackedLayer, X: torch.Tensor, thresholds: Optional[torch
     _check(_select_vmm_batch(ctypes.byref(p.layout), _ptr(p.packed), _ptr(X), T, _ptr(thresholds),
                              ctypes.addressof(cb), n, _ptr(Y), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)),
-           "grinqh_select_vmm_batch", "grinqh_dequant", "grinqh_prefill")
+           "grinqh_select_vmm_batch")
     return Y
 
 
