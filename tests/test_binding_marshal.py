@@ -1,0 +1,95 @@
+"""Every call of the Python binding marshals its arguments into the C ABI and
+turns a rejected call into GrinqhError. Runs without a GPU: stand-in tensors
+carry plausible device addresses, and each call is given a layout or argument
+that the library rejects on the host before anything could be launched."""
+import ctypes
+
+import pytest
+import torch
+
+
+class FakeTensor:
+    """The attributes the binding reads from a CUDA tensor; never dereferenced."""
+
+    def __init__(self, shape, dtype, addr=0x10000):
+        self.shape = tuple(shape)
+        self.dtype = dtype
+        self.is_cuda = True
+        self.device = "cpu"
+        self._addr = addr
+
+    def dim(self):
+        return len(self.shape)
+
+    def is_contiguous(self):
+        return True
+
+    def element_size(self):
+        return torch.empty(0, dtype=self.dtype).element_size()
+
+    def numel(self):
+        n = 1
+        for s in self.shape:
+            n *= s
+        return n
+
+    def data_ptr(self):
+        return self._addr
+
+    def view(self, *a):
+        return self
+
+
+class FakeStream:
+    cuda_stream = 0
+
+
+@pytest.fixture(scope="module")
+def g():
+    from activation_graded_bit_b200 import build
+    build.build()
+    from activation_graded_bit_b200 import grinqh
+    return grinqh
+
+
+def _bad_packed(g, K=64, N=1024):
+    L = g.layout(K, N)
+    L.tile_n = 512   # not a layout grinqh_layout_init makes: every call rejects it
+    return g.PackedLayer(L, FakeTensor((int(L.packed_bytes),), torch.uint8))
+
+
+def _expect_invalid(fn):
+    from activation_graded_bit_b200 import grinqh
+    with pytest.raises(grinqh.GrinqhError) as e:
+        fn()
+    assert e.value.code == 1
+
+
+def test_every_call_marshals_and_reports(g):
+    K, N, T = 64, 1024, 3
+    cl = (0, 2, 3, 4, 8)
+    st = FakeStream()
+    p = _bad_packed(g, K, N)
+    x = FakeTensor((K,), torch.int16)
+    X = FakeTensor((T, K), torch.int16)
+    th = FakeTensor((4,), torch.float32)
+    y = FakeTensor((N,), torch.float32)
+    Y = FakeTensor((T, N), torch.float32)
+    ws = FakeTensor((1 << 20,), torch.uint8)
+    sel = g.Selection(FakeTensor((K,), torch.uint8), FakeTensor((K,), torch.int32),
+                      FakeTensor((len(cl) + 1,), torch.int32), cl)
+    W = FakeTensor((K, N), torch.float32)
+    W16 = FakeTensor((K, N), torch.float16)
+    _expect_invalid(lambda: g.pack(W, out=p, stream=st))
+    _expect_invalid(lambda: g.unpack_codes(p, stream=st))
+    _expect_invalid(lambda: g.vmm(p, x, sel, ws, y=y, stream=st))
+    _expect_invalid(lambda: g.select_vmm(p, x, th, cl, ws, y=y, stream=st))
+    _expect_invalid(lambda: g.select_vmm_batch(p, X, th, cl, ws, Y=Y, stream=st))
+    _expect_invalid(lambda: g.vmm_noalloc(p, x, sel, y, stream=st))
+    _expect_invalid(lambda: g.dequant(p, out=W16, stream=st))
+    _expect_invalid(lambda: g.prefill(p, X, Y=Y, W16=W16, stream=st))
+    # calls without a layout: invalid class sets
+    _expect_invalid(lambda: g.select(x, th, (0, 4, 4), out=sel, stream=st))
+    Xc = FakeTensor((8, K), torch.int16)
+    _expect_invalid(lambda: g.calibrate(Xc, (0, 4, 4), target_bits=2.0, out=th, workspace=ws, stream=st))
+    _expect_invalid(lambda: g.vmm_batch_workspace(g.layout(K, N), 0))
