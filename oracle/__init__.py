@@ -40,7 +40,9 @@ def lib():
         L.orc_dequant_f16.argtypes = [P, P, P, i32, i32, P]
         L.orc_maxent_distribution.argtypes = [P, i32, ctypes.c_double, P]
         L.orc_thresholds.argtypes = [P, i32, i32, P, i32, P]
-        for f in ("orc_rtn_quantize", "orc_rtn_quantize_bmax", "orc_code", "orc_code_bmax", "orc_grade",
+        L.orc_lut_build.argtypes = [P, i32, i32, i32, P, P, P]
+        L.orc_vmm_lut.argtypes = [P, P, P, P, i32, i32, i32, P, P, i32]
+        for f in ("orc_lut_build", "orc_vmm_lut", "orc_rtn_quantize", "orc_rtn_quantize_bmax", "orc_code", "orc_code_bmax", "orc_grade",
                   "orc_compact", "orc_vmm", "orc_vmm_bmax", "orc_dequant_f16",
                   "orc_maxent_distribution", "orc_thresholds"):
             getattr(L, f).restype = ctypes.c_int
@@ -187,3 +189,39 @@ def prefill(X_bits, w16):
     Xf = np.ascontiguousarray(X_bits, np.uint16).view(np.float16).astype(np.float64)
     Wf = np.ascontiguousarray(w16, np.uint16).view(np.float16).astype(np.float64)
     return Xf @ Wf, np.abs(Xf) @ np.abs(Wf)
+
+
+def lut_build(W, bmax=8):
+    """Nested look-up-table codes by incremental upscaling (Section 3.3 on nested
+    non-uniform codes; Section 4 and Appendix E.2 on any-precision LLM weights).
+    Each cluster of width b-1 of a row is split by the optimal 1-D 2-means cut.
+
+    Returns (q uint8 [K,N] codes of bmax bits, lut uint16 [K, 2^(bmax+1)] binary16
+    centroids in heap order (width b, code c at 2^b + c), cent float64 [K, 2^(bmax+1)]
+    the same centroids before rounding)."""
+    W = _c(W, np.float32)
+    K, N = W.shape
+    E = 1 << (bmax + 1)
+    q = np.empty((K, N), np.uint8)
+    lut = np.empty((K, E), np.uint16)
+    cent = np.empty((K, E), np.float64)
+    if lib().orc_lut_build(_p(W), K, N, int(bmax), _p(q), _p(lut), _p(cent)) != 0:
+        raise ValueError("bad sizes or b_max")
+    return q, lut, cent
+
+
+def vmm_lut(x_bits, q, lut, bits, bmax=8, nthreads=1):
+    """fp64 graded product over nested table codes: w_hat = lut[k][2^b + (q >> (bmax - b))]
+    for b = b_k > 0 (no midpoint, no scale or zero point), and bound = sum |x_k w_hat_kn|."""
+    x_bits = _c(x_bits, np.uint16)
+    q = _c(q, np.uint8)
+    lut = _c(lut, np.uint16)
+    bits = _c(bits, np.uint8)
+    K, N = q.shape
+    assert lut.shape == (K, 1 << (bmax + 1))
+    y = np.empty(N, np.float64)
+    bound = np.empty(N, np.float64)
+    if lib().orc_vmm_lut(_p(x_bits), _p(q), _p(lut), _p(bits), K, N, int(bmax), _p(y), _p(bound),
+                         int(nthreads)) != 0:
+        raise ValueError("bad sizes or a width above b_max")
+    return y, bound

@@ -365,4 +365,132 @@ int orc_thresholds(const uint16_t* X, int S, int K, const double* P, int n_class
   return 0;
 }
 
+// ---------------------------------------------------------------------------
+// Nested non-uniform (look-up table) codes.
+// Paper: Section 3.3 "Storage Layout and Weight Loading": the bit planes need a
+// nested quantisation, which uniform codes and k-means codes such as
+// any-precision LLM's satisfy; for non-uniform weights the parent model has
+// b_max bits, and the midpoint term is not used because the nested levels are
+// already centred. Section 4 "Models and Baselines": any-precision LLM weights
+// at b_max = 8, per channel. Appendix E.2: the same framework on nested
+// any-precision weights, built by k-means-based incremental upscaling.
+//
+// Library reading (the pages give no construction of their own):
+//  * one table per row k (the axis the planes are graded on) and width b: the
+//    code c_b = q >> (b_max - b) (the top b bits of the b_max-bit code, as for
+//    uniform codes) selects the level-b centroid of the row; w_hat = that value.
+//  * tables in heap order: entry 2^b + c is centroid c of width b, so width b
+//    occupies entries [2^b, 2^(b+1)) of the row's 2^(b_max+1) entries (entry 1
+//    is the row mean, entry 0 is unused and 0), stored as binary16 (RNE).
+//  * incremental upscaling: width 0 is one cluster holding the whole row; each
+//    cluster of width b-1 is split in two by the optimal one-dimensional
+//    2-means split of its members (lower child bit 0, upper child bit 1). On
+//    sorted values an optimal split is a cut between two neighbours; a cut
+//    between equal values is not used, so equal weights share a code. The cut
+//    maximises the between-cluster sum of squares S^2 m / (s (m - s)) (S the sum
+//    of the s lower members' deviations from the cluster mean, m members), which
+//    is the same as minimising the two children's summed squared error; ties go
+//    to the smallest s. A cluster with fewer than two distinct values keeps all
+//    members in its lower child; an empty child's centroid is its parent's.
+//  * centroids are the fp64 means of their members (each child of a split then
+//    averages, weighted by its count, to its parent).
+// W fp32 [K*N] row-major; q out [K*N] codes of bmax bits; lut out [K*2^(bmax+1)]
+// binary16 bit patterns; cent (optional) [K*2^(bmax+1)] the same centroids in
+// fp64. Returns 0, or -1 on bad sizes.
+// ---------------------------------------------------------------------------
+int orc_lut_build(const float* W, int K, int N, int bmax, uint8_t* q, uint16_t* lut, double* cent) {
+  if (K <= 0 || N <= 0 || bmax < 1 || bmax > 8) return -1;
+  const int E = 1 << (bmax + 1);
+  std::vector<double> c(E);
+  std::vector<int> order(N), code(N);
+  for (int k = 0; k < K; ++k) {
+    const float* w = W + (size_t)k * N;
+    for (int n = 0; n < N; ++n) order[n] = n;
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return w[a] < w[b]; });
+    std::fill(c.begin(), c.end(), 0.0);
+    std::fill(code.begin(), code.end(), 0);
+    // members of each cluster are a contiguous run of `order`: run [lo, hi)
+    std::vector<int> lo(1, 0), hi(1, N);
+    double root = 0.0;
+    for (int n = 0; n < N; ++n) root += (double)w[n];
+    c[1] = root / (double)N;
+    for (int b = 1; b <= bmax; ++b) {
+      std::vector<int> nlo(2 * lo.size()), nhi(2 * lo.size());
+      for (size_t p = 0; p < lo.size(); ++p) {
+        const int a = lo[p], e = hi[p], m = e - a;
+        const double parent = c[(1 << (b - 1)) + (int)p];
+        int cut = e;   // lower child [a, cut), upper child [cut, e)
+        if (m >= 2) {
+          double mean = 0.0;
+          for (int i = a; i < e; ++i) mean += (double)w[order[i]];
+          mean /= (double)m;
+          double S = 0.0, best = -1.0;
+          for (int s = 1; s < m; ++s) {
+            S += (double)w[order[a + s - 1]] - mean;
+            if (!(w[order[a + s - 1]] < w[order[a + s]])) continue;   // no cut between equal values
+            const double B = S * S * (double)m / ((double)s * (double)(m - s));
+            if (B > best) { best = B; cut = a + s; }
+          }
+        }
+        nlo[2 * p] = a; nhi[2 * p] = cut;
+        nlo[2 * p + 1] = cut; nhi[2 * p + 1] = e;
+        for (int ch = 0; ch < 2; ++ch) {
+          const int ca = nlo[2 * p + ch], ce = nhi[2 * p + ch];
+          double v = parent;
+          if (ce > ca) {
+            double t = 0.0;
+            for (int i = ca; i < ce; ++i) t += (double)w[order[i]];
+            v = t / (double)(ce - ca);
+          }
+          c[(1 << b) + 2 * (int)p + ch] = v;
+          for (int i = ca; i < ce; ++i) code[order[i]] = 2 * (int)p + ch;
+        }
+      }
+      lo.swap(nlo);
+      hi.swap(nhi);
+    }
+    for (int n = 0; n < N; ++n) q[(size_t)k * N + n] = (uint8_t)code[n];
+    for (int i = 0; i < E; ++i) {
+      lut[(size_t)k * E + i] = (i == 0) ? 0 : orc_f64_to_f16(c[i]);
+      if (cent) cent[(size_t)k * E + i] = (i == 0) ? 0.0 : c[i];
+    }
+  }
+  return 0;
+}
+
+// ---------------------------------------------------------------------------
+// Graded product over nested table codes (the reading above): for b_k > 0,
+// w_hat[k][n] = lut[k][2^b_k + (q[k][n] >> (bmax - b_k))] (binary16), no
+// midpoint, no scale or zero point; y[n] = sum over k ascending of
+// x_k * w_hat[k][n], bound[n] = sum of |x_k * w_hat[k][n]|. A width above
+// bmax is an error. nthreads > 1 splits the columns as orc_vmm_bmax does.
+// ---------------------------------------------------------------------------
+int orc_vmm_lut(const uint16_t* x, const uint8_t* q, const uint16_t* lut, const uint8_t* bits, int K, int N,
+                int bmax, double* y, double* bound, int nthreads) {
+  if (K < 0 || N <= 0 || bmax < 1 || bmax > 8) return -1;
+  for (int k = 0; k < K; ++k) if (bits[k] > bmax) return -1;
+  const int E = 1 << (bmax + 1);
+  for (int n = 0; n < N; ++n) { y[n] = 0.0; if (bound) bound[n] = 0.0; }
+  if (nthreads < 1) nthreads = 1;
+  const int nchunks = nthreads;
+#pragma omp parallel for num_threads(nthreads) schedule(static, 1) if (nthreads > 1)
+  for (int t = 0; t < nchunks; ++t) {
+    const int n0 = (int)((long long)N * t / nchunks);
+    const int n1 = (int)((long long)N * (t + 1) / nchunks);
+    for (int k = 0; k < K; ++k) {
+      const int b = bits[k];
+      if (b == 0) continue;
+      const double xk = orc_f16_to_f64(x[k]);
+      const uint16_t* row = lut + (size_t)k * E + (1 << b);
+      for (int n = n0; n < n1; ++n) {
+        const double w = orc_f16_to_f64(row[q[(size_t)k * N + n] >> (bmax - b)]);
+        const double t2 = xk * w;
+        y[n] += t2;
+        if (bound) bound[n] += std::fabs(t2);
+      }
+    }
+  }
+  return 0;
+}
+
 }  // extern "C"
