@@ -374,4 +374,47 @@ grinqh_status grinqh_select_vmm_batch(const grinqh_layout* layout, const void* p
   return cuda_status(launch_vmm(a, (cudaStream_t)stream, true));
 }
 
+grinqh_status grinqh_pack_codes(const grinqh_layout* layout, const uint8_t* codes, void* packed, void* stream) {
+  if (!layout_ok(layout) || !codes || !packed) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(packed, 16)) return GRINQH_ERR_ALIGNMENT;
+  const grinqh_layout& L = *layout;
+  return cuda_status(launch_pack_codes(codes, L.K, L.N, L.n_tiles, L.b_max, packed, (cudaStream_t)stream));
+}
+
+grinqh_status grinqh_lut_bytes(const grinqh_layout* layout, size_t* bytes) {
+  if (!layout_ok(layout) || !bytes) return GRINQH_ERR_INVALID_ARG;
+  *bytes = (size_t)layout->K << (layout->b_max + 2);
+  return GRINQH_OK;
+}
+
+grinqh_status grinqh_vmm_lut(const grinqh_layout* layout, const void* packed, const uint16_t* lut,
+                             const uint16_t* x, const int32_t* idx, const int32_t* offsets, const uint8_t* classes,
+                             int32_t n_classes, float* y, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!layout_ok(layout) || !valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
+  if (!classes_fit(classes, n_classes, layout->b_max)) return GRINQH_ERR_INVALID_ARG;
+  if (!packed || !lut || !x || !idx || !offsets || !y) return GRINQH_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(lut, 16) || !aligned(x, 2) || !aligned(idx, 4) || !aligned(offsets, 4) ||
+      !aligned(y, 4))
+    return GRINQH_ERR_ALIGNMENT;
+  const grinqh_layout& L = *layout;
+  const size_t need = vmm_workspace_bytes(L.n_tiles, L.tile_n);
+  if (!workspace || workspace_bytes < need) return GRINQH_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return GRINQH_ERR_ALIGNMENT;
+  VmmArgs a{};
+  a.K = L.K;
+  a.N = L.N;
+  a.n_tiles = L.n_tiles;
+  a.b_max = L.b_max;
+  a.packed = (const uint8_t*)packed;
+  a.lut = (const uint8_t*)lut;
+  a.x = x;
+  a.idx = idx;
+  a.offsets = offsets;
+  a.y = y;
+  a.status = (uint32_t*)workspace;
+  a.partial = (float*)((char*)workspace + 16);
+  a.ct = table(classes, n_classes);
+  return cuda_status(launch_vmm_lut(a, (cudaStream_t)stream));
+}
+
 }  // extern "C"

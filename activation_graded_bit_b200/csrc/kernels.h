@@ -13,6 +13,11 @@ cudaError_t launch_pack(const float* W, int K, int N, int n_tiles, int n_groups,
 cudaError_t launch_unpack(const void* packed, const uint8_t* bits, int K, int N, int n_tiles, int b_max,
                           uint8_t* codes, cudaStream_t st);
 
+// Planes of given b_max-bit codes [K][N] (bits above b_max ignored); the
+// records' scale/zero words are written as zero.
+cudaError_t launch_pack_codes(const uint8_t* codes, int K, int N, int n_tiles, int b_max, void* packed,
+                              cudaStream_t st);
+
 // Full-width w_hat = s (q - z) as binary16, [K][N] row-major.
 cudaError_t launch_dequant(const void* packed, int K, int N, int n_tiles, int b_max, uint16_t* out,
                            cudaStream_t st);
@@ -43,6 +48,7 @@ struct VmmArgs {
   float* partial;       // workspace: per-row-split partial sums [tokens][R][n_tiles * 1024]
   ClassTable ct;
   int tokens;           // batch: token t reads x + t K and writes y + t N (1 for a single vector)
+  const uint8_t* lut;   // grinqh_vmm_lut: binary16 tables, 2^(b_max+2) bytes per row, heap order
 };
 
 size_t vmm_workspace_bytes(int n_tiles, int tile_n);
@@ -52,6 +58,8 @@ size_t vmm_workspace_bytes_batch(int n_tiles, int tokens);
 // a.idx / a.offsets; K <= vmm_fused_max_k().
 cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused = false);
 int vmm_fused_max_k();
+// Nested table codes: a.lut holds the tables; a.idx / a.offsets as for launch_vmm.
+cudaError_t launch_vmm_lut(const VmmArgs& a, cudaStream_t st);
 
 // grinqh_vmm_noalloc's shared device scratch: its size, and its address on the
 // current device.

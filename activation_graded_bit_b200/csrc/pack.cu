@@ -225,4 +225,41 @@ cudaError_t launch_unpack(const void* packed, const uint8_t* bits, int K, int N,
   return cudaGetLastError();
 }
 
+// Planes of codes given by the caller (nested table codes, or any b_max-bit
+// codes quantised elsewhere): one CTA per (row k, tile t), the tile's codes
+// staged in shared memory (bits above b_max dropped, columns past N zero), the
+// record's scale/zero words written as zero, then the plane-pair words as in
+// pack_kernel.
+__global__ void __launch_bounds__(256) pack_codes_kernel(const uint8_t* __restrict__ codes, int K, int N,
+                                                         int n_tiles, int b_max, uint8_t* __restrict__ packed) {
+  __shared__ uint8_t tile[kTileN];
+  const int k = blockIdx.x, t = blockIdx.y;
+  uint8_t* rec = packed + ((size_t)k * n_tiles + t) * record_bytes_for(b_max);
+  const uint32_t keep = (1u << b_max) - 1u;
+  for (int e = threadIdx.x; e < kTileN; e += 256) {
+    const int n = t * kTileN + e;
+    tile[e] = (n < N) ? (uint8_t)(codes[(size_t)k * N + n] & keep) : (uint8_t)0;
+  }
+  if (threadIdx.x < kMetaBytes / 4) reinterpret_cast<uint32_t*>(rec)[threadIdx.x] = 0u;
+  __syncthreads();
+  const int sp = threadIdx.x >> 6, wi = threadIdx.x & 63;
+  if (2 * sp >= b_max) return;
+  const int cbase = 32 * (wi >> 1) + 16 * (wi & 1);
+  uint32_t word = 0;
+#pragma unroll 8
+  for (int L = 0; L < 32; ++L) {
+    int c16, l;
+    pair_col_at(sp, L, c16, l);
+    word |= (uint32_t)((tile[cbase + c16] >> (b_max - 1 - (2 * sp + l))) & 1u) << L;
+  }
+  reinterpret_cast<uint32_t*>(rec + kMetaBytes + sp * kPairBytes)[wi] = word;
+}
+
+cudaError_t launch_pack_codes(const uint8_t* codes, int K, int N, int n_tiles, int b_max, void* packed,
+                              cudaStream_t st) {
+  dim3 grid(K, n_tiles);
+  pack_codes_kernel<<<grid, 256, 0, st>>>(codes, K, N, n_tiles, b_max, (uint8_t*)packed);
+  return cudaGetLastError();
+}
+
 }  // namespace grinqh

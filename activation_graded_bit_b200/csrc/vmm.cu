@@ -510,6 +510,261 @@ __global__ void __launch_bounds__(32 * kRedChains) reduce_partials_kernel(const 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Nested look-up-table codes (grinqh_vmm_lut): the same records of b_max-bit
+// codes in plane pairs, read and rebuilt as above, but a code's value is an
+// entry of its row's table for the row's width b, w_hat = T_k[2^b + c_b] with
+// c_b the code's top b bits (no bin midpoint, no scale or zero point; the
+// records' scale/zero words are not read). Tables are binary16 in heap order,
+// 2^(b_max+1) entries per row, so width b's 2^b entries are contiguous.
+//
+// Per row in flight the warp copies the width-b table into shared memory with
+// cp.async (no registers), issued with the row's plane loads three rows ahead.
+// Before the row's products the warp rewrites it as fp32 values times x_k (an
+// exact product of two binary16 values) in a per-warp slot aligned to 1 KB, so
+// a code's shared address is the slot address with its low bits replaced by
+// 4 c_b: for b <= 6 one shift per register of four codes and one byte-permute
+// per code, for b = 7, 8 a shift and a mask per code. Each weight then costs a
+// shared load and half of a paired fp32 add.
+constexpr int kLutRaw = 256;                        // binary16 entries of the widest table (b = 8)
+constexpr int kLutSlot = 1024;                      // bytes of one fp32 table slot
+
+struct __align__(16) LutSmem {
+  uint32_t rows[kIdxCap];                         // k | b << 24 of this CTA's rows, one pass
+  float red[kWarps * kRedStride];                 // per-warp column sums
+  uint16_t raw[kWarps][kDepth][kLutRaw];          // tables as copied, one slot per row in flight
+  uint8_t tab[kWarps * kDepth * kLutSlot + kLutSlot];   // x_k-scaled fp32 tables (1 KB-aligned slots)
+  int off[10];
+  int width[9];
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16_if(bool on, uint32_t dst, const void* src) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %2, 0;\n\t@p cp.async.cg.shared.global [%0], [%1], 16;\n\t}" ::"r"(dst),
+      "l"(src), "r"((uint32_t)on)
+      : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+__device__ __forceinline__ void warp_sync_mem() { asm volatile("bar.warp.sync 0xffffffff;" ::: "memory"); }
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+
+// Issue the loads of one row (k | b << 24, b >= 1): x_k, this lane's words of
+// plane pairs 0..ceil(b/2)-1, and the row's width-b table into the warp's raw
+// slot (entries [0, 16) of the row for b <= 3, which hold widths 1..3, else
+// entries [2^b, 2^(b+1)); 16-byte copies, lane l the l-th), as one cp.async
+// group. The table buffer holds 2^(kBmax+2) bytes per row, 16-byte aligned.
+template <int kBmax>
+__device__ __forceinline__ void load_row_lut(const uint16_t* __restrict__ x, const uint8_t* __restrict__ lut,
+                                             const RowAddr& ra, uint32_t info, uint32_t raw, int lane,
+                                             RowRegs& r) {
+  constexpr uint32_t kRowBytes = 1u << (kBmax + 2);
+  const uint32_t k = info & 0xFFFFFFu, b = info >> 24;
+  const uint32_t sec = k * ra.nt33 + ra.t33;
+  r.b = b;
+  r.xh = __ldg(x + k);
+  const uint8_t* pw = ra.pairs + 32ull * sec;
+  ld_stream2_at<0>(pw, r.p[0], r.p[1]);
+  ld_stream2_at_if<1 * kPairBytes>(b > 2, pw, r.p[2], r.p[3]);
+  ld_stream2_at_if<2 * kPairBytes>(b > 4, pw, r.p[4], r.p[5]);
+  ld_stream2_at_if<3 * kPairBytes>(b > 6, pw, r.p[6], r.p[7]);
+  const uint32_t off = (b <= 3) ? 0u : (2u << b);
+  const uint32_t bytes = (b <= 3) ? (kRowBytes < 32u ? kRowBytes : 32u) : (2u << b);
+  const uint32_t l16 = 16u * (uint32_t)lane;
+  cp_async16_if(l16 < bytes, raw + l16, lut + (size_t)k * kRowBytes + off + l16);
+  cp_async_commit();
+}
+
+// The products of one row: wait for its table (the kDepth - 1 rows loaded after
+// it may still be in flight), scale it by x_k into the fp32 slot, then add the
+// looked-up values of this lane's 32 columns. acc[2j] holds columns 4j, 4j+1 and
+// acc[2j+1] columns 4j+2, 4j+3 of the lane's 32.
+template <int kBmax>
+__device__ __forceinline__ void row_lut(const RowRegs& r, uint32_t raw, uint32_t tab, int lane,
+                                        float2 (&acc)[16]) {
+  cp_async_wait<kDepth - 1>();
+  warp_sync_mem();
+  const uint32_t b = r.b;
+  const float xk = __half2float(__ushort_as_half((unsigned short)r.xh));
+  const uint32_t e0 = (b <= 3) ? (1u << b) : 0u;   // width b's first entry in the raw slot
+  for (uint32_t c = (uint32_t)lane; c < (1u << b); c += 32u)
+    sts_f32(tab + 4u * c, xk * half_bits_to_float(lds_u16(raw + 2u * (e0 + c))));
+  warp_sync_mem();
+  uint32_t R[8];
+  float mid;
+  assemble_row<kBmax>(r, R, mid);
+  if (b <= 6) {
+    // byte i of R >> (6 - b) is 4 c_b of column 4j + i (the bits below a code are zero)
+    const uint32_t sh = 6u - b;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t t = R[j] >> sh;
+      const float v0 = lds_f32(__byte_perm(t, tab, 0x7650));
+      const float v1 = lds_f32(__byte_perm(t, tab, 0x7651));
+      const float v2 = lds_f32(__byte_perm(t, tab, 0x7652));
+      const float v3 = lds_f32(__byte_perm(t, tab, 0x7653));
+      acc[2 * j] = __fadd2_rn(acc[2 * j], make_float2(v0, v1));
+      acc[2 * j + 1] = __fadd2_rn(acc[2 * j + 1], make_float2(v2, v3));
+    }
+  } else {
+    const uint32_t mask = ((1u << b) - 1u) << 2;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float v0 = lds_f32(((R[j] << (b - 6u)) & mask) | tab);
+      const float v1 = lds_f32(((R[j] >> (14u - b)) & mask) | tab);
+      const float v2 = lds_f32(((R[j] >> (22u - b)) & mask) | tab);
+      const float v3 = lds_f32(((R[j] >> (30u - b)) & mask) | tab);
+      acc[2 * j] = __fadd2_rn(acc[2 * j], make_float2(v0, v1));
+      acc[2 * j + 1] = __fadd2_rn(acc[2 * j + 1], make_float2(v2, v3));
+    }
+  }
+}
+
+template <int kBmax>
+__global__ void __launch_bounds__(kThreads, 1) vmm_lut_kernel(const VmmArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  LutSmem& s = *reinterpret_cast<LutSmem*>(smem_raw);
+  const int tid = threadIdx.x, h = tid >> 5, w = tid & 31;
+  const int t = blockIdx.x, r = blockIdx.y, R = gridDim.y;
+  const uint16_t* xv = a.x;
+
+  // list positions r + R e, the width-0 prefix skipped (as grinqh_vmm)
+  const int nfull = (a.K > r) ? (a.K - r + R - 1) / R : 0;
+  constexpr int kPre = 4;
+  int pre_idx[kPre];
+  pdl_wait();
+#pragma unroll
+  for (int i = 0; i < kPre; ++i) {
+    const int e = tid + i * kThreads;
+    pre_idx[i] = (e < nfull) ? __ldg(a.idx + r + R * e) : 0;
+  }
+  if (tid <= a.ct.n) s.off[tid] = a.offsets[tid];
+#pragma unroll
+  for (int c = 0; c < 9; ++c)
+    if (tid == c && c < a.ct.n) s.width[c] = a.ct.width[c];
+  __syncthreads();
+  pdl_launch_dependents();
+
+  const int n = a.ct.n;
+  const int a0 = (s.width[0] == 0) ? s.off[1] : 0;
+  const int e0 = (a0 > r) ? (a0 - r + R - 1) / R : 0;
+  const int nq_total = nfull - e0;
+
+  float2 acc[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) acc[c] = make_float2(0.0f, 0.0f);
+
+  const uint32_t raw0 = smem_u32(&s.raw[h][0][0]);
+  const uint32_t tab0 = ((smem_u32(s.tab) + (kLutSlot - 1u)) & ~(uint32_t)(kLutSlot - 1)) +
+                        (uint32_t)h * (kDepth * kLutSlot);
+  for (int qb = 0; qb < nq_total; qb += kIdxCap) {
+    const int nq = min(kIdxCap, nq_total - qb);
+    __syncthreads();
+    if (nfull <= kPre * kThreads) {
+#pragma unroll
+      for (int i = 0; i < kPre; ++i) {
+        const int e = tid + i * kThreads;
+        if (e >= e0 && e < nfull) {
+          const int pos = r + R * e;
+          int j = 0;
+          for (int c = 1; c < n; ++c) j += (pos >= s.off[c]) ? 1 : 0;
+          s.rows[e - e0] = (uint32_t)pre_idx[i] | ((uint32_t)s.width[j] << 24);
+        }
+      }
+    } else {
+      for (int e = tid; e < nq; e += kThreads) {
+        const int pos = r + R * (e0 + qb + e);
+        int j = 0;
+        for (int c = 1; c < n; ++c) j += (pos >= s.off[c]) ? 1 : 0;
+        s.rows[e] = (uint32_t)a.idx[pos] | ((uint32_t)s.width[j] << 24);
+      }
+    }
+    __syncthreads();
+    const int nrow = (nq > h) ? (nq - h + kWarps - 1) / kWarps : 0;
+    const RowAddr ra = row_addr(a, t, w);
+    RowRegs S[kDepth];
+    // one cp.async group per row slot, empty where there is no row, so that the
+    // row being multiplied always has exactly kDepth - 1 groups after its own
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d) {
+      if (d < nrow) load_row_lut<kBmax>(xv, a.lut, ra, s.rows[h + kWarps * d], raw0 + d * 2 * kLutRaw, w, S[d]);
+      else cp_async_commit();
+    }
+#pragma unroll 1
+    for (int m = kDepth; m < min(nrow, kDepth + kL2Ahead); ++m) prefetch_row_l2(ra, s.rows[h + kWarps * m]);
+    int m0 = 0;
+#pragma unroll 1
+    for (; m0 + 2 * kDepth + kL2Ahead <= nrow; m0 += kDepth) {
+#pragma unroll
+      for (int d = 0; d < kDepth; ++d) {
+        const int m = m0 + d;
+        row_lut<kBmax>(S[d], raw0 + d * 2 * kLutRaw, tab0 + d * kLutSlot, w, acc);
+        load_row_lut<kBmax>(xv, a.lut, ra, s.rows[h + kWarps * (m + kDepth)], raw0 + d * 2 * kLutRaw, w, S[d]);
+        prefetch_row_l2(ra, s.rows[h + kWarps * (m + kDepth + kL2Ahead)]);
+      }
+    }
+#pragma unroll 1
+    for (int m = m0 + kDepth + kL2Ahead; m < nrow; ++m) prefetch_row_l2(ra, s.rows[h + kWarps * m]);
+#pragma unroll 1
+    for (; m0 < nrow; m0 += kDepth) {
+#pragma unroll
+      for (int d = 0; d < kDepth; ++d) {
+        const int m = m0 + d;
+        if (m < nrow) {
+          row_lut<kBmax>(S[d], raw0 + d * 2 * kLutRaw, tab0 + d * kLutSlot, w, acc);
+          if (m + kDepth < nrow)
+            load_row_lut<kBmax>(xv, a.lut, ra, s.rows[h + kWarps * (m + kDepth)], raw0 + d * 2 * kLutRaw, w, S[d]);
+          else
+            cp_async_commit();
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+
+  // CTA reduction over the 16 warps, as grinqh_vmm
+  float* red = s.red;
+  {
+    float* dst = red + h * kRedStride + w;   // slot c*33 + w holds column 32w + c
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      dst[(4 * j + 0) * kRedPitch] = acc[2 * j].x;
+      dst[(4 * j + 1) * kRedPitch] = acc[2 * j].y;
+      dst[(4 * j + 2) * kRedPitch] = acc[2 * j + 1].x;
+      dst[(4 * j + 3) * kRedPitch] = acc[2 * j + 1].y;
+    }
+  }
+  __syncthreads();
+  float* out = (R == 1) ? a.y : a.partial + (size_t)r * a.n_tiles * kTileN;
+  const int limit = (R == 1) ? a.N : a.n_tiles * kTileN;
+#pragma unroll
+  for (int e = tid; e < kTileN; e += kThreads) {
+    float v = 0.0f;
+#pragma unroll
+    for (int rl = 0; rl < kWarps; ++rl) v += red[rl * kRedStride + (e % kWords) * kRedPitch + e / kWords];
+    const int col = t * kTileN + e;
+    if (col < limit) out[col] = v;
+  }
+}
+
 static int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -605,6 +860,62 @@ cudaError_t launch_vmm(const VmmArgs& a, cudaStream_t st, bool fused) {
   if (a.tokens > 1)
     return cudaLaunchKernelEx(&rc, reduce_partials_kernel<true>, (const float*)a.partial, R, a.n_tiles * kTileN,
                               a.y, a.N);
+  return cudaLaunchKernelEx(&rc, reduce_partials_kernel<false>, (const float*)a.partial, R, a.n_tiles * kTileN, a.y,
+                            a.N);
+}
+
+// grinqh_vmm_lut: the table kernel, then the partial sums as for grinqh_vmm.
+template <int kBmax>
+static cudaError_t launch_lut_one(const cudaLaunchConfig_t& cfg, const VmmArgs& a) {
+  static_assert(sizeof(LutSmem) + 16 <= 227 * 1024, "table kernel shared memory");
+  return cudaLaunchKernelEx(&cfg, vmm_lut_kernel<kBmax>, a);
+}
+
+static cudaError_t ensure_lut_smem_attrs() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<bool> done[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  const int smem = (int)sizeof(LutSmem);
+  const cudaFuncAttribute at = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  e = cudaFuncSetAttribute(vmm_lut_kernel<8>, at, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(vmm_lut_kernel<6>, at, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(vmm_lut_kernel<4>, at, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(vmm_lut_kernel<2>, at, smem);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev].store(true, std::memory_order_release);
+  return e;
+}
+
+cudaError_t launch_vmm_lut(const VmmArgs& a, cudaStream_t st) {
+  cudaError_t e = ensure_lut_smem_attrs();
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  const int R = row_splits(a.n_tiles);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.n_tiles, R, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (int)sizeof(LutSmem);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  switch (a.b_max) {
+    case 2: e = launch_lut_one<2>(cfg, a); break;
+    case 4: e = launch_lut_one<4>(cfg, a); break;
+    case 6: e = launch_lut_one<6>(cfg, a); break;
+    case 8: e = launch_lut_one<8>(cfg, a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess || R == 1) return e;
+  cudaLaunchConfig_t rc = {};
+  rc.gridDim = dim3((a.N + 31) / 32, 1, 1);
+  rc.blockDim = dim3(32 * kRedChains, 1, 1);
+  rc.stream = st;
+  rc.attrs = attr;
+  rc.numAttrs = 1;
   return cudaLaunchKernelEx(&rc, reduce_partials_kernel<false>, (const float*)a.partial, R, a.n_tiles * kTileN, a.y,
                             a.N);
 }

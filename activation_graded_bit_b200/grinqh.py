@@ -71,13 +71,17 @@ _batch_ws = _sig("grinqh_vmm_batch_workspace_bytes", [_LP, _I, ctypes.POINTER(ct
 _select_vmm_batch = _sig("grinqh_select_vmm_batch", [_LP, _P, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
 _dequant = _sig("grinqh_dequant", [_LP, _P, _P, _P])
 _prefill = _sig("grinqh_prefill", [_LP, _P, _P, _I, _P, _P, _P])
+_pack_codes = _sig("grinqh_pack_codes", [_LP, _P, _P, _P])
+_lut_bytes = _sig("grinqh_lut_bytes", [_LP, ctypes.POINTER(ctypes.c_size_t)])
+_vmm_lut = _sig("grinqh_vmm_lut", [_LP, _P, _P, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
 
 # Every exported symbol of the C ABI, for the export check in the tests.
 EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grinqh_layout_init_bmax", "grinqh_pack",
            "grinqh_unpack_codes", "grinqh_maxent_distribution", "grinqh_calibrate_workspace_bytes",
            "grinqh_calibrate", "grinqh_select", "grinqh_vmm_workspace_bytes", "grinqh_vmm",
            "grinqh_vmm_noalloc", "grinqh_select_vmm", "grinqh_vmm_batch_workspace_bytes",
-           "grinqh_select_vmm_batch", "grinqh_dequant", "grinqh_prefill")
+           "grinqh_select_vmm_batch", "grinqh_dequant", "grinqh_prefill", "grinqh_pack_codes",
+           "grinqh_lut_bytes", "grinqh_vmm_lut")
 
 
 def version() -> str:
@@ -303,4 +307,35 @@ def vmm_noalloc(p: PackedLayer, x: torch.Tensor, sel: Selection, y: torch.Tensor
     cb, n = _classes_buf(sel.classes)
     _check(_vmm_noalloc(ctypes.byref(p.layout), _ptr(p.packed), _ptr(x), _ptr(sel.idx), _ptr(sel.offsets),
                         ctypes.addressof(cb), n, _ptr(y), _stream(stream)), "grinqh_vmm_noalloc")
+    return y
+
+def pack_codes(codes: torch.Tensor, b_max: int = 8, out: Optional[PackedLayer] = None, stream=None) -> PackedLayer:
+    """grinqh_pack_codes: bit planes of given b_max-bit codes (uint8 [K, N] CUDA
+    tensor, e.g. nested look-up-table codes); the records' scale/zero words are zero."""
+    assert codes.dtype == torch.uint8 and codes.is_cuda and codes.is_contiguous() and codes.dim() == 2
+    K, N = codes.shape
+    p = out if out is not None else empty_packed(K, N, codes.device, b_max)
+    _check(_pack_codes(ctypes.byref(p.layout), _ptr(codes), _ptr(p.packed), _stream(stream)), "grinqh_pack_codes")
+    return p
+
+
+def lut_bytes(L: Layout) -> int:
+    """grinqh_lut_bytes: K * 2^(b_max+2) (binary16 tables in heap order per row)."""
+    n = ctypes.c_size_t(0)
+    _check(_lut_bytes(ctypes.byref(L), ctypes.byref(n)), "grinqh_lut_bytes")
+    return n.value
+
+
+def vmm_lut(p: PackedLayer, lut: torch.Tensor, x: torch.Tensor, sel: Selection, workspace: torch.Tensor,
+            y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """grinqh_vmm_lut: y[N] fp32 = x . W_hat with w_hat[k][n] = lut[k][2^b_k + c_b]
+    (lut: 16-bit [K, 2^(b_max+1)] CUDA tensor of binary16 bit patterns, heap order)."""
+    assert lut.is_cuda and lut.is_contiguous() and lut.element_size() == 2
+    assert lut.numel() * 2 == lut_bytes(p.layout), "table buffer size"
+    if y is None:
+        y = torch.empty(p.N, dtype=torch.float32, device=p.packed.device)
+    cb, n = _classes_buf(sel.classes)
+    _check(_vmm_lut(ctypes.byref(p.layout), _ptr(p.packed), _ptr(lut), _ptr(x), _ptr(sel.idx), _ptr(sel.offsets),
+                    ctypes.addressof(cb), n, _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                    _stream(stream)), "grinqh_vmm_lut")
     return y

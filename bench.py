@@ -779,6 +779,100 @@ def run_batch(args):
                       "points": out}))
 
 
+def run_lut(args):
+    """Nested look-up-table codes through grinqh_vmm_lut on the decode step (the
+    same 21 (linear, width) pairs, selections and two rotated copies as the main
+    run): synthetic b_max-bit codes and binary16 tables (timing does not depend
+    on their values), microseconds per VMM and per select+VMM pair, graph-replayed,
+    with grinqh_vmm on the uniform codes of the same pairs timed beside it."""
+    import torch
+    from activation_graded_bit_b200 import grinqh as g
+    from activation_graded_bit_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    pairs = build_workload(g, wl, torch, dev, copies=2)
+    gen = torch.Generator(device=dev)
+    E = 1 << (BMAX + 1)
+    tot_alg = 0.0
+    for i, pr in enumerate(pairs):
+        K, N = pr["K"], pr["N"]
+        gen.manual_seed(2_000_003 + 7919 * i)
+        codes = torch.randint(0, 1 << BMAX, (K, N), generator=gen, device=dev, dtype=torch.uint8)
+        pr["packed_lut"] = g.pack_codes(codes, b_max=BMAX)
+        del codes
+        pr["lut"] = torch.randn((K, E), generator=gen, device=dev).half().view(torch.int16).contiguous()
+        if pr["copy"] == 0:
+            bits = pr["sel"].bits.cpu().numpy().astype(np.int64)
+            active = bits > 0
+            # planes + each active row's width-b table once + x + channel list + y
+            tot_alg += (bits.sum() * N / 8.0 + float((2 << bits[active]).sum()) + 2.0 * K
+                        + 4.0 * int(active.sum()) + 4.0 * N)
+    torch.cuda.synchronize()
+    groups = {}
+    for pr in pairs:
+        groups.setdefault(pr["copy"], []).append(pr)
+    copies = sorted(groups)
+    n_pairs = len(groups[copies[0]])
+    stream = torch.cuda.Stream(device=dev)
+
+    def graphs_of(fn):
+        out = {}
+        with torch.cuda.stream(stream):
+            for c in copies:
+                fn(c)
+            torch.cuda.synchronize()
+            for c in copies:
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=stream):
+                    fn(c)
+                out[c] = gr
+        torch.cuda.synchronize()
+        return out
+
+    def lut_only(c):
+        for pr in groups[c]:
+            g.vmm_lut(pr["packed_lut"], pr["lut"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
+
+    def lut_pairs(c):
+        for pr in groups[c]:
+            g.select(pr["x"], pr["th"], CLASSES, out=pr["sel"], stream=stream)
+            g.vmm_lut(pr["packed_lut"], pr["lut"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
+
+    def uniform_only(c):
+        for pr in groups[c]:
+            g.vmm(pr["packed"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
+
+    def timed(graphs):
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup):
+                graphs[copies[i % len(copies)]].replay()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(args.steps):
+                graphs[copies[i % len(copies)]].replay()
+            e1.record(stream)
+        stream.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / (args.steps * n_pairs)
+
+    us_lut = timed(graphs_of(lut_only))
+    us_pair = timed(graphs_of(lut_pairs))
+    us_uni = timed(graphs_of(uniform_only))
+    assert all(bool(torch.isfinite(pr["y"]).all()) for pr in pairs)
+    peak, peak_kind = _peaks()
+    achieved = tot_alg / n_pairs / (us_lut * 1e-6) / 1e9
+    print(json.dumps({"metric": "grinqh_vmm_lut: µs per batch-1 VMM over nested look-up-table codes",
+                      "value": round(us_lut, 4), "unit": "µs", "higher_is_better": False, "steps": args.steps,
+                      "warmup": args.warmup, "data": "synthetic codes and tables",
+                      "config": {"workload": WORKLOAD, "classes": list(CLASSES), "b_max": BMAX,
+                                 "l2": "two packed copies of the layer set rotate (inputs larger than L2)"},
+                      "select_plus_vmm_lut_us": round(us_pair, 4), "vmm_uniform_us_same_run": round(us_uni, 4),
+                      "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                                   "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                                   "bytes_per_step": tot_alg}}))
+
+
 def run_prefill(args):
     """The prefill path on the Llama3-8B linears (Section 4 of the paper: unpack at
     full b_max precision, then a dense product): for T tokens, microseconds of
@@ -871,6 +965,7 @@ def main():
     ap.add_argument("--stack-steps", type=int, default=256)
     ap.add_argument("--batch", action="store_true", help="batch 1..16 through the batched fused call (one JSON line)")
     ap.add_argument("--prefill", action="store_true", help="prefill path: dequant + GEMM on the linears (one JSON line)")
+    ap.add_argument("--lut", action="store_true", help="nested look-up-table codes through grinqh_vmm_lut (one JSON line)")
     ap.add_argument("--bmax", type=int, default=8, choices=(4, 6, 8),
                     help="stored code width; 4 or 6 grade into the classes {0, 2, ..., b_max}")
     ap.add_argument("--family", default="llama3", choices=("llama3", "qwen3"),
@@ -900,6 +995,9 @@ def main():
         return
     if args.prefill:
         run_prefill(args)
+        return
+    if args.lut:
+        run_lut(args)
         return
     if args.profile:
         run_profile_case(args)

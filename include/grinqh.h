@@ -24,6 +24,10 @@
  *   grinqh_vmm_noalloc       grinqh_vmm on the library's own static scratch
  *   grinqh_dequant / grinqh_prefill   full-width weights and the dense prefill
  *                            product for many tokens
+ * and, for nested look-up-table codes (any-precision style) quantised elsewhere:
+ *   grinqh_pack_codes        bit planes of given b_max-bit codes
+ *   grinqh_lut_bytes         size of the per-row table buffer
+ *   grinqh_vmm_lut           y = x . W_hat with w_hat a table entry per width
  *
  * Conventions for every call:
  *   - W is K x N: K input channels (rows), N output channels (columns).
@@ -179,6 +183,48 @@ grinqh_status grinqh_dequant(const grinqh_layout* layout, const void* packed, ui
  */
 grinqh_status grinqh_prefill(const grinqh_layout* layout, const void* packed, const uint16_t* X, int32_t T,
                              float* Y, uint16_t* W16, void* stream);
+
+/*
+ * Nested look-up-table codes. Paper: Section 3.3 ("Storage Layout and Weight
+ * Loading": the planes need a nested quantisation, met by uniform codes and by
+ * k-means codes such as any-precision LLM's; with such tables no midpoint term
+ * is used, the nested levels being centred already), Section 4 ("Models and
+ * Baselines": any-precision LLM weights at b_max = 8) and Appendix E.2.
+ * Library reading: each row k has one table per width b = 1..b_max; the top b
+ * bits c_b = q >> (b_max - b) of a b_max-bit code q select its entry, and
+ * w_hat = T_k[2^b + c_b]. The tables of a row are stored in heap order as
+ * binary16: entry 2^b + c is entry c of width b, entries 0 and 1 are never read,
+ * so a row holds 2^(b_max+1) entries (2^(b_max+2) bytes, 1 KB at b_max = 8).
+ */
+
+/*
+ * Bit planes of caller-given codes: the packed layout of grinqh_layout_init_bmax
+ * with every record's scale/zero words zero and the planes of codes[k][n] (only
+ * its low b_max bits are used). Columns >= N are zero bits.
+ *   codes   device uint8 [K][N] row-major, any alignment.
+ *   packed  device, packed_bytes, 16-byte aligned, fully overwritten.
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ */
+grinqh_status grinqh_pack_codes(const grinqh_layout* layout, const uint8_t* codes, void* packed, void* stream);
+
+/* Bytes of the table buffer of grinqh_vmm_lut: K * 2^(b_max+2). */
+grinqh_status grinqh_lut_bytes(const grinqh_layout* layout, size_t* bytes);
+
+/*
+ * y = x . W_hat over nested table codes, graded as grinqh_vmm: for a channel of
+ * width b_k > 0, w_hat[k][n] = lut[k][2^b_k + (q[k][n] >> (b_max - b_k))]; rows of
+ * width 0 are not read. Reads only the top b_k planes of row k (not its
+ * scale/zero words) and the b_k-bit part of row k's table.
+ *   packed     device, from grinqh_pack_codes (or grinqh_pack: its codes are
+ *              then read as table indices), 16-byte aligned.
+ *   lut        device binary16 [K][2^(b_max+1)] in heap order, 16-byte aligned.
+ *   x, idx, offsets, classes, n_classes, y, workspace, workspace_bytes: as for
+ *              grinqh_vmm (the same selection and the same workspace size).
+ * Errors: INVALID_ARG (also a class wider than b_max), ALIGNMENT, WORKSPACE, CUDA.
+ */
+grinqh_status grinqh_vmm_lut(const grinqh_layout* layout, const void* packed, const uint16_t* lut,
+                             const uint16_t* x, const int32_t* idx, const int32_t* offsets, const uint8_t* classes,
+                             int32_t n_classes, float* y, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Maximum-entropy precision distribution P over a class set for a requested

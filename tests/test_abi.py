@@ -192,3 +192,32 @@ def test_prefill_validation_rejects_before_launch(g):
     assert g._prefill(ctypes.byref(L), P(0x1000), P(0x1001), 4, P(0x1000), P(0x1000), None) == 2  # X odd
     assert g._prefill(ctypes.byref(L), P(0x1000), P(0x1000), 4, P(0x1002), P(0x1000), None) == 2  # Y
     assert g._prefill(None, P(0x1000), P(0x1000), 4, P(0x1000), P(0x1000), None) == 1
+
+
+def test_lut_validation_rejects_before_launch(g):
+    P = ctypes.c_void_p
+    cl = (ctypes.c_uint8 * 5)(0, 2, 3, 4, 8)
+    cl6 = (ctypes.c_uint8 * 4)(0, 2, 4, 6)
+    L = g.layout(64, 1024)
+    L4 = g.layout(64, 1024, b_max=4)
+    n = ctypes.c_size_t()
+    assert g._lut_bytes(ctypes.byref(L), ctypes.byref(n)) == 0 and n.value == 64 * 1024
+    assert g._lut_bytes(ctypes.byref(L4), ctypes.byref(n)) == 0 and n.value == 64 * 64
+    assert g._lut_bytes(None, ctypes.byref(n)) == 1
+    assert g._pack_codes(ctypes.byref(L), None, P(0x1000), None) == 1
+    assert g._pack_codes(ctypes.byref(L), P(0x1001), P(0x1008), None) == 2     # packed not 16-byte aligned
+    need = g.vmm_workspace_bytes(L)
+
+    def vl(layout, lut=0x1000, x=0x1000, y=0x1000, classes=cl, nc=5, ws=0x1000, wsb=need):
+        return g._vmm_lut(ctypes.byref(layout), P(0x1000), P(lut), P(x), P(0x1000), P(0x1000),
+                          ctypes.addressof(classes), nc, P(y), P(ws), wsb, None)
+
+    assert vl(L, lut=0) == 1                  # no tables
+    assert vl(L, lut=0x1008) == 2             # tables not 16-byte aligned
+    assert vl(L, x=0x1001) == 2
+    assert vl(L, y=0x1002) == 2
+    assert vl(L, wsb=need - 1) == 4
+    assert vl(L4, classes=cl6, nc=4) == 1     # width 6 above b_max = 4
+    Lbad = g.layout(64, 1024)
+    Lbad.tile_n = 512
+    assert vl(Lbad) == 1

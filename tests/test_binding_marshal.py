@@ -88,6 +88,11 @@ def test_every_call_marshals_and_reports(g):
     _expect_invalid(lambda: g.vmm_noalloc(p, x, sel, y, stream=st))
     _expect_invalid(lambda: g.dequant(p, out=W16, stream=st))
     _expect_invalid(lambda: g.prefill(p, X, Y=Y, W16=W16, stream=st))
+    codes = FakeTensor((K, N), torch.uint8)
+    lut = FakeTensor((K, 512), torch.int16)
+    _expect_invalid(lambda: g.pack_codes(codes, out=p, stream=st))
+    _expect_invalid(lambda: g.lut_bytes(p.layout))
+    _expect_invalid(lambda: g.vmm_lut(p, lut, x, sel, ws, y=y, stream=st))
     # calls without a layout: invalid class sets
     _expect_invalid(lambda: g.select(x, th, (0, 4, 4), out=sel, stream=st))
     Xc = FakeTensor((8, K), torch.int16)
