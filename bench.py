@@ -481,8 +481,9 @@ def run_reference(args):
 
 
 def run_profile_case(args):
-    """One (linear, width) pair, `--iters` eager select+vmm calls, no timing: the
-    small case that ncu captures."""
+    """One (linear, width) pair, `--iters` eager select+vmm calls (select+vmm_lut
+    over synthetic table codes with --lut), no timing: the small case that ncu
+    captures."""
     import torch
     from activation_graded_bit_b200 import grinqh as g
     from activation_graded_bit_b200 import workloads as wl
@@ -501,12 +502,22 @@ def run_profile_case(args):
     ws = g.vmm_workspace(p.layout, dev)
     y = torch.empty(N, dtype=torch.float32, device=dev)
     sel = g.empty_selection(K, wl.CLASSES, dev)
+    if args.lut:
+        # nested table codes on the same layer: synthetic codes and tables
+        codes = torch.randint(0, 256, (K, N), generator=gen, device=dev, dtype=torch.uint8)
+        p = g.pack_codes(codes)
+        del codes
+        lut = torch.randn((K, 512), generator=gen, device=dev).half().view(torch.int16).contiguous()
     for _ in range(args.iters):
         g.select(x_d, th, wl.CLASSES, out=sel)
-        g.vmm(p, x_d, sel, ws, y=y)
+        if args.lut:
+            g.vmm_lut(p, lut, x_d, sel, ws, y=y)
+        else:
+            g.vmm(p, x_d, sel, ws, y=y)
     torch.cuda.synchronize()
     assert bool(torch.isfinite(y).all())
-    print("profile case %s @ %g bits: %d select+vmm calls" % (args.profile, args.bits, args.iters))
+    print("profile case %s @ %g bits: %d select+%s calls" % (args.profile, args.bits, args.iters,
+                                                              "vmm_lut" if args.lut else "vmm"))
 
 
 
@@ -996,7 +1007,7 @@ def main():
     if args.prefill:
         run_prefill(args)
         return
-    if args.lut:
+    if args.lut and not args.profile:
         run_lut(args)
         return
     if args.profile:
