@@ -72,6 +72,7 @@ _select_vmm_batch = _sig("grinqh_select_vmm_batch", [_LP, _P, _P, _I, _P, _P, _I
 _dequant = _sig("grinqh_dequant", [_LP, _P, _P, _P])
 _prefill = _sig("grinqh_prefill", [_LP, _P, _P, _I, _P, _P, _P])
 _pack_codes = _sig("grinqh_pack_codes", [_LP, _P, _P, _P])
+_lut_build = _sig("grinqh_lut_build", [_P, _I, _I, _I, _P, _P])
 _lut_bytes = _sig("grinqh_lut_bytes", [_LP, ctypes.POINTER(ctypes.c_size_t)])
 _vmm_lut = _sig("grinqh_vmm_lut", [_LP, _P, _P, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
 
@@ -81,7 +82,7 @@ EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grin
            "grinqh_calibrate", "grinqh_select", "grinqh_vmm_workspace_bytes", "grinqh_vmm",
            "grinqh_vmm_noalloc", "grinqh_select_vmm", "grinqh_vmm_batch_workspace_bytes",
            "grinqh_select_vmm_batch", "grinqh_dequant", "grinqh_prefill", "grinqh_pack_codes",
-           "grinqh_lut_bytes", "grinqh_vmm_lut")
+           "grinqh_lut_bytes", "grinqh_vmm_lut", "grinqh_lut_build")
 
 
 def version() -> str:
@@ -339,3 +340,18 @@ def vmm_lut(p: PackedLayer, lut: torch.Tensor, x: torch.Tensor, sel: Selection, 
                     ctypes.addressof(cb), n, _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),
                     _stream(stream)), "grinqh_vmm_lut")
     return y
+
+
+def lut_build(W, b_max: int = 8):
+    """grinqh_lut_build (host, offline): nested 2-means codes and binary16 tables of a
+    fp32 [K, N] weight matrix (numpy array or CPU tensor). Returns CPU tensors
+    (codes uint8 [K, N], tables int16 [K, 2^(b_max+1)] holding binary16 bit patterns)."""
+    import numpy as np
+    Wn = W.detach().cpu().numpy() if isinstance(W, torch.Tensor) else W
+    Wn = np.ascontiguousarray(Wn, np.float32)
+    assert Wn.ndim == 2
+    K, N = Wn.shape
+    codes = np.empty((K, N), np.uint8)
+    lut = np.empty((K, 1 << (b_max + 1)), np.int16)
+    _check(_lut_build(Wn.ctypes.data, K, N, b_max, codes.ctypes.data, lut.ctypes.data), "grinqh_lut_build")
+    return torch.from_numpy(codes), torch.from_numpy(lut)

@@ -24,7 +24,8 @@
  *   grinqh_vmm_noalloc       grinqh_vmm on the library's own static scratch
  *   grinqh_dequant / grinqh_prefill   full-width weights and the dense prefill
  *                            product for many tokens
- * and, for nested look-up-table codes (any-precision style) quantised elsewhere:
+ * and, for nested look-up-table codes (any-precision style):
+ *   grinqh_lut_build         offline nested 2-means codes and tables (host)
  *   grinqh_pack_codes        bit planes of given b_max-bit codes
  *   grinqh_lut_bytes         size of the per-row table buffer
  *   grinqh_vmm_lut           y = x . W_hat with w_hat a table entry per width
@@ -206,6 +207,24 @@ grinqh_status grinqh_prefill(const grinqh_layout* layout, const void* packed, co
  * Errors: INVALID_ARG, ALIGNMENT, CUDA.
  */
 grinqh_status grinqh_pack_codes(const grinqh_layout* layout, const uint8_t* codes, void* packed, void* stream);
+
+/*
+ * Offline construction of nested table codes on the host (no CUDA): any-precision
+ * style incremental upscaling (Appendix E.2). For each row, width 0 is one
+ * cluster; every cluster of width b - 1 is cut in two at the optimal 1-D 2-means
+ * point of its sorted members (never between equal values; the smallest cut on a
+ * tie; the lower half gets bit 0; a cluster with fewer than two distinct values
+ * keeps all members in its lower half, and an empty half takes its parent's
+ * value). Entry c of width b is its members' mean, rounded once to binary16, at
+ * heap index 2^b + c (entry 0 is 0, entry 1 the row mean); a weight's code is
+ * its cluster at width b_max. Unweighted (the pages' seed model and sensitivity
+ * weights need trained models). Cost O(K N (log N + b_max)).
+ *   W      host fp32 [K][N] row-major, finite.
+ *   codes  host uint8 [K][N] row-major, output (b_max-bit codes for grinqh_pack_codes).
+ *   lut    host binary16 [K][2^(b_max+1)], output (the tables of grinqh_vmm_lut).
+ * Errors: INVALID_ARG (sizes, b_max not in {2, 4, 6, 8}, NULL, non-finite W).
+ */
+grinqh_status grinqh_lut_build(const float* W, int32_t K, int32_t N, int32_t b_max, uint8_t* codes, uint16_t* lut);
 
 /* Bytes of the table buffer of grinqh_vmm_lut: K * 2^(b_max+2). */
 grinqh_status grinqh_lut_bytes(const grinqh_layout* layout, size_t* bytes);
