@@ -449,12 +449,29 @@ def _oracle_sample(budget_s, nthreads):
     return done, secs, names
 
 
+def _cpu_model():
+    """The host CPU's model name (first 'model name' line of /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline(args):
     nthreads = os.cpu_count() or 1
     done, secs, names = _oracle_sample(args.cpu_budget, nthreads)
+    # the same oracle on one thread, on a shorter bounded sample (the first pairs)
+    done1, secs1, names1 = _oracle_sample(min(5.0, args.cpu_budget / 4.0), 1)
     return {"value": round(secs * 1e6 / max(done, 1), 1), "unit": UNIT, "cores": nthreads, "kind": "oracle",
             "sample": "fp64 oracle select+vmm on %d of the %d (linear, width) pairs: %s" % (
-                done, 7 * len(TARGETS), ", ".join(names))}
+                done, 7 * len(TARGETS), ", ".join(names)),
+            "single_thread": {"value": round(secs1 * 1e6 / max(done1, 1), 1), "unit": UNIT, "cores": 1,
+                              "sample": ", ".join(names1)},
+            "cpu_model": _cpu_model()}
 
 
 def run_reference(args):
