@@ -901,6 +901,53 @@ def run_lut(args):
                                    "bytes_per_step": tot_alg}}))
 
 
+def run_cold(args):
+    """Isolated cold calls: for every (linear, width) pair of the decode step, one
+    grinqh_select and one grinqh_vmm (with its partial sums) right after a write of
+    twice the L2 size, each bracketed by CUDA events on the launching stream;
+    median over `--iters` repetitions per pair (one untimed first repetition)."""
+    import torch
+    from activation_graded_bit_b200 import grinqh as g
+    from activation_graded_bit_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    pairs = build_workload(g, wl, torch, dev, copies=1)
+    stream = torch.cuda.Stream(device=dev)
+    l2 = int(torch.cuda.get_device_properties(dev).L2_cache_size)
+    flush = torch.empty(max(2 * l2 // 4, 1 << 20), dtype=torch.float32, device=dev)
+    reps = max(args.iters, 5)
+    points = []
+    for pr in pairs:
+        t_sel, t_vmm = [], []
+        for r in range(reps + 1):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e2 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                flush.fill_(float(r))
+                e0.record(stream)
+                g.select(pr["x"], pr["th"], CLASSES, out=pr["sel"], stream=stream)
+                e1.record(stream)
+                g.vmm(pr["packed"], pr["x"], pr["sel"], pr["ws"], y=pr["y"], stream=stream)
+                e2.record(stream)
+            stream.synchronize()
+            if r > 0:
+                t_sel.append(e0.elapsed_time(e1) * 1e3)
+                t_vmm.append(e1.elapsed_time(e2) * 1e3)
+        points.append({"linear": pr["name"], "K": pr["K"], "N": pr["N"], "target_bits": pr["target"],
+                       "select_us": round(statistics.median(t_sel), 3), "vmm_us": round(statistics.median(t_vmm), 3)})
+    assert all(bool(torch.isfinite(pr["y"]).all()) for pr in pairs)
+    n = len(points)
+    print(json.dumps({"metric": "isolated cold select and VMM: µs per call after an L2 flush",
+                      "unit": "µs", "higher_is_better": False, "data": "synthetic",
+                      "config": {"workload": WORKLOAD, "classes": list(CLASSES), "b_max": BMAX,
+                                 "l2": "%d bytes written before every call pair (2x L2)" % (4 * flush.numel()),
+                                 "repetitions": reps},
+                      "select_us_mean": round(sum(p["select_us"] for p in points) / n, 3),
+                      "vmm_us_mean": round(sum(p["vmm_us"] for p in points) / n, 3),
+                      "points": points}))
+
+
 def run_prefill(args):
     """The prefill path on the Llama3-8B linears (Section 4 of the paper: unpack at
     full b_max precision, then a dense product): for T tokens, microseconds of
@@ -994,6 +1041,7 @@ def main():
     ap.add_argument("--batch", action="store_true", help="batch 1..16 through the batched fused call (one JSON line)")
     ap.add_argument("--prefill", action="store_true", help="prefill path: dequant + GEMM on the linears (one JSON line)")
     ap.add_argument("--lut", action="store_true", help="nested look-up-table codes through grinqh_vmm_lut (one JSON line)")
+    ap.add_argument("--cold", action="store_true", help="isolated cold select and VMM after an L2 flush (one JSON line)")
     ap.add_argument("--bmax", type=int, default=8, choices=(4, 6, 8),
                     help="stored code width; 4 or 6 grade into the classes {0, 2, ..., b_max}")
     ap.add_argument("--family", default="llama3", choices=("llama3", "qwen3"),
@@ -1026,6 +1074,9 @@ def main():
         return
     if args.lut and not args.profile:
         run_lut(args)
+        return
+    if args.cold:
+        run_cold(args)
         return
     if args.profile:
         run_profile_case(args)
