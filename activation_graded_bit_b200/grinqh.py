@@ -109,6 +109,22 @@ def _classes_buf(classes: Sequence[int]):
     return arr, len(classes)
 
 
+def _need(t, count: int, esize: int, what: str):
+    """The library reads or writes `count` elements of `esize` bytes at t's address;
+    the C ABI sees only the pointer, so a smaller buffer or another element size is
+    refused here, before anything is launched."""
+    if t is None:
+        return
+    if t.element_size() != esize or t.numel() < count:
+        raise ValueError("%s: needs %d elements of %d bytes, got %d of %d" % (
+            what, count, esize, t.numel(), t.element_size()))
+
+
+def _need_selection(sel, K: int, what: str):
+    _need(sel.idx, K, 4, what + " idx")
+    _need(sel.offsets, len(sel.classes) + 1, 4, what + " offsets")
+
+
 def layout(K: int, N: int, b_max: int = 8) -> Layout:
     L = Layout()
     if b_max == 8:
@@ -154,6 +170,7 @@ def pack(W: torch.Tensor, out: Optional[PackedLayer] = None, stream=None, b_max:
     assert W.dtype == torch.float32 and W.is_cuda and W.is_contiguous() and W.dim() == 2
     K, N = W.shape
     p = out if out is not None else empty_packed(K, N, W.device, b_max)
+    _need(W, p.K * p.N, 4, "grinqh_pack W")
     _check(_pack(ctypes.byref(p.layout), _ptr(W), _ptr(p.packed), _stream(stream)), "grinqh_pack")
     return p
 
@@ -186,6 +203,9 @@ def calibrate(X: torch.Tensor, classes: Sequence[int], P: Optional[Sequence[floa
     S, K = X.shape
     cb, n = _classes_buf(classes)
     th = out if out is not None else torch.empty(max(n - 1, 1), dtype=torch.float32, device=X.device)
+    _need(th, n - 1, 4, "grinqh_calibrate thresholds")
+    if P is not None and len(P) != n:
+        raise ValueError("grinqh_calibrate: P has %d entries for %d classes" % (len(P), n))
     ws_bytes = calibrate_workspace_bytes(S, n)
     ws = workspace if workspace is not None else torch.empty(ws_bytes, dtype=torch.uint8, device=X.device)
     Pbuf = None
@@ -218,6 +238,10 @@ def select(x: torch.Tensor, thresholds: torch.Tensor, classes: Sequence[int],
     K = x.shape[0]
     sel = out if out is not None else empty_selection(K, classes, x.device)
     cb, n = _classes_buf(classes)
+    _need(thresholds, n - 1, 4, "grinqh_select thresholds")
+    _need(sel.bits, K, 1, "grinqh_select bits")
+    _need(sel.idx, K, 4, "grinqh_select idx")
+    _need(sel.offsets, n + 1, 4, "grinqh_select offsets")
     _check(_select(_ptr(x), K, _ptr(thresholds), ctypes.addressof(cb), n, _ptr(sel.bits), _ptr(sel.idx),
                    _ptr(sel.offsets), _stream(stream)), "grinqh_select")
     return sel
@@ -239,6 +263,9 @@ def vmm(p: PackedLayer, x: torch.Tensor, sel: Selection, workspace: torch.Tensor
     """grinqh_vmm: y[N] fp32 = x . W_hat over the graded bit planes."""
     if y is None:
         y = torch.empty(p.N, dtype=torch.float32, device=p.packed.device)
+    _need(x, p.K, 2, "grinqh_vmm x")
+    _need(y, p.N, 4, "grinqh_vmm y")
+    _need_selection(sel, p.K, "grinqh_vmm")
     cb, n = _classes_buf(sel.classes)
     _check(_vmm(ctypes.byref(p.layout), _ptr(p.packed), _ptr(x), _ptr(sel.idx), _ptr(sel.offsets),
                 ctypes.addressof(cb), n, _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -252,6 +279,9 @@ def select_vmm(p: PackedLayer, x: torch.Tensor, thresholds: Optional[torch.Tenso
     if y is None:
         y = torch.empty(p.N, dtype=torch.float32, device=p.packed.device)
     cb, n = _classes_buf(classes)
+    _need(x, p.K, 2, "grinqh_select_vmm x")
+    _need(y, p.N, 4, "grinqh_select_vmm y")
+    _need(thresholds, n - 1, 4, "grinqh_select_vmm thresholds")
     _check(_select_vmm(ctypes.byref(p.layout), _ptr(p.packed), _ptr(x), _ptr(thresholds), ctypes.addressof(cb), n,
                        _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
            "grinqh_select_vmm")
@@ -274,6 +304,8 @@ def select_vmm_batch(p: PackedLayer, X: torch.Tensor, thresholds: Optional[torch
     if Y is None:
         Y = torch.empty((T, p.N), dtype=torch.float32, device=X.device)
     cb, n = _classes_buf(classes)
+    _need(Y, T * p.N, 4, "grinqh_select_vmm_batch Y")
+    _need(thresholds, n - 1, 4, "grinqh_select_vmm_batch thresholds")
     _check(_select_vmm_batch(ctypes.byref(p.layout), _ptr(p.packed), _ptr(X), T, _ptr(thresholds),
                              ctypes.addressof(cb), n, _ptr(Y), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)),
@@ -284,6 +316,7 @@ def select_vmm_batch(p: PackedLayer, X: torch.Tensor, thresholds: Optional[torch
 def dequant(p: PackedLayer, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """grinqh_dequant: full-width w_hat as binary16 [K, N] (returned as float16)."""
     W16 = out if out is not None else torch.empty((p.K, p.N), dtype=torch.float16, device=p.packed.device)
+    _need(W16, p.K * p.N, 2, "grinqh_dequant W16")
     _check(_dequant(ctypes.byref(p.layout), _ptr(p.packed), _ptr(W16), _stream(stream)), "grinqh_dequant")
     return W16
 
@@ -297,6 +330,8 @@ def prefill(p: PackedLayer, X: torch.Tensor, Y: Optional[torch.Tensor] = None, W
         Y = torch.empty((T, p.N), dtype=torch.float32, device=X.device)
     if W16 is None:
         W16 = torch.empty((p.K, p.N), dtype=torch.float16, device=X.device)
+    _need(Y, T * p.N, 4, "grinqh_prefill Y")
+    _need(W16, p.K * p.N, 2, "grinqh_prefill W16")
     _check(_prefill(ctypes.byref(p.layout), _ptr(p.packed), _ptr(X), T, _ptr(Y), _ptr(W16), _stream(stream)),
            "grinqh_prefill")
     return Y
@@ -305,6 +340,9 @@ def prefill(p: PackedLayer, X: torch.Tensor, Y: Optional[torch.Tensor] = None, W
 def vmm_noalloc(p: PackedLayer, x: torch.Tensor, sel: Selection, y: torch.Tensor, stream=None) -> torch.Tensor:
     """grinqh_vmm_noalloc: as vmm, with the library's shared static scratch instead of a
     workspace; y (fp32 [N] CUDA tensor) must be given, since this call allocates nothing."""
+    _need(x, p.K, 2, "grinqh_vmm_noalloc x")
+    _need(y, p.N, 4, "grinqh_vmm_noalloc y")
+    _need_selection(sel, p.K, "grinqh_vmm_noalloc")
     cb, n = _classes_buf(sel.classes)
     _check(_vmm_noalloc(ctypes.byref(p.layout), _ptr(p.packed), _ptr(x), _ptr(sel.idx), _ptr(sel.offsets),
                         ctypes.addressof(cb), n, _ptr(y), _stream(stream)), "grinqh_vmm_noalloc")
@@ -316,6 +354,7 @@ def pack_codes(codes: torch.Tensor, b_max: int = 8, out: Optional[PackedLayer] =
     assert codes.dtype == torch.uint8 and codes.is_cuda and codes.is_contiguous() and codes.dim() == 2
     K, N = codes.shape
     p = out if out is not None else empty_packed(K, N, codes.device, b_max)
+    _need(codes, p.K * p.N, 1, "grinqh_pack_codes codes")
     _check(_pack_codes(ctypes.byref(p.layout), _ptr(codes), _ptr(p.packed), _stream(stream)), "grinqh_pack_codes")
     return p
 
@@ -335,6 +374,9 @@ def vmm_lut(p: PackedLayer, lut: torch.Tensor, x: torch.Tensor, sel: Selection, 
     assert lut.numel() * 2 == lut_bytes(p.layout), "table buffer size"
     if y is None:
         y = torch.empty(p.N, dtype=torch.float32, device=p.packed.device)
+    _need(x, p.K, 2, "grinqh_vmm_lut x")
+    _need(y, p.N, 4, "grinqh_vmm_lut y")
+    _need_selection(sel, p.K, "grinqh_vmm_lut")
     cb, n = _classes_buf(sel.classes)
     _check(_vmm_lut(ctypes.byref(p.layout), _ptr(p.packed), _ptr(lut), _ptr(x), _ptr(sel.idx), _ptr(sel.offsets),
                     ctypes.addressof(cb), n, _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(),

@@ -98,3 +98,43 @@ def test_every_call_marshals_and_reports(g):
     Xc = FakeTensor((8, K), torch.int16)
     _expect_invalid(lambda: g.calibrate(Xc, (0, 4, 4), target_bits=2.0, out=th, workspace=ws, stream=st))
     _expect_invalid(lambda: g.vmm_batch_workspace(g.layout(K, N), 0))
+
+
+def test_short_or_mistyped_buffers_are_refused_before_the_call(g):
+    # a valid layout: only the binding's size checks stand between these stand-in
+    # buffers and the library, and each of them fails one
+    K, N, T = 64, 1024, 3
+    cl = (0, 2, 3, 4, 8)
+    L = g.layout(K, N)
+    p = g.PackedLayer(L, FakeTensor((int(L.packed_bytes),), torch.uint8))
+    x = FakeTensor((K,), torch.int16)
+    y = FakeTensor((N,), torch.float32)
+    ws = FakeTensor((1 << 20,), torch.uint8)
+    sel = g.Selection(FakeTensor((K,), torch.uint8), FakeTensor((K,), torch.int32),
+                      FakeTensor((len(cl) + 1,), torch.int32), cl)
+    short_sel = g.Selection(sel.bits, FakeTensor((K - 1,), torch.int32), sel.offsets, cl)
+    th = FakeTensor((4,), torch.float32)
+    cases = [
+        lambda: g.vmm(p, FakeTensor((K - 1,), torch.int16), sel, ws, y=y),
+        lambda: g.vmm(p, FakeTensor((K,), torch.float32), sel, ws, y=y),
+        lambda: g.vmm(p, x, sel, ws, y=FakeTensor((N - 1,), torch.float32)),
+        lambda: g.vmm(p, x, short_sel, ws, y=y),
+        lambda: g.vmm_noalloc(p, x, sel, FakeTensor((N,), torch.float16)),
+        lambda: g.select_vmm(p, x, FakeTensor((3,), torch.float32), cl, ws, y=y),
+        lambda: g.select_vmm_batch(p, FakeTensor((T, K), torch.int16), th, cl, ws,
+                                   Y=FakeTensor((T, N - 1), torch.float32)),
+        lambda: g.dequant(p, out=FakeTensor((K, N - 1), torch.float16)),
+        lambda: g.prefill(p, FakeTensor((T, K), torch.int16), Y=FakeTensor((T, N), torch.float32),
+                          W16=FakeTensor((K - 1, N), torch.float16)),
+        lambda: g.select(x, FakeTensor((2,), torch.float32), cl, out=sel),
+        lambda: g.select(x, th, cl, out=short_sel),
+        lambda: g.pack(FakeTensor((K, N - 1), torch.float32), out=p),
+        lambda: g.pack_codes(FakeTensor((K, N - 1), torch.uint8), out=p),
+        lambda: g.vmm_lut(p, FakeTensor((K, 512), torch.int16), x, short_sel, ws, y=y),
+        lambda: g.calibrate(FakeTensor((8, K), torch.int16), cl, target_bits=3.0, out=FakeTensor((3,), torch.float32),
+                            workspace=ws),
+        lambda: g.calibrate(FakeTensor((8, K), torch.int16), cl, P=(0.5, 0.5), out=th, workspace=ws),
+    ]
+    for i, fn in enumerate(cases):
+        with pytest.raises(ValueError):
+            fn()
