@@ -3,6 +3,7 @@ turns a rejected call into GrinqhError. Runs without a GPU: stand-in tensors
 carry plausible device addresses, and each call is given a layout or argument
 that the library rejects on the host before anything could be launched."""
 import ctypes
+import os
 
 import pytest
 import torch
@@ -138,3 +139,20 @@ def test_short_or_mistyped_buffers_are_refused_before_the_call(g):
     for i, fn in enumerate(cases):
         with pytest.raises(ValueError):
             fn()
+
+
+def test_binding_refuses_to_load_without_the_library(tmp_path):
+    # a copy of the package without libgrinqh.so: importing the binding fails
+    # loudly (no CPU or library fallback exists)
+    import shutil
+    import subprocess
+    import sys
+    src = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "activation_graded_bit_b200")
+    dst = tmp_path / "activation_graded_bit_b200"
+    dst.mkdir()
+    for f in ("__init__.py", "grinqh.py", "workloads.py", "build.py"):
+        shutil.copy(os.path.join(src, f), dst / f)
+    r = subprocess.run([sys.executable, "-c", "import activation_graded_bit_b200.grinqh"], cwd=str(tmp_path),
+                       capture_output=True, text=True, env={**os.environ, "PYTHONPATH": str(tmp_path)})
+    assert r.returncode != 0
+    assert "libgrinqh.so is not built" in r.stderr
