@@ -106,7 +106,7 @@ grinqh_status grinqh_layout_init_bmax(int32_t K, int32_t N, int32_t b_max, grinq
   L.record_bytes = record_bytes_for(b_max);
   L.b_max = b_max;
   L.reserved = 0;
-  L.packed_bytes = (int64_t)K * L.n_tiles * L.record_bytes;
+  L.packed_bytes = (int64_t)K * L.n_tiles * (L.record_bytes + kMetaBytes);
   *out = L;
   return GRINQH_OK;
 }
@@ -271,6 +271,7 @@ grinqh_status grinqh_vmm(const grinqh_layout* layout, const void* packed, const 
   a.n_tiles = L.n_tiles;
   a.b_max = L.b_max;
   a.packed = (const uint8_t*)packed;
+  a.meta_offset = meta_offset_for(L.K, L.n_tiles, L.b_max);
   a.x = x;
   a.idx = idx;
   a.offsets = offsets;
@@ -299,6 +300,7 @@ grinqh_status grinqh_vmm_noalloc(const grinqh_layout* layout, const void* packed
   a.n_tiles = L.n_tiles;
   a.b_max = L.b_max;
   a.packed = (const uint8_t*)packed;
+  a.meta_offset = meta_offset_for(L.K, L.n_tiles, L.b_max);
   a.x = x;
   a.idx = idx;
   a.offsets = offsets;
@@ -328,6 +330,7 @@ grinqh_status grinqh_select_vmm(const grinqh_layout* layout, const void* packed,
   a.n_tiles = L.n_tiles;
   a.b_max = L.b_max;
   a.packed = (const uint8_t*)packed;
+  a.meta_offset = meta_offset_for(L.K, L.n_tiles, L.b_max);
   a.x = x;
   a.thresholds = thresholds;
   a.y = y;
@@ -364,12 +367,13 @@ grinqh_status grinqh_select_vmm_batch(const grinqh_layout* layout, const void* p
   a.n_tiles = L.n_tiles;
   a.b_max = L.b_max;
   a.packed = (const uint8_t*)packed;
+  a.meta_offset = meta_offset_for(L.K, L.n_tiles, L.b_max);
   a.x = X;
   a.thresholds = thresholds;
   a.y = Y;
+  a.ct = table(classes, n_classes);
   a.status = (uint32_t*)workspace;
   a.partial = (float*)((char*)workspace + 16);
-  a.ct = table(classes, n_classes);
   a.tokens = tokens;
   return cuda_status(launch_vmm(a, (cudaStream_t)stream, true));
 }
@@ -406,6 +410,7 @@ grinqh_status grinqh_vmm_lut(const grinqh_layout* layout, const void* packed, co
   a.n_tiles = L.n_tiles;
   a.b_max = L.b_max;
   a.packed = (const uint8_t*)packed;
+  a.meta_offset = meta_offset_for(L.K, L.n_tiles, L.b_max);
   a.lut = (const uint8_t*)lut;
   a.x = x;
   a.idx = idx;

@@ -1,9 +1,12 @@
 // Device-side helpers shared by the GRINQH kernels (sm_100a).
 //
-// Plane-pair word format (see include/grinqh.h): planes 2s and 2s+1 (plane 0
-// is the most significant bit of the 8-bit code) of a tile row share 256 bytes,
-// "pair s". Lane w of a warp owns words 2w (local columns 32w..32w+15) and
-// 2w+1 (columns 32w+16..32w+31) of every pair. In either word, local column
+// Packed layout (see include/grinqh.h): the planes of every (row k, column
+// tile t) record come first, record k * n_tiles + t at byte
+// (k * n_tiles + t) * 128 * b_max (a multiple of 256), and the 32 bytes of
+// scale/zero words of every record follow in a separate array. Inside a
+// record, planes 2s and 2s+1 (plane 0 is the most significant bit of the code)
+// share 256 bytes, "pair s". Lane w of a warp owns words 2w (local columns
+// 32w..32w+15) and 2w+1 (columns 32w+16..32w+31) of every pair. In either word, local column
 // 4j' + i of the half (j' in 0..3, i in 0..3) of plane 2s + l sits at bit
 // (8i + 2j' + 7 - 2s - l) mod 32. The placement is chosen so that the bits a
 // register of four codes needs from a pair sit under one rotated mask
@@ -16,6 +19,7 @@
 // rebuilds them), with its 2-bit segments; odd widths take the top plane of
 // their last pair under a one-plane mask.
 #pragma once
+#include <cstddef>
 #include <cstdint>
 #include <cuda_fp16.h>
 
@@ -24,14 +28,18 @@ namespace grinqh {
 constexpr int kPlanes = 8;
 constexpr int kGroup = 128;
 constexpr int kTileN = 1024;                          // columns per tile
-constexpr int kMetaBytes = 4 * (kTileN / kGroup);     // scale/zero words at the head of a record
+constexpr int kMetaBytes = 4 * (kTileN / kGroup);     // scale/zero words of one (row, tile) record
 constexpr int kPlaneBytes = kTileN / 8;               // one plane of one tile row
 constexpr int kPairBytes = 2 * kPlaneBytes;           // two planes of one tile row
-constexpr int kRecordBytes = kMetaBytes + kPlanes * kPlaneBytes;   // 1056 = 33 sectors of 32 B
 
-// Bytes of a (row, tile) record that stores b_max planes: the scale/zero words,
-// then b_max / 2 plane pairs (a whole number of 32-byte sectors).
-__host__ __device__ constexpr int record_bytes_for(int b_max) { return kMetaBytes + b_max * kPlaneBytes; }
+// Plane bytes of a (row, tile) record that stores b_max planes: b_max / 2 plane
+// pairs of 256 bytes.
+__host__ __device__ constexpr int record_bytes_for(int b_max) { return b_max * kPlaneBytes; }
+
+// Byte offset of the scale/zero words in a packed layer: after every record's planes.
+__host__ __device__ constexpr size_t meta_offset_for(int K, int n_tiles, int b_max) {
+  return (size_t)K * (size_t)n_tiles * (size_t)record_bytes_for(b_max);
+}
 
 // The column (0..15 inside the half) and plane offset l stored at bit L of a
 // pair-s word (the inverse of the placement above: column 4j'+i of plane 2s+l

@@ -7,6 +7,8 @@
 
 namespace grinqh {
 
+// Every packed-layer kernel takes the layer's planes at packed and its
+// scale/zero words at packed + meta_offset (K * n_tiles * record_bytes_for(b_max)).
 cudaError_t launch_pack(const float* W, int K, int N, int n_tiles, int n_groups, int b_max, void* packed,
                         cudaStream_t st);
 
@@ -14,7 +16,7 @@ cudaError_t launch_unpack(const void* packed, const uint8_t* bits, int K, int N,
                           uint8_t* codes, cudaStream_t st);
 
 // Planes of given b_max-bit codes [K][N] (bits above b_max ignored); the
-// records' scale/zero words are written as zero.
+// scale/zero words are written as zero.
 cudaError_t launch_pack_codes(const uint8_t* codes, int K, int N, int n_tiles, int b_max, void* packed,
                               cudaStream_t st);
 
@@ -38,7 +40,8 @@ cudaError_t launch_select(const uint16_t* x, int K, const float* thresholds, con
 struct VmmArgs {
   int K, N, n_tiles;
   int b_max;                 // bits per stored code (2, 4, 6 or 8); records of record_bytes_for(b_max)
-  const uint8_t* packed;
+  const uint8_t* packed;     // planes of every record, then the scale/zero words
+  size_t meta_offset;        // byte offset of the scale/zero words in packed
   const uint16_t* x;
   const int32_t* idx;
   const int32_t* offsets;

@@ -37,7 +37,9 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ W, 
   const float* row = W + (size_t)k * N;
   const int rbytes = record_bytes_for(b_max);
   const double levels = (double)((1 << b_max) - 1);
-  uint8_t* rec = packed + ((size_t)k * n_tiles + t) * rbytes;
+  const size_t ri = (size_t)k * n_tiles + t;
+  uint8_t* rec = packed + ri * rbytes;                                                    // its planes
+  uint32_t* meta = reinterpret_cast<uint32_t*>(packed + meta_offset_for(K, n_tiles, b_max) + ri * kMetaBytes);
 
   float v[4];
   float mn = INFINITY, mx = -INFINITY;
@@ -76,8 +78,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ W, 
     }
     codes[warp * kGroup + lane + 32 * e] = q;
   }
-  if (lane == 0)
-    reinterpret_cast<uint32_t*>(rec)[warp] = live ? ((uint32_t)sb | ((uint32_t)zb << 16)) : 0u;
+  if (lane == 0) meta[warp] = live ? ((uint32_t)sb | ((uint32_t)zb << 16)) : 0u;
   __syncthreads();
 
   // thread -> (pair s, word wi): b_max/2 plane pairs x 64 words for a
@@ -94,7 +95,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ W, 
     const int p = 2 * sp + l;
     word |= (uint32_t)((codes[cbase + c16] >> (b_max - 1 - p)) & 1u) << L;
   }
-  reinterpret_cast<uint32_t*>(rec + kMetaBytes + sp * kPairBytes)[wi] = word;
+  reinterpret_cast<uint32_t*>(rec + sp * kPairBytes)[wi] = word;
 }
 
 // Decoder: one warp per (row, tile) record, 8 records per CTA. The planes are
@@ -106,7 +107,7 @@ __device__ __forceinline__ void decode_word(const uint8_t* rec, int w, int b_max
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
     const bool used = 2 * s < B;   // pair s holds planes 2s, 2s+1
-    const uint32_t* pw = reinterpret_cast<const uint32_t*>(rec + kMetaBytes + s * kPairBytes);
+    const uint32_t* pw = reinterpret_cast<const uint32_t*>(rec + s * kPairBytes);
     P[2 * s] = used ? pw[2 * w] : 0u;
     P[2 * s + 1] = used ? pw[2 * w + 1] : 0u;
   }
@@ -158,11 +159,11 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
 // scale and a 9-bit code difference is exact). A lane's 32 columns are 64
 // contiguous bytes, written as four 16-byte stores when the row allows it.
 template <int B>
-__device__ __forceinline__ void dequant_record(const uint8_t* rec, int w, int k, int N, int n0,
+__device__ __forceinline__ void dequant_record(const uint8_t* rec, const uint8_t* meta, int w, int k, int N, int n0,
                                                __half* __restrict__ out) {
   uint32_t R[8];
   decode_word<B>(rec, w, B, R);
-  const uint32_t m = reinterpret_cast<const uint32_t*>(rec)[w >> 2];   // this lane's group's scale | zero
+  const uint32_t m = reinterpret_cast<const uint32_t*>(meta)[w >> 2];   // this lane's group's scale | zero
   const float s = __half2float(__ushort_as_half((unsigned short)(m & 0xFFFFu)));
   const float z = __half2float(__ushort_as_half((unsigned short)(m >> 16)));
   __half2 h[16];
@@ -193,14 +194,16 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
   const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int w = threadIdx.x & 31;
   if (k >= K) return;
-  const uint8_t* rec = packed + ((size_t)k * n_tiles + t) * record_bytes_for(b_max);
+  const size_t ri = (size_t)k * n_tiles + t;
+  const uint8_t* rec = packed + ri * record_bytes_for(b_max);
+  const uint8_t* meta = packed + meta_offset_for(K, n_tiles, b_max) + ri * kMetaBytes;
   const int n0 = t * kTileN + 32 * w;
   if (n0 >= N) return;
   switch (b_max) {
-    case 2: dequant_record<2>(rec, w, k, N, n0, out); break;
-    case 4: dequant_record<4>(rec, w, k, N, n0, out); break;
-    case 6: dequant_record<6>(rec, w, k, N, n0, out); break;
-    default: dequant_record<8>(rec, w, k, N, n0, out); break;
+    case 2: dequant_record<2>(rec, meta, w, k, N, n0, out); break;
+    case 4: dequant_record<4>(rec, meta, w, k, N, n0, out); break;
+    case 6: dequant_record<6>(rec, meta, w, k, N, n0, out); break;
+    default: dequant_record<8>(rec, meta, w, k, N, n0, out); break;
   }
 }
 
@@ -234,13 +237,15 @@ __global__ void __launch_bounds__(256) pack_codes_kernel(const uint8_t* __restri
                                                          int n_tiles, int b_max, uint8_t* __restrict__ packed) {
   __shared__ uint8_t tile[kTileN];
   const int k = blockIdx.x, t = blockIdx.y;
-  uint8_t* rec = packed + ((size_t)k * n_tiles + t) * record_bytes_for(b_max);
+  const size_t ri = (size_t)k * n_tiles + t;
+  uint8_t* rec = packed + ri * record_bytes_for(b_max);
+  uint32_t* meta = reinterpret_cast<uint32_t*>(packed + meta_offset_for(K, n_tiles, b_max) + ri * kMetaBytes);
   const uint32_t keep = (1u << b_max) - 1u;
   for (int e = threadIdx.x; e < kTileN; e += 256) {
     const int n = t * kTileN + e;
     tile[e] = (n < N) ? (uint8_t)(codes[(size_t)k * N + n] & keep) : (uint8_t)0;
   }
-  if (threadIdx.x < kMetaBytes / 4) reinterpret_cast<uint32_t*>(rec)[threadIdx.x] = 0u;
+  if (threadIdx.x < kMetaBytes / 4) meta[threadIdx.x] = 0u;
   __syncthreads();
   const int sp = threadIdx.x >> 6, wi = threadIdx.x & 63;
   if (2 * sp >= b_max) return;
@@ -252,7 +257,7 @@ __global__ void __launch_bounds__(256) pack_codes_kernel(const uint8_t* __restri
     pair_col_at(sp, L, c16, l);
     word |= (uint32_t)((tile[cbase + c16] >> (b_max - 1 - (2 * sp + l))) & 1u) << L;
   }
-  reinterpret_cast<uint32_t*>(rec + kMetaBytes + sp * kPairBytes)[wi] = word;
+  reinterpret_cast<uint32_t*>(rec + sp * kPairBytes)[wi] = word;
 }
 
 cudaError_t launch_pack_codes(const uint8_t* codes, int K, int N, int n_tiles, int b_max, void* packed,

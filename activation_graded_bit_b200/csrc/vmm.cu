@@ -18,36 +18,41 @@
 // Data movement. Each of the 16 warps takes rows h, h+16, ... of its CTA. Lane
 // w of a warp owns columns 32w..32w+31 of the tile, so for a row of width b it
 // needs its two words of each of plane pairs 0..ceil(b/2)-1 (one 8-byte load
-// per pair: 256 contiguous bytes per pair across the warp, one coalesced
-// request) and the scale/zero word of its 128-column group. The lanes load
+// per pair: 256 contiguous, 256-byte-aligned bytes per pair across the warp,
+// one coalesced request) and the scale/zero word of its 128-column group (the
+// scale/zero words of all records sit in their own array, so the plane records
+// are whole 256-byte units and no DRAM sector is shared between records). The lanes load
 // those words straight into registers with plain read-only loads, kDepth rows
 // ahead of the one they are rebuilding: a software pipeline in registers, with
 // no shared-memory staging and no barriers. On this part that reads scattered
 // 300..1100-byte rows faster than bulk (TMA) copies, whose completion rate per
 // issuing warp, not their size, limits the bandwidth for rows this short. The
-// record prefixes of the kL2Ahead rows beyond the pipeline are requested into
-// L2 (one 128-byte line per lane, no register), so the register loads hit L2
+// planes and scale/zero words of the kL2Ahead rows beyond the pipeline are
+// requested into L2 (one 128-byte line per lane, no register), so the register
+// loads hit L2
 // instead of DRAM. With those requests a pipeline of three rows is enough, and
 // the registers it frees go to the compiler's scheduling (measured: 3 rows in
 // flight 13% faster than 6 on the 14336 x 4096 layer). Blocks of kDepth rows
 // whose loads and requests all exist run without per-row tests; the loads of
 // narrower rows are switched off by predicates, not branches.
 //
-// Arithmetic per row and thread. a = x_k * s is exact in fp32 (two 11-bit
-// significands). The plane pairs are merged into 8 registers of 4 truncated
-// codes each (one LOP3 per pair plus one rotate, thanks to the bit order chosen
-// at pack time); the merge enters one fall-through sequence at the last pair, so
-// all widths share one copy of the code. Codes become floats without a
-// per-code integer extraction: a byte-permute puts two codes c1:c0 in the low
-// 16 bits of an otherwise zero word, i.e. the subnormal float (256 c1 + c0)
-// 2^-149; adding 2^-118 with round-down leaves exactly 2^-118 + c1 2^-141, so
-// one more subtraction gives hi = c1 2^-141 and another gives lo = c0 2^-149,
-// all exact and all on the FP32 pipe (B200 runs FFMA with subnormal operands at
-// full rate, while byte extraction would run on the half-rate integer pipe).
-// The products use coefficients a 2^95 and a 2^87, so the accumulators hold a *
-// code * 2^-54 (no overflow for |a| <= 2^32, no precision loss for the sizes
-// that matter). The per-row constant a * (mid_b - z) goes to one scalar per
-// thread, since all 32 columns of a thread share one 128-column group.
+// Arithmetic per row and thread. The row's coefficient a = x_k * s is one
+// mixed-precision FMA of the two binary16 values (exact in fp32), and
+// z - mid one mixed-precision add. The plane pairs are merged into 8 registers
+// of 4 truncated codes each (one LOP3 per pair plus one rotate, thanks to the
+// bit order chosen at pack time); the merge enters one fall-through sequence at
+// the last pair, so all widths share one copy of the code. Codes become floats
+// without a per-code integer extraction: a byte-permute puts two codes c1:c0 in
+// the low 16 bits of an otherwise zero word, i.e. the subnormal float
+// (256 c1 + c0) 2^-149; a multiply by 2^-8 rounded toward zero leaves exactly
+// hi = c1 2^-149 (the subnormal grid is 2^-149) and one FMA gives
+// lo = c0 2^-149 = X - 256 hi, both exact and on the FP32 pipe (B200 runs
+// FFMA with subnormal operands at full rate, while byte extraction would run on
+// the half-rate integer pipe). Both halves take the same coefficient a 2^95,
+// so the accumulators hold a * code * 2^-54 (no overflow for |a| <= 2^32, no
+// precision loss for the sizes that matter). The per-row constant
+// a * (mid_b - z) goes to one scalar per thread, since all 32 columns of a
+// thread share one 128-column group.
 //
 // Reduction. Each warp stores its 1024 column sums into shared memory as soon
 // as its own rows are done (the buffer is not shared with the row list); after
@@ -102,30 +107,35 @@ struct RowRegs {
   uint32_t b;
 };
 
-// Per-thread constants of the row addressing: a row's record starts at
-// packed + 32 * (k * n_tiles * S + t * S) (records are S = 1 + 4 b_max sectors
-// of 32 B: 33 for b_max = 8),
-// so one integer multiply-add gives its offset in sectors (below 2^32: a valid
-// layout has K * N <= 2^34, so K * n_tiles <= 2^25) and one wide multiply-add
-// each of this lane's addresses in it.
+// Per-thread constants of the row addressing. A row's record index
+// rec = k * n_tiles + t is below 2^26 (a valid layout has K * N <= 2^34), so one
+// wide multiply-add gives each address: the planes of record rec start at
+// packed + rec * 128 b_max, its scale/zero words at packed + meta_offset + 32 rec.
 struct RowAddr {
-  const uint8_t* meta;    // packed + this lane's scale/zero word within a record
-  const uint8_t* pairs;   // packed + this lane's two words of pair 0 within a record
-  const uint8_t* lines;   // packed + 128 * lane (the lane's L2 line within a record prefix)
-  uint32_t nt33, t33;     // sectors per row of records, sector offset of tile t
-  uint32_t lane128;       // 128 * lane
+  const uint8_t* meta;    // this lane's scale/zero word within record 0's
+  const uint8_t* pairs;   // this lane's two words of pair 0 within record 0
+  const uint8_t* line;    // the L2 line this lane requests for record 0: plane line `lane` (lanes < b_max)
+                          // or the scale/zero words (lane b_max)
+  uint32_t line_mul;      // bytes per record in the array `line` points into
+  uint32_t lane;
+  uint32_t nt, t;         // column tiles, this CTA's tile
 };
 
 __device__ __forceinline__ RowAddr row_addr(const VmmArgs& a, int t, int w) {
-  const uint32_t kSectors = (uint32_t)record_bytes_for(a.b_max) / 32u;   // 9, 17, 25 or 33
-  static_assert(kMetaBytes % 32 == 0 && kPlaneBytes % 16 == 0, "records are whole 32-byte sectors");
+  const uint8_t* meta0 = a.packed + a.meta_offset;
   RowAddr ra;
-  ra.meta = a.packed + 4 * (w >> 2);
-  ra.pairs = a.packed + kMetaBytes + 8 * w;
-  ra.lines = a.packed + 128 * w;
-  ra.nt33 = (uint32_t)a.n_tiles * kSectors;
-  ra.t33 = (uint32_t)t * kSectors;
-  ra.lane128 = 128u * (uint32_t)w;
+  ra.meta = meta0 + 4 * (w >> 2);
+  ra.pairs = a.packed + 8 * w;
+  ra.lane = (uint32_t)w;
+  if (w < a.b_max) {
+    ra.line = a.packed + 128 * w;
+    ra.line_mul = (uint32_t)record_bytes_for(a.b_max);
+  } else {
+    ra.line = meta0;
+    ra.line_mul = (uint32_t)kMetaBytes;
+  }
+  ra.nt = (uint32_t)a.n_tiles;
+  ra.t = (uint32_t)t;
   return ra;
 }
 
@@ -152,20 +162,23 @@ __device__ __forceinline__ void ld_stream2_at_if(bool on, const void* ptr, uint3
       : "l"(ptr), "r"((uint32_t)on), "n"(kOff));
 }
 
-// Per-row coefficients for codes of kBmax bits, rebuilt in the 8-bit frame
+// Per-row coefficient for codes of kBmax bits, rebuilt in the 8-bit frame
 // (plane p at bit 7-p, so a code c of kBmax bits reads as c 2^(8-kBmax)):
-// A0 = a 2^(87+kBmax) (for c_lo 2^-149), A1 = a 2^(79+kBmax) (for c_hi 2^-141),
-// so the products carry a * c 2^-54 in kBmax-bit units, and the row's constant
-// a * (mid - z) is added to cacc (mid = 2^(kBmax-b-1) for b < kBmax, 0 at
-// b = kBmax, in the same units as z).
+// A = a 2^(87+kBmax) for codes held as c 2^-149, so the products carry
+// a * c 2^-54 in kBmax-bit units; the row's constant a * (mid - z) is added to
+// cacc (mid = 2^(kBmax-b-1) for b < kBmax, 0 at b = kBmax, in the units of z).
+// a = x * s is one mixed-precision FMA of the binary16 values (exact in fp32)
+// and z - mid one mixed-precision add (exact).
 template <int kBmax>
-__device__ __forceinline__ void row_coef(uint32_t m, float mid, float xk, float& A0, float& A1, float& cacc) {
-  const float s = half_bits_to_float(m);
-  const float z = half_bits_to_float(m >> 16);
-  const float av = xk * s;                                      // exact
-  cacc = fmaf(av, mid - z, cacc);
-  A0 = av * (float)(1ull << (23 + kBmax)) * 0x1p64f;
-  A1 = av * (float)(1ull << (15 + kBmax)) * 0x1p64f;
+__device__ __forceinline__ void row_coef(uint32_t m, uint32_t xh, float mid, float& A, float& cacc) {
+  float a, zt;
+  asm("{\n\t.reg .b16 s, z;\n\tmov.b32 {s, z}, %2;\n\t"
+      "fma.rn.f32.f16 %0, %3, s, 0f00000000;\n\t"
+      "add.rn.f32.f16 %1, z, %4;\n\t}"
+      : "=f"(a), "=f"(zt)
+      : "r"(m), "h"((unsigned short)xh), "f"(-mid));
+  cacc = fmaf(-a, zt, cacc);
+  A = a * ((float)(1ull << (23 + kBmax)) * 0x1p64f);
 }
 
 // The bin midpoint of width b for codes of kBmax bits, 0 at full width.
@@ -174,22 +187,21 @@ __device__ __forceinline__ constexpr float midpoint(int b) {
   return b >= kBmax ? 0.0f : (float)(1u << (kBmax - b - 1));
 }
 
-// acc += codes * coefficients for the 32 columns held in R (one row).
-__device__ __forceinline__ void fma_codes(const uint32_t (&R)[8], float A0s, float A1s, float2 (&acc)[16]) {
-  const float2 A0 = make_float2(A0s, A0s), A1 = make_float2(A1s, A1s);
-  const float2 M = make_float2(0x1p-118f, 0x1p-118f);
-  const float2 NM = make_float2(-0x1p-118f, -0x1p-118f);
-  const float2 NEG1 = make_float2(-1.0f, -1.0f);
+// acc += codes * A for the 32 columns held in R (one row): acc[2j] holds
+// columns 4j, 4j+2 and acc[2j+1] columns 4j+1, 4j+3.
+__device__ __forceinline__ void fma_codes(const uint32_t (&R)[8], float As, float2 (&acc)[16]) {
+  const float2 A = make_float2(As, As);
+  const float2 S8 = make_float2(0x1p-8f, 0x1p-8f);
+  const float2 M256 = make_float2(-256.0f, -256.0f);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     // X.x = codes of columns 4j+1 : 4j, X.y = columns 4j+3 : 4j+2, as subnormals
     const float2 X = make_float2(__uint_as_float(__byte_perm(R[j], 0u, 0x4410u)),
                                  __uint_as_float(__byte_perm(R[j], 0u, 0x4432u)));
-    const float2 u = __fadd2_rd(X, M);           // 2^-118 + c_hi 2^-141
-    const float2 hi = __fadd2_rn(u, NM);         // c_hi 2^-141
-    const float2 lo = __ffma2_rn(hi, NEG1, X);   // c_lo 2^-149
-    acc[2 * j] = __ffma2_rn(A0, lo, acc[2 * j]);           // columns 4j, 4j+2
-    acc[2 * j + 1] = __ffma2_rn(A1, hi, acc[2 * j + 1]);   // columns 4j+1, 4j+3
+    const float2 hi = __fmul2_rz(X, S8);         // c_hi 2^-149 (the c_lo part is cut off)
+    const float2 lo = __ffma2_rn(hi, M256, X);   // c_lo 2^-149
+    acc[2 * j] = __ffma2_rn(A, lo, acc[2 * j]);
+    acc[2 * j + 1] = __ffma2_rn(A, hi, acc[2 * j + 1]);
   }
 }
 
@@ -199,14 +211,15 @@ __device__ __forceinline__ void fma_codes(const uint32_t (&R)[8], float A0s, flo
 // coalesced 256-byte request across the warp). Pairs 1..3 are loaded under a
 // predicate: a narrow row reads no pair it does not use, and no branch is taken.
 // Every row that reaches the loop has b >= 1 (the width-0 class is never staged).
+template <int kBmax>
 __device__ __forceinline__ void load_row(const uint16_t* __restrict__ x, const RowAddr& ra, uint32_t info,
                                          RowRegs& r) {
   const uint32_t k = info & 0xFFFFFFu, b = info >> 24;
-  const uint32_t sec = k * ra.nt33 + ra.t33;                  // record offset in 32-byte sectors
+  const uint32_t rec = k * ra.nt + ra.t;
   r.b = b;
-  r.m = ld_stream(ra.meta + 32ull * sec);
+  r.m = ld_stream(ra.meta + (size_t)rec * kMetaBytes);
   r.xh = __ldg(x + k);
-  const uint8_t* pw = ra.pairs + 32ull * sec;                  // this lane's two words of pair 0
+  const uint8_t* pw = ra.pairs + (size_t)rec * (uint32_t)record_bytes_for(kBmax);   // this lane's two words of pair 0
   ld_stream2_at<0>(pw, r.p[0], r.p[1]);
   ld_stream2_at_if<1 * kPairBytes>(b > 2, pw, r.p[2], r.p[3]);
   ld_stream2_at_if<2 * kPairBytes>(b > 4, pw, r.p[4], r.p[5]);
@@ -249,14 +262,14 @@ __device__ __forceinline__ void assemble_row(const RowRegs& r, uint32_t (&out)[8
   finish_codes(T, out);
 }
 
-// Ask L2 for the record prefix of one row (k | b << 24): 32 + 256 ceil(b/2)
-// bytes from the record start, one 128-byte line per lane, issued under a
-// predicate (no branch) for the lines the prefix touches.
-__device__ __forceinline__ void prefetch_row_l2(const RowAddr& ra, uint32_t info) {
-  const uint32_t sec = (info & 0xFFFFFFu) * ra.nt33 + ra.t33;
-  const uint32_t bytes = kMetaBytes + 128u * (((info >> 24) + 1u) & ~1u);
-  const uint8_t* line = ra.lines + 128ull * (sec >> 2);      // the record's first line, plus this lane's
-  const uint32_t on = (ra.lane128 < 32u * (sec & 3u) + bytes) ? 1u : 0u;
+// Ask L2 for what one row (k | b << 24) will load: the 2 ceil(b/2) plane lines
+// of its record (lane p < 2 ceil(b/2): line p, 128 bytes) and its scale/zero
+// words (lane b_max, 32 bytes), one request per lane under a predicate.
+__device__ __forceinline__ void prefetch_row_l2(const RowAddr& ra, uint32_t info, int b_max) {
+  const uint32_t rec = (info & 0xFFFFFFu) * ra.nt + ra.t;
+  const uint32_t lines = ((info >> 24) + 1u) & ~1u;
+  const uint8_t* line = ra.line + (size_t)rec * ra.line_mul;
+  const uint32_t on = (ra.lane < lines || ra.lane == (uint32_t)b_max) ? 1u : 0u;
   asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p prefetch.global.L2 [%0];\n\t}" ::"l"(line),
                "r"(on));
 }
@@ -266,9 +279,9 @@ __device__ __forceinline__ void row_fma(const RowRegs& r, float2 (&acc)[16], flo
   uint32_t R[8];
   float mid;
   assemble_row<kBmax>(r, R, mid);
-  float A0, A1;
-  row_coef<kBmax>(r.m, mid, __half2float(__ushort_as_half((unsigned short)r.xh)), A0, A1, cacc);
-  fma_codes(R, A0, A1, acc);
+  float A;
+  row_coef<kBmax>(r.m, r.xh, mid, A, cacc);
+  fma_codes(R, A, acc);
 }
 
 // ---------------------------------------------------------------------------
@@ -402,9 +415,9 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
     RowRegs S[kDepth];
 #pragma unroll
     for (int d = 0; d < kDepth; ++d)
-      if (d < nrow) load_row(xv, ra, s.u.rows[h + kWarps * d], S[d]);
+      if (d < nrow) load_row<kBmax>(xv, ra, s.u.rows[h + kWarps * d], S[d]);
 #pragma unroll 1
-    for (int m = kDepth; m < min(nrow, kDepth + kL2Ahead); ++m) prefetch_row_l2(ra, s.u.rows[h + kWarps * m]);
+    for (int m = kDepth; m < min(nrow, kDepth + kL2Ahead); ++m) prefetch_row_l2(ra, s.u.rows[h + kWarps * m], kBmax);
     int m0 = 0;
     // blocks whose loads and prefetches all exist: no per-row tests
 #pragma unroll 1
@@ -413,16 +426,16 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
       for (int d = 0; d < kDepth; ++d) {
         const int m = m0 + d;
         row_fma<kBmax>(S[d], acc, cacc);
-        load_row(xv, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
+        load_row<kBmax>(xv, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
         // the record prefix of the row kL2Ahead rows further on goes to L2 now,
         // one 128-byte line per lane, so its register loads later hit L2
-        prefetch_row_l2(ra, s.u.rows[h + kWarps * (m + kDepth + kL2Ahead)]);
+        prefetch_row_l2(ra, s.u.rows[h + kWarps * (m + kDepth + kL2Ahead)], kBmax);
       }
     }
     // the last blocks, row by row: first the record prefixes of the rows that no
     // block above sent to L2
 #pragma unroll 1
-    for (int m = m0 + kDepth + kL2Ahead; m < nrow; ++m) prefetch_row_l2(ra, s.u.rows[h + kWarps * m]);
+    for (int m = m0 + kDepth + kL2Ahead; m < nrow; ++m) prefetch_row_l2(ra, s.u.rows[h + kWarps * m], kBmax);
 #pragma unroll 1
     for (; m0 < nrow; m0 += kDepth) {
 #pragma unroll
@@ -430,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_kernel(const VmmArgs a) {
         const int m = m0 + d;
         if (m < nrow) {
           row_fma<kBmax>(S[d], acc, cacc);
-          if (m + kDepth < nrow) load_row(xv, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
+          if (m + kDepth < nrow) load_row<kBmax>(xv, ra, s.u.rows[h + kWarps * (m + kDepth)], S[d]);
         }
       }
     }
@@ -578,10 +591,10 @@ __device__ __forceinline__ void load_row_lut(const uint16_t* __restrict__ x, con
                                              RowRegs& r) {
   constexpr uint32_t kRowBytes = 1u << (kBmax + 2);
   const uint32_t k = info & 0xFFFFFFu, b = info >> 24;
-  const uint32_t sec = k * ra.nt33 + ra.t33;
+  const uint32_t rec = k * ra.nt + ra.t;
   r.b = b;
   r.xh = __ldg(x + k);
-  const uint8_t* pw = ra.pairs + 32ull * sec;
+  const uint8_t* pw = ra.pairs + (size_t)rec * (uint32_t)record_bytes_for(kBmax);
   ld_stream2_at<0>(pw, r.p[0], r.p[1]);
   ld_stream2_at_if<1 * kPairBytes>(b > 2, pw, r.p[2], r.p[3]);
   ld_stream2_at_if<2 * kPairBytes>(b > 4, pw, r.p[4], r.p[5]);
@@ -709,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_lut_kernel(const VmmArgs a) {
       else cp_async_commit();
     }
 #pragma unroll 1
-    for (int m = kDepth; m < min(nrow, kDepth + kL2Ahead); ++m) prefetch_row_l2(ra, s.rows[h + kWarps * m]);
+    for (int m = kDepth; m < min(nrow, kDepth + kL2Ahead); ++m) prefetch_row_l2(ra, s.rows[h + kWarps * m], kBmax);
     int m0 = 0;
 #pragma unroll 1
     for (; m0 + 2 * kDepth + kL2Ahead <= nrow; m0 += kDepth) {
@@ -718,11 +731,11 @@ __global__ void __launch_bounds__(kThreads, 1) vmm_lut_kernel(const VmmArgs a) {
         const int m = m0 + d;
         row_lut<kBmax>(S[d], raw0 + d * 2 * kLutRaw, tab0 + d * kLutSlot, w, acc);
         load_row_lut<kBmax>(xv, a.lut, ra, s.rows[h + kWarps * (m + kDepth)], raw0 + d * 2 * kLutRaw, w, S[d]);
-        prefetch_row_l2(ra, s.rows[h + kWarps * (m + kDepth + kL2Ahead)]);
+        prefetch_row_l2(ra, s.rows[h + kWarps * (m + kDepth + kL2Ahead)], kBmax);
       }
     }
 #pragma unroll 1
-    for (int m = m0 + kDepth + kL2Ahead; m < nrow; ++m) prefetch_row_l2(ra, s.rows[h + kWarps * m]);
+    for (int m = m0 + kDepth + kL2Ahead; m < nrow; ++m) prefetch_row_l2(ra, s.rows[h + kWarps * m], kBmax);
 #pragma unroll 1
     for (; m0 < nrow; m0 += kDepth) {
 #pragma unroll
@@ -934,24 +947,14 @@ size_t vmm_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
 int vmm_fused_max_k() { return kFusedMaxK; }
 
-// The scratch's device address on the current device, looked up once per
-// device (with that device current) and remembered.
+// The scratch's device address in the current device's context. Looked up on
+// every call: a host-side query, and a context that was reset and created again
+// may have loaded the module (and the array) at another address.
 cudaError_t vmm_noalloc_scratch(void** ptr) {
-  constexpr int kMaxDevices = 64;
-  static std::mutex mu;
-  static void* addr[kMaxDevices] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_vmm_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_vmm_scratch);
-    if (e != cudaSuccess) return e;
-    addr[dev] = p;
-  }
-  *ptr = addr[dev];
+  *ptr = p;
   return cudaSuccess;
 }
 

@@ -136,7 +136,8 @@ def layout(K: int, N: int, b_max: int = 8) -> Layout:
 
 @dataclass
 class PackedLayer:
-    """Bit-plane packed K x N layer: one uint8 buffer of (row, tile) records."""
+    """Bit-plane packed K x N layer: one uint8 buffer holding the planes of every
+    (row, tile) record, then the scale/zero words of every record."""
     layout: Layout
     packed: torch.Tensor
 
@@ -152,11 +153,26 @@ class PackedLayer:
     def b_max(self):
         return self.layout.b_max
 
-    def meta_words(self) -> torch.Tensor:
-        """uint32 view [K, n_tiles, 8] of the scale | zero << 16 words of every record."""
+    @property
+    def meta_offset(self) -> int:
+        """Byte offset of the scale/zero words: after the planes of every record."""
         L = self.layout
-        rec = self.packed.view(L.K, L.n_tiles, L.record_bytes)
-        return rec[:, :, :32].contiguous().view(torch.int32).view(L.K, L.n_tiles, 8)
+        return L.K * L.n_tiles * L.record_bytes
+
+    def planes(self) -> torch.Tensor:
+        """uint8 view [K, n_tiles, record_bytes] of every record's planes (plane pair s in bytes 256 s .. 256 s + 255)."""
+        L = self.layout
+        return self.packed[: self.meta_offset].view(L.K, L.n_tiles, L.record_bytes)
+
+    def meta_bytes(self) -> torch.Tensor:
+        """uint8 view [K, n_tiles, 32] of every record's scale/zero words."""
+        L = self.layout
+        return self.packed[self.meta_offset: self.meta_offset + L.K * L.n_tiles * 32].view(L.K, L.n_tiles, 32)
+
+    def meta_words(self) -> torch.Tensor:
+        """int32 copy [K, n_tiles, 8] of the scale | zero << 16 words of every record."""
+        L = self.layout
+        return self.meta_bytes().contiguous().view(torch.int32).view(L.K, L.n_tiles, 8)
 
 
 def empty_packed(K: int, N: int, device="cuda", b_max: int = 8) -> PackedLayer:

@@ -66,6 +66,17 @@ def _weights(torch, gen, K, N, dev):
     return W * 0.02
 
 
+def kernel_source_hash():
+    """sha256 of the VMM kernel sources (vmm.cu, common.cuh): the key under which a
+    traffic capture is valid."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("vmm.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "activation_graded_bit_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -361,13 +372,16 @@ def run_gpu(args):
         L = pr["packed"].layout
         launches_per_step += 2 + (1 if pr["ws"].numel() > 16 + L.n_tiles * 4096 else 0)
 
-    # DRAM traffic comes from an ncu capture of the default workload (Llama3-8B
-    # linears, b_max 8); for any other workload it was not measured
+    # DRAM traffic per step comes from an ncu capture (profiles/vmm_traffic.json)
+    # of the default workload; it is reported only when that capture was taken on
+    # the kernel source that runs now (same hash), else null
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "vmm_traffic.json")
     if os.path.exists(tpath) and FAMILY == "llama3" and BMAX == 8:
         try:
-            traffic = json.load(open(tpath)).get("bytes_per_launch_scaled")
+            tj = json.load(open(tpath))
+            if tj.get("kernel_source_sha256") == kernel_source_hash():
+                traffic = tj.get("bytes_per_launch_scaled")
         except Exception:
             traffic = None
 

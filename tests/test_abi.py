@@ -43,10 +43,10 @@ def test_version_and_status_strings(g):
 def test_layout(g):
     L = g.layout(4096, 14336)
     assert (L.K, L.N, L.n_groups, L.tile_n, L.n_tiles) == (4096, 14336, 112, 1024, 14)
-    assert L.record_bytes == 32 + 8 * 128
-    assert L.packed_bytes == 4096 * 14 * 1056
+    assert L.record_bytes == 8 * 128                      # the planes of one (row, tile) record
+    assert L.packed_bytes == 4096 * 14 * (1024 + 32)       # planes, then 32 bytes of scale/zero per record
     L = g.layout(4, 4)
-    assert (L.n_groups, L.n_tiles, L.record_bytes) == (1, 1, 1056)
+    assert (L.n_groups, L.n_tiles, L.record_bytes) == (1, 1, 1024)
     for K, N in ((0, 4), (4, 0), (-1, 5), (1 << 24 + 1, 1), (1 << 24, 1 << 24)):
         with pytest.raises(g.GrinqhError) as e:
             g.layout(K, N)
@@ -125,11 +125,11 @@ def test_host_validation_rejects_before_launch(g):
 
 
 def test_layout_bmax(g):
-    for bmax, rec in ((2, 288), (4, 544), (6, 800), (8, 1056)):
+    for bmax, rec in ((2, 256), (4, 512), (6, 768), (8, 1024)):
         L = g.layout(4096, 4096, bmax)
         assert (L.b_max, L.record_bytes, L.reserved) == (bmax, rec, 0)
-        assert L.record_bytes == 32 + 128 * bmax and L.record_bytes % 32 == 0
-        assert L.packed_bytes == 4096 * 4 * rec
+        assert L.record_bytes == 128 * bmax and L.record_bytes % 128 == 0
+        assert L.packed_bytes == 4096 * 4 * (rec + 32)
     assert g.layout(8, 8).b_max == 8
     for bad in (0, 1, 3, 5, 7, 9, 16, -2):
         with pytest.raises(g.GrinqhError) as e:

@@ -74,7 +74,7 @@ def test_plain_c_program_uses_the_abi(lib, orc, tmp_path):
     out = subprocess.run([str(exe), str(wpath), str(K), str(N), str(opath)], capture_output=True, text=True)
     assert out.returncode == 0, out.stderr
     lines = dict(l.split(" ", 1) for l in out.stdout.strip().splitlines())
-    assert lines["layout"].split() == ["4096", "14336", "112", "14", "1056", str(4096 * 14 * 1056)]
+    assert lines["layout"].split() == ["4096", "14336", "112", "14", "1024", str(4096 * 14 * (1024 + 32))]
     assert int(lines["lut_bytes"]) == 4096 * 1024
     assert lines["status"] == "ok|workspace missing or too small"
     P = np.array([float(v) for v in lines["maxent"].split()])

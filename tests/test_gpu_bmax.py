@@ -30,7 +30,7 @@ def _even_classes(bmax):
 def _pack_check(g, orc, W, bmax, bits):
     K, N = W.shape
     p = g.pack(torch.from_numpy(W).cuda(), b_max=bmax)
-    assert p.layout.b_max == bmax and p.layout.record_bytes == 32 + 128 * bmax
+    assert p.layout.b_max == bmax and p.layout.record_bytes == 128 * bmax
     q, s, z = orc.rtn_quantize(W, bmax)
     ms, mz = meta_split(p)
     assert np.array_equal(ms, s), "scale bits differ"

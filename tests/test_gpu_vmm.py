@@ -101,12 +101,11 @@ def test_skipped_rows_are_never_used(g, orc):
     skip = np.nonzero(bits == 0)[0]
     assert skip.size > 50
     L = p.layout
-    rec = p.packed.view(K, L.n_tiles, L.record_bytes)
+    planes, meta = p.planes(), p.meta_bytes()
     sk = torch.from_numpy(skip).cuda()
     nan_words = torch.full((skip.size, L.n_tiles, 8), 0x7E007E00, dtype=torch.int32, device="cuda")
-    rec[sk, :, :32] = nan_words.view(torch.uint8).view(skip.size, L.n_tiles, 32)   # NaN scale and zero
-    rec[sk, :, 32:] = torch.randint(0, 256, (skip.size, L.n_tiles, L.record_bytes - 32), dtype=torch.uint8,
-                                    device="cuda")
+    meta[sk] = nan_words.view(torch.uint8).view(skip.size, L.n_tiles, 32)   # NaN scale and zero
+    planes[sk] = torch.randint(0, 256, (skip.size, L.n_tiles, L.record_bytes), dtype=torch.uint8, device="cuda")
     sel = g.select(dev_u16(x), torch.from_numpy(th).cuda(), CL)
     y = _vmm_guarded(g, p, dev_u16(x), sel, g.vmm_workspace(L))
     assert np.all(np.isfinite(y))
@@ -129,7 +128,7 @@ def test_brute_force_4x4(g, orc):
         y = g.vmm(p, xd, sel, ws).cpu().numpy()
         yr, bound = orc.vmm(x, q, s, z, bits)
         worst = max(worst, assert_close(y, yr, bound, str(b)))
-    assert int(ws[:16].count_nonzero()) == 0
+    assert int(ws[:16].count_nonzero()) == 0, "status word set"
 
 
 def test_brute_force_4x4_threshold_driven(g, orc):
