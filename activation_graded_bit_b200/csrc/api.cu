@@ -240,6 +240,7 @@ grinqh_status grinqh_select(const uint16_t* x, int32_t K, const float* threshold
                             int32_t n_classes, uint8_t* bits, int32_t* idx, int32_t* offsets, void* stream) {
   if (!valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
   if (K < 1 || K > kMaxDim) return GRINQH_ERR_INVALID_ARG;
+  if (K > kSelectMaxK) return GRINQH_ERR_UNSUPPORTED;
   if (!x || !bits || !idx || !offsets || (n_classes > 1 && !thresholds)) return GRINQH_ERR_INVALID_ARG;
   if (!aligned(x, 2) || !aligned(idx, 4) || !aligned(offsets, 4) || (thresholds && !aligned(thresholds, 4)))
     return GRINQH_ERR_ALIGNMENT;

@@ -34,6 +34,9 @@ struct ClassTable {
   uint8_t width[9];   // bit width of class j
 };
 
+// Largest K of launch_select: each 1024-channel block reads all of x to count
+// the channels ahead of it, K^2 / 512 bytes of L2 reads per call (8 MiB here).
+constexpr int kSelectMaxK = 1 << 16;
 cudaError_t launch_select(const uint16_t* x, int K, const float* thresholds, const ClassTable& ct,
                           uint8_t* bits, int32_t* idx, int32_t* offsets, cudaStream_t st);
 

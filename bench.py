@@ -547,8 +547,15 @@ def run_profile_case(args):
             g.vmm(p, x_d, sel, ws, y=y)
     torch.cuda.synchronize()
     assert bool(torch.isfinite(y).all())
-    print("profile case %s @ %g bits: %d select+%s calls" % (args.profile, args.bits, args.iters,
-                                                              "vmm_lut" if args.lut else "vmm"))
+    # the counts a capture is divided by: (row, tile) records of nonzero width and
+    # the algorithmic bytes of one call (planes of the selected widths, the
+    # records' scale/zero words, x, the channel list and y)
+    bits = sel.bits.cpu().numpy().astype(np.int64)
+    active = int((bits > 0).sum())
+    alg = bits.sum() * N / 8.0 + 4.0 * ((N + 127) // 128) * active + 2.0 * K + 4.0 * active + 4.0 * N
+    print("profile case %s @ %g bits: %d select+%s calls; %d active rows, %d records, %d algorithmic bytes"
+          % (args.profile, args.bits, args.iters, "vmm_lut" if args.lut else "vmm", active,
+             active * p.layout.n_tiles, int(alg)))
 
 
 

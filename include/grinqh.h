@@ -72,22 +72,25 @@ typedef enum {
  * Physical layout of a packed K x N layer. Filled by grinqh_layout_init or
  * grinqh_layout_init_bmax; treat as read-only. One device buffer (packed_bytes,
  * 16-byte aligned) holds the layer. Each row is cut into n_tiles column tiles
- * of tile_n = 1024 columns; row k, tile t is one record of record_bytes =
- * 32 + 128 * b_max bytes (1056 for b_max = 8) at byte offset
- * (k*n_tiles + t)*record_bytes (a row's tiles are adjacent):
- *   bytes [0, 32)      8 uint32 words; word g is scale_fp16 | (zero_fp16 << 16)
- *                      of columns [t*1024 + 128g, +128) (0 past the last group);
- *   bytes [32, ...)    the b_max bit planes of the b_max-bit codes, MSB first
- *                      (plane p = 0 is bit b_max-1 of the code, p = b_max-1 is
- *                      bit 0), in b_max/2 plane pairs (the paper's 2-bit
- *                      segments): pair s holds planes 2s and 2s+1 in bytes
- *                      [32 + 256s, 32 + 256(s+1)).
- * So the scale/zero words and the top b planes of a (row, tile) are one
- * contiguous, 32-byte-aligned run of 32 + 256 ceil(b/2) bytes (for odd b the
- * last pair's second plane is read and not used). Inside pair s, 32-bit word
- * 2w holds local columns 32w..32w+15 and word 2w+1 columns 32w+16..32w+31; in
- * either word, column 4j' + i of that half (j' in 0..3, i in 0..3) of plane
- * 2s + l sits at bit (8i + 2j' + 7 - 2s - l) mod 32. Columns >= N are zero bits.
+ * of tile_n = 1024 columns; row k, tile t is record r = k*n_tiles + t (a row's
+ * tiles are adjacent). The buffer holds two arrays:
+ *   planes   bytes [0, K*n_tiles*record_bytes): record r's planes at byte
+ *            r*record_bytes, record_bytes = 128 * b_max (1024 for b_max = 8):
+ *            the b_max bit planes of the b_max-bit codes, MSB first (plane
+ *            p = 0 is bit b_max-1 of the code, p = b_max-1 is bit 0), in b_max/2
+ *            plane pairs (the paper's 2-bit segments): pair s holds planes 2s
+ *            and 2s+1 in bytes [256s, 256(s+1)) of the record;
+ *   scale/zero  bytes [K*n_tiles*record_bytes, packed_bytes): 32 bytes per
+ *            record, record r's at r*32 from the start of the array: 8 uint32
+ *            words, word g = scale_fp16 | (zero_fp16 << 16) of columns
+ *            [t*1024 + 128g, +128) (0 past the last group).
+ * So the top b planes of a (row, tile) are one contiguous, 256-byte-aligned run
+ * of 256 ceil(b/2) bytes (for odd b the last pair's second plane is read and
+ * not used), and its scale/zero words one 32-byte sector: no DRAM sector holds
+ * bytes of two records. Inside pair s, 32-bit word 2w holds local columns
+ * 32w..32w+15 and word 2w+1 columns 32w+16..32w+31; in either word, column
+ * 4j' + i of that half (j' in 0..3, i in 0..3) of plane 2s + l sits at bit
+ * (8i + 2j' + 7 - 2s - l) mod 32. Columns >= N are zero bits.
  */
 typedef struct {
   int32_t K;             /* input channels (rows) */
@@ -95,10 +98,10 @@ typedef struct {
   int32_t n_groups;      /* ceil(N / 128) */
   int32_t tile_n;        /* columns per tile (1024) */
   int32_t n_tiles;       /* ceil(N / tile_n) */
-  int32_t record_bytes;  /* bytes per (row, tile) record: 32 + 128 * b_max */
+  int32_t record_bytes;  /* plane bytes per (row, tile) record: 128 * b_max */
   int32_t b_max;         /* bits per stored code: 2, 4, 6 or 8 */
   int32_t reserved;      /* 0 */
-  int64_t packed_bytes;  /* K * n_tiles * record_bytes */
+  int64_t packed_bytes;  /* K * n_tiles * (record_bytes + 32): planes, then scale/zero words */
 } grinqh_layout;
 
 /* Library version string (static storage). */
@@ -114,9 +117,9 @@ const char* grinqh_status_string(grinqh_status s);
 grinqh_status grinqh_layout_init(int32_t K, int32_t N, grinqh_layout* out);
 
 /*
- * The same for codes of b_max bits. Paper: Section 3.3 ("each weight is
- * quantized to a b_max-bit integer", stored as 2-bit segments, so widths
- * b in {0, 2, ..., b_max} can be fetched; b_max in {4, 6, 8} is evaluated).
+ * The same for codes of b_max bits. Paper: Section 3.3 (every weight becomes
+ * one b_max-bit integer kept as 2-bit segments, so that any even width
+ * b in {0, 2, ..., b_max} can be fetched; the evaluation uses b_max in {4, 6, 8}).
  * This library takes any width 0..b_max (1-bit planes in pairs) and
  * b_max in {2, 4, 6, 8}; grinqh_layout_init(K, N, out) is b_max = 8. Host only.
  * Errors: INVALID_ARG for out == NULL, sizes outside the limits above or b_max
@@ -300,7 +303,12 @@ grinqh_status grinqh_calibrate(const uint16_t* X, int32_t S, int32_t K, const ui
  *   offsets    device int32 [n_classes + 1], output: offsets[j] = first position
  *              of class j in idx, offsets[n_classes] = K.
  * All device pointers 4-byte aligned except x (2) and bits (1).
- * Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ * Limits: 1 <= K <= 65536. Every block of 1024 channels reads all of x (from
+ * L2) to count the channels of each class ahead of it, so one call reads
+ * K^2 / 512 bytes from L2: 8 MiB at K = 65536, more than every linear of the
+ * evaluated models needs. For larger K the call returns UNSUPPORTED; callers
+ * with such layers build idx and offsets themselves for grinqh_vmm.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (K > 65536), CUDA.
  */
 grinqh_status grinqh_select(const uint16_t* x, int32_t K, const float* thresholds,
                             const uint8_t* classes, int32_t n_classes, uint8_t* bits,

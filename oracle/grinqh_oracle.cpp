@@ -75,9 +75,9 @@ uint16_t orc_f64_to_f16(double v) {
 
 // ---------------------------------------------------------------------------
 // RTN asymmetric quantisation to b_max bits per (row k, 128-column group g).
-// Paper: Section 3.3 ("each weight w_ij is quantized to a b_max-bit integer",
-// with scale s and zero point z fixed at full b_max precision; b_max in
-// {4, 6, 8} is evaluated), Section 4 (RTN, G = 128) and Appendix E.1 (the RTN
+// Paper: Section 3.3 (every weight w_ij becomes one b_max-bit integer whose
+// scale s and zero point z are set once at the full b_max precision; the
+// evaluation uses b_max in {4, 6, 8}), Section 4 (RTN, G = 128) and Appendix E.1 (the RTN
 // model at b_max is the parent of every truncated width).
 // Library convention, with L = 2^b_max - 1 levels: s = fp16(range / L) rounded
 // to nearest even straight from fp64, s := 1 if that rounds to 0, s := 65504

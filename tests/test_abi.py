@@ -90,6 +90,8 @@ def test_host_validation_rejects_before_launch(g):
     assert g._select(P(0x1000), 8, P(0x1000), ctypes.addressof(bad_cl), 3, P(0x1000), P(0x1000), P(0x1000), None) == 1
     assert g._select(P(0x1000), 8, P(0x1000), ctypes.addressof(cl), 10, P(0x1000), P(0x1000), P(0x1000), None) == 1
     assert g._select(P(0x1000), 0, P(0x1000), ctypes.addressof(cl), 5, P(0x1000), P(0x1000), P(0x1000), None) == 1
+    # beyond 65536 channels the chunked count would read K^2/512 bytes: refused before any launch
+    assert g._select(P(0x1000), 65537, P(0x1000), ctypes.addressof(cl), 5, P(0x1000), P(0x1000), P(0x1000), None) == 3
     assert g._select(P(0x1000), 8, P(0x1000), ctypes.addressof(cl), 5, P(0x1000), P(0x1002), P(0x1000), None) == 2
     assert g._select(None, 8, P(0x1000), ctypes.addressof(cl), 5, P(0x1000), P(0x1000), P(0x1000), None) == 1
     # vmm: workspace too small / missing, misaligned y
