@@ -393,11 +393,9 @@ def run_gpu(args):
             "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step / args.steps, 6), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "u8 planes, fp32 accumulate", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "pairs_per_step": n_pairs, "classes": list(CLASSES), "b_max": BMAX,
-                       "l2": "inputs larger than L2: every pair of a step reads its own packed copy; "
-                             "%d packed layers (%.2f GB) rotate" % (
-                                 len(pairs), sum(pr["packed"].packed.numel() for pr in pairs) / 1e9),
-                       "parallelism": "replicas only" if world > 1 else "single GPU"},
+            "config": _config(n_pairs),
+            "parallelism": "replicas only" if world > 1 else "single GPU",
+            "resident_bytes": int(sum(pr["packed"].packed.numel() for pr in pairs)),
             "vmm_us": round(us_vmm, 4), "select_plus_vmm_us": round(us_pair, 4),
             "select_vmm_fused": {"us": round(us_fused, 4), "achieved": round(achieved_fused, 1), "unit": "GB/s",
                                  "frac": round(achieved_fused / peak, 4),
@@ -488,25 +486,75 @@ def cpu_baseline(args):
             "cpu_model": _cpu_model()}
 
 
+def _config(n_pairs):
+    """The workload description both arms print (the same dict: same config)."""
+    return {"workload": WORKLOAD, "pairs_per_step": n_pairs, "classes": list(CLASSES), "b_max": BMAX,
+            "l2": "inputs larger than L2: every pair of a step reads its own packed copy of its layer, "
+                  "the copies rotate"}
+
+
+def _oracle_pairs(cols):
+    """Untimed setup of the reference arm: for each of the 21 (linear, width)
+    pairs of a step, the same weights, thresholds and activation vector as the
+    CPU baseline draws, RTN codes of a column sample (`cols` columns as whole
+    128-column groups spread over the layer, the last group included)."""
+    import oracle
+    from activation_graded_bit_b200 import workloads as wl
+    classes = np.array(CLASSES, np.uint8)
+    shapes, draw = _family(wl)
+    pairs = []
+    for li, (name, K, N) in enumerate(shapes):
+        W = (wl.weights_rowstd_loguniform(K, N, key=(1, 9, li, 0)) if FAMILY == "qwen3"
+             else wl.weights_gaussian(K, N, key=(1, 9, li, 0)))
+        ng = (N + 127) // 128
+        take = max(1, min(ng, cols // 128))
+        groups = sorted(set(np.linspace(0, ng - 1, take).round().astype(int).tolist()))
+        sel_cols = np.concatenate([np.arange(128 * g, min(N, 128 * g + 128)) for g in groups])
+        q, s, z = oracle.rtn_quantize(np.ascontiguousarray(W[:, sel_cols]), BMAX)
+        del W
+        Xc = draw(K, 32, (1, 0, li, 1), li)
+        for ti, t in enumerate(TARGETS):
+            th = oracle.thresholds(Xc, oracle.maxent_distribution(classes, t))
+            x = draw(K, 1, (1, 0, li, 2 + ti), li)[0]
+            pairs.append(dict(name="%s@%g" % (name, t), x=x, th=th, q=q, s=s, z=z, N=N, n=len(sel_cols)))
+    return pairs
+
+
 def run_reference(args):
+    """The reference arm: the fp64 CPU oracle (select + VMM) on every one of the
+    step's 21 (linear, width) pairs, each step. Selection runs on the whole
+    vector; the VMM on a column sample of each layer, its time scaled by
+    N / sampled columns (the oracle's VMM time is linear in the columns it
+    computes). value = mean microseconds per pair, like the GPU arm."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import oracle
     nthreads = os.cpu_count() or 1
-    per = []
-    total_done = 0
+    cols = 1024
+    pairs = _oracle_pairs(cols)
+    classes = np.array(CLASSES, np.uint8)
+    per_step = []
     for i in range(args.warmup + args.steps):
-        done, secs, names = _oracle_sample(args.cpu_budget / max(args.steps + args.warmup, 1), nthreads)
+        tot = 0.0
+        for pr in pairs:
+            t0 = time.perf_counter()
+            bits, idx, off = oracle.select(pr["x"], pr["th"], classes)
+            t1 = time.perf_counter()
+            oracle.vmm(pr["x"], pr["q"], pr["s"], pr["z"], bits, nthreads=nthreads, bmax=BMAX)
+            t2 = time.perf_counter()
+            tot += (t1 - t0) + (t2 - t1) * pr["N"] / pr["n"]
         if i >= args.warmup:
-            per.append(secs / max(done, 1))
-            total_done += done
-    v = statistics.mean(per) * 1e6
+            per_step.append(tot / len(pairs))
+    v = statistics.mean(per_step) * 1e6
+    sample = ("fp64 oracle select (whole x) + vmm on %d-column samples of each layer (time scaled by N/%d), "
+              "all %d (linear, width) pairs every step" % (cols, cols, len(pairs)))
     out = {"impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": 0,
            "steps": args.steps, "warmup": args.warmup, "higher_is_better": False, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": WORKLOAD, "parallelism": "host cores"},
+           "config": _config(len(pairs)), "parallelism": "host cores",
            "cpu_baseline": {"value": round(v, 1), "unit": UNIT, "cores": nthreads, "kind": "oracle",
-                            "sample": "fp64 oracle select+vmm, %d pairs over %d steps" % (total_done, args.steps)},
+                            "sample": sample},
            "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out))
 
@@ -589,32 +637,43 @@ def _graph_time_us(torch, stream, fn, reps, warmup=3):
 
 
 def run_sweep(args):
-    """Average-bit sweep on a 14336x4096 layer: microseconds and effective GB/s
-    of the VMM (and of select+VMM) against the achieved mean width, Gaussian and
-    SiLU(a)*b activations, and a least-squares line t = a + b * mean_bits."""
+    """Average-bit sweep: microseconds, effective GB/s and roofline fraction of
+    the VMM (and of select+VMM and the fused call) against the achieved mean
+    width, with a least-squares line t = a + b * mean_bits per shape and
+    activation distribution. Shapes: the 14336x4096 down-proj layer (Gaussian
+    and SiLU(a)*b activations) and the pages' isolated-kernel matrix 16384x4096
+    (Section 4 "Setup for Kernel Benchmarking", Appendix C.2 Fig. 11; Gaussian
+    activations), the latter also at the figure's configuration: b_max 8, target
+    4 bits, uniformly distributed thresholds, read as the five even widths
+    {0, 2, 4, 6, 8} with equal shares (mean width 4)."""
     import torch
     from activation_graded_bit_b200 import grinqh as g
     from activation_graded_bit_b200 import workloads as wl
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
-    K, N = 14336, 4096
-    classes = wl.CLASSES
-    copies = []
-    for c in range(6):   # 6 x 60 MB: a replay of one point never finds the weights in L2
-        gen = torch.Generator(device=dev)
-        gen.manual_seed(3_000_017 + c)
-        copies.append(g.pack(torch.randn(K, N, generator=gen, device=dev, dtype=torch.float32) * 0.02))
     stream = torch.cuda.Stream(device=dev)
-    ws = g.vmm_workspace(copies[0].layout, dev)
-    y = torch.empty(N, dtype=torch.float32, device=dev)
     peak, peak_kind = _peaks()
     points = []
-    for dist in ("gaussian", "silu_gated"):
-        gen_x = wl.activations_gaussian if dist == "gaussian" else wl.activations_silu_gated
-        Xc = torch.from_numpy(gen_x(K, 128, key=(3, 1, dist == "gaussian")).view(np.int16)).to(dev)
-        x = torch.from_numpy(gen_x(K, 1, key=(3, 2, dist == "gaussian"))[0].view(np.int16)).to(dev)
-        for t in (0.5, 1.0, 2.0, 3.0, 4.0, 5.0, 6.0, 8.0):
-            th = g.calibrate(Xc, classes, target_bits=t)
+    fits = {}
+    shapes = (("down_proj 14336x4096", 14336, 4096, ("gaussian", "silu_gated")),
+              ("isolated 16384x4096", 16384, 4096, ("gaussian",)))
+    for si, (label, K, N, dists) in enumerate(shapes):
+        copies = []
+        for c in range(6):   # 6 packed copies (>= 360 MB): a replay of one point never finds the weights in L2
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(3_000_017 + 101 * si + c)
+            copies.append(g.pack(torch.randn(K, N, generator=gen, device=dev, dtype=torch.float32) * 0.02))
+        ws = g.vmm_workspace(copies[0].layout, dev)
+        y = torch.empty(N, dtype=torch.float32, device=dev)
+        runs = [(d, wl.CLASSES, t, None) for d in dists for t in (0.5, 1.0, 2.0, 3.0, 4.0, 5.0, 6.0, 8.0)]
+        if si == 1:
+            runs.append(("gaussian", (0, 2, 4, 6, 8), 4.0, [0.2] * 5))   # Fig. 11's configuration
+        for dist, classes, t, P in runs:
+            gen_x = wl.activations_gaussian if dist == "gaussian" else wl.activations_silu_gated
+            Xc = torch.from_numpy(gen_x(K, 128, key=(3, 1, dist == "gaussian", si)).view(np.int16)).to(dev)
+            x = torch.from_numpy(gen_x(K, 1, key=(3, 2, dist == "gaussian", si))[0].view(np.int16)).to(dev)
+            th = (g.calibrate(Xc, classes, P=np.array(P, np.float64)) if P is not None
+                  else g.calibrate(Xc, classes, target_bits=t))
             sel = g.select(x, th, classes)
             torch.cuda.synchronize()
             bits = sel.bits.cpu().numpy().astype(np.int64)
@@ -625,34 +684,38 @@ def run_sweep(args):
                 for p in copies:
                     g.vmm(p, x, sel, ws, y=y, stream=st)
 
-            def pair(st, sel=sel, th=th):
+            def pair(st, sel=sel, th=th, classes=classes):
                 for p in copies:
                     g.select(x, th, classes, out=sel, stream=st)
                     g.vmm(p, x, sel, ws, y=y, stream=st)
-            def fused(st, th=th):
+
+            def fused(st, th=th, classes=classes):
                 for p in copies:
                     g.select_vmm(p, x, th, classes, ws, y=y, stream=st)
             tv = _graph_time_us(torch, stream, vmm_only, reps=8) / len(copies)
             tp = _graph_time_us(torch, stream, pair, reps=8) / len(copies)
             tf = _graph_time_us(torch, stream, fused, reps=8) / len(copies)
-            points.append(dict(dist=dist, target_bits=t, mean_bits=round(float(bits.mean()), 4),
-                               active_frac=round(active / K, 4), alg_bytes=int(alg), vmm_us=round(tv, 3),
-                               select_plus_vmm_us=round(tp, 3), select_vmm_fused_us=round(tf, 3),
-                               gbs=round(alg / (tv * 1e-6) / 1e9, 1),
+            points.append(dict(shape=label, K=K, N=N, dist=dist, classes=list(classes), target_bits=t,
+                               thresholds="uniform shares" if P is not None else "maximum entropy",
+                               mean_bits=round(float(bits.mean()), 4), active_frac=round(active / K, 4),
+                               alg_bytes=int(alg), vmm_us=round(tv, 3), select_plus_vmm_us=round(tp, 3),
+                               select_vmm_fused_us=round(tf, 3), gbs=round(alg / (tv * 1e-6) / 1e9, 1),
                                frac=round(alg / (tv * 1e-6) / 1e9 / peak, 4)))
-    fits = {}
-    for dist in ("gaussian", "silu_gated"):
-        pts = [q for q in points if q["dist"] == dist]
-        xb = np.array([q["mean_bits"] for q in pts])
-        tt = np.array([q["vmm_us"] for q in pts])
-        slope, icpt = np.polyfit(xb, tt, 1)
-        pred = icpt + slope * xb
-        r2 = 1.0 - float(((tt - pred) ** 2).sum() / ((tt - tt.mean()) ** 2).sum())
-        fits[dist] = dict(us_per_bit=round(float(slope), 4), us_at_0_bits=round(float(icpt), 4), r2=round(r2, 5))
-    print(json.dumps({"metric": "vmm us and effective GB/s vs average bits (14336x4096 sweep)", "unit": UNIT,
+        for dist in dists:
+            pts = [q for q in points if q["shape"] == label and q["dist"] == dist and q["thresholds"] != "uniform shares"]
+            xb = np.array([q["mean_bits"] for q in pts])
+            tt = np.array([q["vmm_us"] for q in pts])
+            slope, icpt = np.polyfit(xb, tt, 1)
+            pred = icpt + slope * xb
+            r2 = 1.0 - float(((tt - pred) ** 2).sum() / ((tt - tt.mean()) ** 2).sum())
+            fits["%s %s" % (label, dist)] = dict(us_per_bit=round(float(slope), 4), us_at_0_bits=round(float(icpt), 4),
+                                                 r2=round(r2, 5))
+        del copies
+        torch.cuda.empty_cache()
+    print(json.dumps({"metric": "vmm us, effective GB/s and roofline fraction vs average bits", "unit": UNIT,
                       "higher_is_better": False, "data": "synthetic", "peak": peak, "peak_kind": peak_kind,
-                      "config": {"workload": "down-proj-shaped 14336x4096, classes %s, 6 packed copies rotated"
-                                 % (list(classes),)}, "points": points, "linear_fit": fits}))
+                      "config": {"workload": "14336x4096 and 16384x4096 layers, 6 packed copies rotated per shape"},
+                      "points": points, "linear_fit": fits}))
 
 
 def run_stack(args):
@@ -937,6 +1000,7 @@ def run_cold(args):
     l2 = int(torch.cuda.get_device_properties(dev).L2_cache_size)
     flush = torch.empty(max(2 * l2 // 4, 1 << 20), dtype=torch.float32, device=dev)
     reps = max(args.iters, 5)
+    peak, peak_kind = _peaks()
     points = []
     for pr in pairs:
         t_sel, t_vmm = [], []
@@ -955,8 +1019,11 @@ def run_cold(args):
             if r > 0:
                 t_sel.append(e0.elapsed_time(e1) * 1e3)
                 t_vmm.append(e1.elapsed_time(e2) * 1e3)
+        tv = statistics.median(t_vmm)
+        alg = algorithmic_bytes(pr)[1]
         points.append({"linear": pr["name"], "K": pr["K"], "N": pr["N"], "target_bits": pr["target"],
-                       "select_us": round(statistics.median(t_sel), 3), "vmm_us": round(statistics.median(t_vmm), 3)})
+                       "select_us": round(statistics.median(t_sel), 3), "vmm_us": round(tv, 3),
+                       "alg_bytes": int(alg), "frac": round(alg / (tv * 1e-6) / 1e9 / peak, 4)})
     assert all(bool(torch.isfinite(pr["y"]).all()) for pr in pairs)
     n = len(points)
     print(json.dumps({"metric": "isolated cold select and VMM: µs per call after an L2 flush",
@@ -964,6 +1031,7 @@ def run_cold(args):
                       "config": {"workload": WORKLOAD, "classes": list(CLASSES), "b_max": BMAX,
                                  "l2": "%d bytes written before every call pair (2x L2)" % (4 * flush.numel()),
                                  "repetitions": reps},
+                      "peak": peak, "peak_kind": peak_kind,
                       "select_us_mean": round(sum(p["select_us"] for p in points) / n, 3),
                       "vmm_us_mean": round(sum(p["vmm_us"] for p in points) / n, 3),
                       "points": points}))
