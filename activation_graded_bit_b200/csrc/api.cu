@@ -144,6 +144,17 @@ grinqh_status grinqh_prefill(const grinqh_layout* layout, const void* packed, co
   return cuda_status(e);
 }
 
+grinqh_status grinqh_prefill_tc(const grinqh_layout* layout, const void* packed, const uint16_t* X, int32_t T,
+                                float* Y, uint32_t* status, void* stream) {
+  if (!layout_ok(layout) || !packed || !X || !Y || !status) return GRINQH_ERR_INVALID_ARG;
+  if (T < 1 || T > kMaxDim) return GRINQH_ERR_INVALID_ARG;
+  const grinqh_layout& L = *layout;
+  if (L.K % 8 != 0) return GRINQH_ERR_UNSUPPORTED;   // the TMA row pitch of X is a multiple of 16 bytes
+  if ((T + 255) / 256 > 65535) return GRINQH_ERR_UNSUPPORTED;   // token tiles on the grid's y axis
+  if (!aligned(packed, 16) || !aligned(X, 16) || !aligned(Y, 4) || !aligned(status, 16)) return GRINQH_ERR_ALIGNMENT;
+  return cuda_status(launch_prefill_tc(X, packed, T, L.K, L.N, L.n_tiles, L.b_max, Y, status, (cudaStream_t)stream));
+}
+
 grinqh_status grinqh_maxent_distribution(const uint8_t* classes, int32_t n_classes, double target_bits,
                                          double* P) {
   if (!valid_classes(classes, n_classes) || !P) return GRINQH_ERR_INVALID_ARG;

@@ -26,6 +26,13 @@ cudaError_t launch_dequant(const void* packed, int K, int N, int n_tiles, int b_
 
 // Y[T][N] (fp32) = X[T][K] (fp16) . W16[K][N] (fp16), fp32 accumulation, on the
 // stream (a plain library GEMM).
+// The fused prefill product on the tensor cores (prefill_tc.cu): X fp16 [T][K]
+// (K % 8 == 0, 16-byte aligned), Y fp32 [T][N]; bit 0 of *status is set if a
+// bounded wait of the kernel gave up.
+cudaError_t launch_prefill_tc(const uint16_t* X, const void* packed, int T, int K, int N, int n_tiles, int b_max,
+                              float* Y, uint32_t* status, cudaStream_t st);
+size_t prefill_tc_smem_bytes();
+
 cudaError_t launch_prefill_gemm(const uint16_t* X, const uint16_t* W16, float* Y, int T, int K, int N,
                                 cudaStream_t st);
 

@@ -1,0 +1,366 @@
+// Fused prefill product on the 5th-generation tensor cores (sm_100a):
+// Y[T][N] = X[T][K] . W_hat[K][N], with W_hat rebuilt from the packed bit planes
+// straight into the MMA's shared-memory operand tiles (no binary16 copy of the
+// weights in HBM).
+//
+// Paper: "GRINQH" Section 4, "Prefill vs. Decoding Evaluation": prefill takes
+// every weight at its full b_max precision and runs a dense matrix-matrix
+// product; Section 5 credits efficient unpacking fused with the product for the
+// prefill speed. The operand values are those of grinqh_dequant: w_hat =
+// fp16_rne(s * (q - z)) per (row k, 128-column group), q the b_max-bit code.
+//
+// One CTA computes a tile of 128 output columns (the MMA's M, from W_hat) by 256
+// tokens (the MMA's N, from X) with fp32 accumulators in tensor memory, looping
+// over K in stages of 64 rows held in a 4-deep shared-memory ring:
+//   warp 0      X tiles by TMA (no multicast): 256 tokens x 64 k, K-major,
+//               128-byte swizzle, one mbarrier transaction per stage;
+//   warp 1      allocates 256 TMEM columns and, from one lane, issues the four
+//               kind::f16 MMAs (K = 16 each) of a stage once both operand tiles
+//               are full, then commits to the stage's "empty" barrier;
+//   warps 2..5  rebuild the stage's 64 x 128 weight tile: 4 lanes per row, each
+//               lane the 32 columns of one record word, written as binary16 in the
+//               MN-major 128-byte-swizzled layout the A descriptor names; then,
+//               after the last stage, the epilogue (TMEM -> registers -> Y).
+// Every wait on an mbarrier is bounded by the global timer (about one second);
+// a wait that gives up sets bit 0 of the status word and the CTA skips the rest
+// of its work, frees its tensor memory and returns.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace grinqh {
+namespace {
+
+constexpr int kPM = 128;                       // output columns per CTA (MMA M)
+constexpr int kPN = 256;                       // tokens per CTA (MMA N)
+constexpr int kPK = 64;                        // k rows per stage (four MMAs of K = 16)
+constexpr int kPStages = 4;
+constexpr int kPABytes = kPM * kPK * 2;        // 16 KB of binary16 weights per stage
+constexpr int kPBBytes = kPN * kPK * 2;        // 32 KB of binary16 activations per stage
+constexpr int kPThreads = 192;
+constexpr unsigned long long kPWaitNs = 1000000000ull;   // bound of one wait
+
+struct PfSync {
+  unsigned long long full_a[kPStages];   // 4 arrivals: the rebuild warps
+  unsigned long long full_b[kPStages];   // 1 arrival + the TMA's bytes
+  unsigned long long empty[kPStages];    // the MMAs that read the stage have completed
+  unsigned long long accum;              // every MMA of the CTA has completed
+  uint32_t tmem;                         // base address of the accumulator columns
+  uint32_t failed;                       // some wait of this CTA gave up
+};
+
+constexpr size_t kPSmem = 1024 + (size_t)kPStages * (kPABytes + kPBBytes) + sizeof(PfSync);
+
+__device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void bar_expect(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool bar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+// Wait for the phase of parity `parity` to complete; false after about a second.
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
+  if (bar_test(bar, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (bar_test(bar, parity)) return true;
+    if (now_ns() - t0 > kPWaitNs) return false;
+  }
+}
+
+// 2-D tiled TMA load of box {64 k, 256 tokens} at (k0, t0) into shared memory.
+__device__ __forceinline__ void tma_x(uint32_t dst, const CUtensorMap* map, int k0, int t0, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(map), "r"(k0), "r"(t0), "r"(bar)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05): start address, leading and stride
+// byte offsets in 16-byte units, descriptor version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: D fp32, A and B binary16, A (weights)
+// MN-major, B (activations) K-major, N = 256, M = 128.
+constexpr uint32_t kPIdesc = (1u << 4) | (1u << 15) | ((uint32_t)(kPN >> 3) << 17) | ((uint32_t)(kPM >> 4) << 24);
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(kPIdesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// The binary16 weights of one (row, 32-column record word): fp16_rne(s (q - z))
+// for the lane's 32 columns, as 16 words of two values (columns 2i, 2i+1).
+template <int kBmax>
+__device__ __forceinline__ void rebuild_word(const uint8_t* __restrict__ planes, const uint8_t* __restrict__ meta,
+                                             int w, uint32_t (&h)[16]) {
+  uint32_t P[8];
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    if (2 * s < kBmax) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(planes + s * kPairBytes) + w);
+      P[2 * s] = v.x;
+      P[2 * s + 1] = v.y;
+    } else {
+      P[2 * s] = P[2 * s + 1] = 0u;
+    }
+  }
+  const uint32_t m = __ldg(reinterpret_cast<const uint32_t*>(meta) + (w >> 2));
+  const float sc = half_bits_to_float(m), z = half_bits_to_float(m >> 16);
+  uint32_t R[8];
+  assemble<kBmax>(P, R);   // byte i of R[j]: the code of column 4j+i in the 8-bit frame
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t q = R[j] >> (8 - kBmax);   // b_max-bit codes, one per byte
+    const __half2 lo = __floats2half2_rn(sc * ((float)(q & 0xFFu) - z), sc * ((float)((q >> 8) & 0xFFu) - z));
+    const __half2 hi = __floats2half2_rn(sc * ((float)((q >> 16) & 0xFFu) - z), sc * ((float)(q >> 24) - z));
+    h[2 * j] = *reinterpret_cast<const uint32_t*>(&lo);
+    h[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&hi);
+  }
+}
+
+template <int kBmax>
+__global__ void __launch_bounds__(kPThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint8_t* __restrict__ packed, size_t meta_offset,
+                      int T, int K, int N, int n_tiles, float* __restrict__ Y, uint32_t* __restrict__ status) {
+  extern __shared__ __align__(16) uint8_t pf_smem[];
+  const uint32_t raw = saddr(pf_smem);
+  const uint32_t a0 = (raw + 1023u) & ~1023u;   // 1 KB-aligned operand ring (swizzle atoms)
+  const uint32_t b0 = a0 + kPStages * kPABytes;
+  PfSync& sy = *reinterpret_cast<PfSync*>(pf_smem + (a0 - raw) + kPStages * (kPABytes + kPBBytes));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kPM, t0 = blockIdx.y * kPN;
+  const int n_k = (K + kPK - 1) / kPK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPStages; ++i) {
+      bar_init(saddr(&sy.full_a[i]), 4);
+      bar_init(saddr(&sy.full_b[i]), 1);
+      bar_init(saddr(&sy.empty[i]), 1);
+    }
+    bar_init(saddr(&sy.accum), 1);
+    sy.failed = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(&sy.tmem)),
+                 "r"(kPN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  const uint32_t tmem = sy.tmem;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ---------------- activations: one TMA per stage ----------------
+    int issued = -1;
+    for (int it = 0; it < n_k && ok; ++it) {
+      const int st = it % kPStages;
+      ok = bar_wait(saddr(&sy.empty[st]), ((uint32_t)(it / kPStages) & 1u) ^ 1u);
+      if (ok && lane == 0) {
+        bar_expect(saddr(&sy.full_b[st]), kPBBytes);
+        tma_x(b0 + st * kPBBytes, &xmap, it * kPK, t0, saddr(&sy.full_b[st]));
+      }
+      if (ok) issued = it;
+      __syncwarp();
+    }
+    // the CTA's last copies have landed before anything here can end
+    for (int it = (issued - kPStages + 1 > 0 ? issued - kPStages + 1 : 0); it <= issued; ++it)
+      bar_wait(saddr(&sy.full_b[it % kPStages]), (uint32_t)(it / kPStages) & 1u);
+  } else if (warp == 1) {
+    // ---------------- MMA issue ----------------
+    for (int it = 0; it < n_k && ok; ++it) {
+      const int st = it % kPStages;
+      const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
+      ok = bar_wait(saddr(&sy.full_a[st]), ph) && bar_wait(saddr(&sy.full_b[st]), ph);
+      tc_after();
+      if (ok && lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < kPK / 16; ++kk) {
+          // A: MN-major; 64-column atoms 1 KB apart along M, 8-row groups 2 KB apart along K
+          const uint64_t ad = smem_desc(a0 + st * kPABytes + kk * 4096, 1024, 2048);
+          // B: K-major rows of 128 bytes, 8-row groups 1 KB apart; K = 16 is 32 bytes into the row
+          const uint64_t bd = smem_desc(b0 + st * kPBBytes + kk * 32, 16, 1024);
+          mma_f16(tmem, ad, bd, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(saddr(&sy.empty[st]));
+      }
+      __syncwarp();
+    }
+    if (ok && lane == 0) mma_commit(saddr(&sy.accum));
+    __syncwarp();
+  } else {
+    // ---------------- weight rebuild ----------------
+    // warp d = warp - 2 rebuilds k rows 16 d .. 16 d + 15 of a stage, 8 rows per
+    // pass, lane = 4 (row in pass) + q; lane quarter q owns columns 32 q .. 32 q + 31
+    // of the CTA's 128, record word w = 4 (128-column slice of the tile) + q
+    const int d = warp - 2, q = lane & 3;
+    const int t_rec = n0 / kTileN, w = 4 * ((n0 % kTileN) / kPM) + q;
+    const size_t rbytes = (size_t)record_bytes_for(kBmax);
+    for (int it = 0; it < n_k && ok; ++it) {
+      const int st = it % kPStages;
+      ok = bar_wait(saddr(&sy.empty[st]), ((uint32_t)(it / kPStages) & 1u) ^ 1u);
+      if (!ok) break;
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        const int kl = 16 * d + 8 * pass + (lane >> 2);
+        const int k = it * kPK + kl;
+        uint32_t h[16];
+        if (k < K) {
+          const size_t rec = (size_t)k * n_tiles + t_rec;
+          rebuild_word<kBmax>(packed + rec * rbytes, packed + meta_offset + rec * kMetaBytes, w, h);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) h[j] = 0u;
+        }
+        // element (column c of the lane's 32, row kl): atom (kl / 8, q / 2) at
+        // (2 (kl / 8) + q / 2) KB, row kl % 8 at 128 bytes each, 16-byte chunk
+        // 4 (q % 2) + c / 8 stored at chunk index (chunk ^ (kl % 8))
+        const uint32_t r8 = (uint32_t)(kl & 7);
+        const uint32_t row = a0 + st * kPABytes + (uint32_t)((2 * (kl >> 3) + (q >> 1)) * 1024) + r8 * 128u;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const uint32_t chunk = ((uint32_t)(4 * (q & 1) + cc)) ^ r8;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + chunk * 16u), "r"(h[4 * cc]),
+                       "r"(h[4 * cc + 1]), "r"(h[4 * cc + 2]), "r"(h[4 * cc + 3])
+                       : "memory");
+        }
+      }
+      // the tensor core reads the tile through the async proxy
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) bar_arrive(saddr(&sy.full_a[st]));
+    }
+    // ---------------- epilogue ----------------
+    // TMEM lane i of quarter (warp % 4) holds output column n0 + 32 (warp % 4) + i;
+    // TMEM column j holds token t0 + j
+    if (ok) ok = bar_wait(saddr(&sy.accum), 0u);
+    tc_after();
+    if (ok) {
+      const int qq = warp & 3;
+      const int n = n0 + 32 * qq + lane;
+#pragma unroll 1
+      for (int cc = 0; cc < kPN / 32; ++cc) {
+        if (t0 + 32 * cc >= T) break;
+        uint32_t v[32];
+        const uint32_t taddr = tmem + ((uint32_t)(32 * qq) << 16) + (uint32_t)(32 * cc);
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+            "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+              "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]),
+              "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+              "=r"(v[30]), "=r"(v[31])
+            : "r"(taddr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (n < N) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int t = t0 + 32 * cc + i;
+            if (t < T) Y[(size_t)t * N + n] = __uint_as_float(v[i]);
+          }
+        }
+      }
+    }
+  }
+  if (!ok) sy.failed = 1u;
+  tc_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && sy.failed) atomicOr(status, 1u);
+  if (warp == 1) {
+    tc_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPN) : "memory");
+  }
+}
+
+}  // namespace
+
+size_t prefill_tc_smem_bytes() { return kPSmem; }
+
+cudaError_t launch_prefill_tc(const uint16_t* X, const void* packed, int T, int K, int N, int n_tiles, int b_max,
+                              float* Y, uint32_t* status, cudaStream_t st) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (encode == nullptr) {
+    cudaDriverEntryPointQueryResult qr;
+    void* fn = nullptr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr);
+    if (e != cudaSuccess) return e;
+    if (fn == nullptr || qr != cudaDriverEntryPointSuccess) return cudaErrorNotSupported;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)T};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2u};
+  const cuuint32_t box[2] = {(cuuint32_t)kPK, (cuuint32_t)kPN};
+  const cuuint32_t estr[2] = {1u, 1u};
+  if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const size_t meta_offset = meta_offset_for(K, n_tiles, b_max);
+  const dim3 grid((unsigned)((N + kPM - 1) / kPM), (unsigned)((T + kPN - 1) / kPN));
+  cudaError_t e;
+#define GRINQH_PF_CASE(B)                                                                                      \
+  case B:                                                                                                      \
+    e = cudaFuncSetAttribute(prefill_tc_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmem); \
+    if (e != cudaSuccess) return e;                                                                            \
+    prefill_tc_kernel<B><<<grid, kPThreads, kPSmem, st>>>(map, (const uint8_t*)packed, meta_offset, T, K, N,   \
+                                                          n_tiles, Y, status);                                 \
+    break;
+  switch (b_max) {
+    GRINQH_PF_CASE(2)
+    GRINQH_PF_CASE(4)
+    GRINQH_PF_CASE(6)
+    GRINQH_PF_CASE(8)
+    default: return cudaErrorInvalidValue;
+  }
+#undef GRINQH_PF_CASE
+  return cudaGetLastError();
+}
+
+}  // namespace grinqh

@@ -71,6 +71,7 @@ _batch_ws = _sig("grinqh_vmm_batch_workspace_bytes", [_LP, _I, ctypes.POINTER(ct
 _select_vmm_batch = _sig("grinqh_select_vmm_batch", [_LP, _P, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P])
 _dequant = _sig("grinqh_dequant", [_LP, _P, _P, _P])
 _prefill = _sig("grinqh_prefill", [_LP, _P, _P, _I, _P, _P, _P])
+_prefill_tc = _sig("grinqh_prefill_tc", [_LP, _P, _P, _I, _P, _P, _P])
 _pack_codes = _sig("grinqh_pack_codes", [_LP, _P, _P, _P])
 _lut_build = _sig("grinqh_lut_build", [_P, _I, _I, _I, _P, _P])
 _lut_bytes = _sig("grinqh_lut_bytes", [_LP, ctypes.POINTER(ctypes.c_size_t)])
@@ -81,7 +82,7 @@ EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grin
            "grinqh_unpack_codes", "grinqh_maxent_distribution", "grinqh_calibrate_workspace_bytes",
            "grinqh_calibrate", "grinqh_select", "grinqh_vmm_workspace_bytes", "grinqh_vmm",
            "grinqh_vmm_noalloc", "grinqh_select_vmm", "grinqh_vmm_batch_workspace_bytes",
-           "grinqh_select_vmm_batch", "grinqh_dequant", "grinqh_prefill", "grinqh_pack_codes",
+           "grinqh_select_vmm_batch", "grinqh_dequant", "grinqh_prefill", "grinqh_prefill_tc", "grinqh_pack_codes",
            "grinqh_lut_bytes", "grinqh_vmm_lut", "grinqh_lut_build")
 
 
@@ -350,6 +351,21 @@ def prefill(p: PackedLayer, X: torch.Tensor, Y: Optional[torch.Tensor] = None, W
     _need(W16, p.K * p.N, 2, "grinqh_prefill W16")
     _check(_prefill(ctypes.byref(p.layout), _ptr(p.packed), _ptr(X), T, _ptr(Y), _ptr(W16), _stream(stream)),
            "grinqh_prefill")
+    return Y
+
+
+def prefill_tc(p: PackedLayer, X: torch.Tensor, status: torch.Tensor, Y: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """grinqh_prefill_tc: Y fp32 [T, N] = X [T, K] (fp16 or its bit view) . w_hat at full
+    width, fused on the tensor cores; status is a zero-filled 16-byte CUDA tensor."""
+    assert X.is_cuda and X.dim() == 2 and X.is_contiguous() and X.element_size() == 2 and X.shape[1] == p.K
+    T = X.shape[0]
+    if Y is None:
+        Y = torch.empty((T, p.N), dtype=torch.float32, device=X.device)
+    _need(Y, T * p.N, 4, "grinqh_prefill_tc Y")
+    _need(status, 4, 4, "grinqh_prefill_tc status")
+    _check(_prefill_tc(ctypes.byref(p.layout), _ptr(p.packed), _ptr(X), T, _ptr(Y), _ptr(status), _stream(stream)),
+           "grinqh_prefill_tc")
     return Y
 
 

@@ -189,6 +189,29 @@ grinqh_status grinqh_prefill(const grinqh_layout* layout, const void* packed, co
                              float* Y, uint16_t* W16, void* stream);
 
 /*
+ * The prefill product fused on the tensor cores: the same Y = X . W_hat (same
+ * binary16 operands w_hat = fp16_rne(s (q - z)) as grinqh_dequant, fp32
+ * accumulation) without writing W_hat to memory: each CTA rebuilds a 128-column
+ * slice of W_hat from the bit planes into shared memory, 64 rows at a time, and
+ * the 5th-generation tensor cores (tcgen05, sm_100a) multiply it with TMA-loaded
+ * tiles of 256 tokens, accumulating in tensor memory. Paper: Section 4,
+ * "Prefill vs. Decoding Evaluation" (full b_max precision, dense product) and
+ * Section 5 (unpacking fused with the product). Allocates nothing and links no
+ * library kernel; the summation order differs from grinqh_prefill's, so the two
+ * agree within the tolerance, not bitwise.
+ *   X       device fp16 [T][K] row-major, 16-byte aligned; K a multiple of 8;
+ *           1 <= T <= 65535 * 256.
+ *   Y       device fp32 [T][N] row-major, output (overwritten), 4-byte aligned.
+ *   status  device, 16 bytes, 16-byte aligned, zero-filled before first use;
+ *           bit 0 of its first word is set if a wait inside the kernel gave up
+ *           after about a second (Y is then invalid); no call clears it.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (K not a multiple of 8, T above the
+ * limit), CUDA.
+ */
+grinqh_status grinqh_prefill_tc(const grinqh_layout* layout, const void* packed, const uint16_t* X, int32_t T,
+                                float* Y, uint32_t* status, void* stream);
+
+/*
  * Nested look-up-table codes. Paper: Section 3.3 ("Storage Layout and Weight
  * Loading": the planes need a nested quantisation, met by uniform codes and by
  * k-means codes such as any-precision LLM's; with such tables no midpoint term

@@ -44,10 +44,21 @@ def test_config0_vectors(g, orc):
         _select_compare(g, orc, v, th, CL)
 
 
-@pytest.mark.parametrize("K", [1, 2, 7, 1023, 1024, 1025, 4096, 4099, 14336, 65537])
+@pytest.mark.parametrize("K", [1, 2, 7, 1023, 1024, 1025, 4096, 4099, 14336, 65535, 65536])
 def test_sizes(g, orc, K):
     x = wl.activations_student_t(K, 1, key=(21, K))[0]
     _select_compare(g, orc, x, [0.2, 0.6, 1.1, 2.5], CL)
+
+
+def test_above_max_k_is_refused(g):
+    # every 1024-channel block reads all of x: above 65536 channels the call is
+    # refused before any launch, and the outputs are left untouched
+    K = 65537
+    x = torch.zeros(K, dtype=torch.int16, device="cuda")
+    th = torch.tensor([0.2, 0.6, 1.1, 2.5], dtype=torch.float32, device="cuda")
+    with pytest.raises(g.GrinqhError) as e:
+        g.select(x, th, CL)
+    assert e.value.code == 3
 
 
 @pytest.mark.parametrize("classes,theta", [
