@@ -17,10 +17,17 @@
 //   warp 1      allocates 256 TMEM columns and, from one lane, issues the four
 //               kind::f16 MMAs (K = 16 each) of a stage once both operand tiles
 //               are full, then commits to the stage's "empty" barrier;
-//   warps 2..5  rebuild the stage's 64 x 128 weight tile: 4 lanes per row, each
-//               lane the 32 columns of one record word, written as binary16 in the
-//               MN-major 128-byte-swizzled layout the A descriptor names; then,
-//               after the last stage, the epilogue (TMEM -> registers -> Y).
+//   warps 2..9  rebuild the stage's 64 x 128 weight tile, 8 rows per warp: 4 lanes
+//               per row, each lane the 32 columns of one record word, written as
+//               binary16 in the MN-major 128-byte-swizzled layout the A descriptor
+//               names; a lane loads a stage's words three stages before it fills
+//               it. Codes become binary16 without an integer
+//               conversion: a byte-permute puts code c under the exponent of 1024
+//               (0x6400 | c = 1024 + c, exact), a paired subtract of 1024 + z gives
+//               c - z exactly, and a paired multiply by s rounds s (c - z) once to
+//               binary16, the value grinqh_dequant writes. After the last stage the
+//               same warps read the accumulators (TMEM -> registers -> Y), two warps
+//               per TMEM lane quarter, each half of the 256 token columns.
 // Every wait on an mbarrier is bounded by the global timer (about one second);
 // a wait that gives up sets bit 0 of the status word and the CTA skips the rest
 // of its work, frees its tensor memory and returns.
@@ -43,11 +50,13 @@ constexpr int kPK = 64;                        // k rows per stage (four MMAs of
 constexpr int kPStages = 4;
 constexpr int kPABytes = kPM * kPK * 2;        // 16 KB of binary16 weights per stage
 constexpr int kPBBytes = kPN * kPK * 2;        // 32 KB of binary16 activations per stage
-constexpr int kPThreads = 192;
+constexpr int kPRebuildWarps = 8;           // 8 k rows of a stage each
+constexpr int kPAhead = 3;                  // stages a rebuild lane loads ahead
+constexpr int kPThreads = 32 * (2 + kPRebuildWarps);
 constexpr unsigned long long kPWaitNs = 1000000000ull;   // bound of one wait
 
 struct PfSync {
-  unsigned long long full_a[kPStages];   // 4 arrivals: the rebuild warps
+  unsigned long long full_a[kPStages];   // one arrival per rebuild warp
   unsigned long long full_b[kPStages];   // 1 arrival + the TMA's bytes
   unsigned long long empty[kPStages];    // the MMAs that read the stage have completed
   unsigned long long accum;              // every MMA of the CTA has completed
@@ -130,33 +139,49 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 __device__ __forceinline__ void tc_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// The binary16 weights of one (row, 32-column record word): fp16_rne(s (q - z))
-// for the lane's 32 columns, as 16 words of two values (columns 2i, 2i+1).
+// One lane's words of one (row, tile) record: its two words of each plane pair
+// and its group's scale | zero word.
+struct PfWords {
+  uint32_t p[8];
+  uint32_t m;
+};
+
 template <int kBmax>
-__device__ __forceinline__ void rebuild_word(const uint8_t* __restrict__ planes, const uint8_t* __restrict__ meta,
-                                             int w, uint32_t (&h)[16]) {
-  uint32_t P[8];
+__device__ __forceinline__ void load_words(const uint8_t* __restrict__ planes, const uint8_t* __restrict__ meta, int w,
+                                           PfWords& v) {
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
     if (2 * s < kBmax) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(planes + s * kPairBytes) + w);
-      P[2 * s] = v.x;
-      P[2 * s + 1] = v.y;
+      const uint2 u = __ldg(reinterpret_cast<const uint2*>(planes + s * kPairBytes) + w);
+      v.p[2 * s] = u.x;
+      v.p[2 * s + 1] = u.y;
     } else {
-      P[2 * s] = P[2 * s + 1] = 0u;
+      v.p[2 * s] = v.p[2 * s + 1] = 0u;
     }
   }
-  const uint32_t m = __ldg(reinterpret_cast<const uint32_t*>(meta) + (w >> 2));
-  const float sc = half_bits_to_float(m), z = half_bits_to_float(m >> 16);
+  v.m = __ldg(reinterpret_cast<const uint32_t*>(meta) + (w >> 2));
+}
+
+// The binary16 weights of the lane's 32 columns, fp16_rne(s (q - z)), as 16 words
+// of two values (columns 2i, 2i+1).
+template <int kBmax>
+__device__ __forceinline__ void rebuild_half2(const PfWords& v, uint32_t (&h)[16]) {
   uint32_t R[8];
-  assemble<kBmax>(P, R);   // byte i of R[j]: the code of column 4j+i in the 8-bit frame
+  assemble<kBmax>(v.p, R);   // byte i of R[j]: the code of column 4j+i in the 8-bit frame
+  // {s, s} and {1024 + z, 1024 + z} as binary16 pairs (z is an integer <= 255)
+  const uint32_t s2 = (v.m & 0xFFFFu) * 0x10001u;
+  __half2 z2 = __halves2half2(__ushort_as_half((unsigned short)(v.m >> 16)), __ushort_as_half((unsigned short)(v.m >> 16)));
+  z2 = __hadd2(z2, __halves2half2(__ushort_as_half((unsigned short)0x6400u), __ushort_as_half((unsigned short)0x6400u)));
+  const __half2 sh = *reinterpret_cast<const __half2*>(&s2);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint32_t q = R[j] >> (8 - kBmax);   // b_max-bit codes, one per byte
-    const __half2 lo = __floats2half2_rn(sc * ((float)(q & 0xFFu) - z), sc * ((float)((q >> 8) & 0xFFu) - z));
-    const __half2 hi = __floats2half2_rn(sc * ((float)((q >> 16) & 0xFFu) - z), sc * ((float)(q >> 24) - z));
-    h[2 * j] = *reinterpret_cast<const uint32_t*>(&lo);
-    h[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&hi);
+    const uint32_t lo = __byte_perm(q, 0x64646464u, 0x5140u);   // {1024 + c0, 1024 + c1}
+    const uint32_t hi = __byte_perm(q, 0x64646464u, 0x7362u);   // {1024 + c2, 1024 + c3}
+    const __half2 a = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&lo), z2), sh);
+    const __half2 b = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&hi), z2), sh);
+    h[2 * j] = *reinterpret_cast<const uint32_t*>(&a);
+    h[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&b);
   }
 }
 
@@ -175,7 +200,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPStages; ++i) {
-      bar_init(saddr(&sy.full_a[i]), 4);
+      bar_init(saddr(&sy.full_a[i]), kPRebuildWarps);
       bar_init(saddr(&sy.full_b[i]), 1);
       bar_init(saddr(&sy.empty[i]), 1);
     }
@@ -235,33 +260,47 @@ __global__ void __launch_bounds__(kPThreads, 1)
     __syncwarp();
   } else {
     // ---------------- weight rebuild ----------------
-    // warp d = warp - 2 rebuilds k rows 16 d .. 16 d + 15 of a stage, 8 rows per
-    // pass, lane = 4 (row in pass) + q; lane quarter q owns columns 32 q .. 32 q + 31
-    // of the CTA's 128, record word w = 4 (128-column slice of the tile) + q
+    // warp d = warp - 2 rebuilds k rows 8 d .. 8 d + 7 of a stage: lane = 4 (row)
+    // + q; lane quarter q owns columns 32 q .. 32 q + 31 of the CTA's 128, record
+    // word w = 4 (128-column slice of the tile) + q
     const int d = warp - 2, q = lane & 3;
     const int t_rec = n0 / kTileN, w = 4 * ((n0 % kTileN) / kPM) + q;
     const size_t rbytes = (size_t)record_bytes_for(kBmax);
-    for (int it = 0; it < n_k && ok; ++it) {
-      const int st = it % kPStages;
-      ok = bar_wait(saddr(&sy.empty[st]), ((uint32_t)(it / kPStages) & 1u) ^ 1u);
-      if (!ok) break;
+    const int kl = 8 * d + (lane >> 2);   // this lane's k row within a stage
+    // element (column c of the lane's 32, row kl): atom (kl / 8, q / 2) at
+    // (2 (kl / 8) + q / 2) KB, row kl % 8 at 128 bytes each, 16-byte chunk
+    // 4 (q % 2) + c / 8 stored at chunk index (chunk ^ (kl % 8))
+    const uint32_t r8 = (uint32_t)(kl & 7);
+    const uint32_t row_off = (uint32_t)((2 * (kl >> 3) + (q >> 1)) * 1024) + r8 * 128u;
+    auto load_stage = [&](int it, PfWords& v) {
+      const int k = it * kPK + kl;
+      if (k < K) {
+        const size_t rec = (size_t)k * n_tiles + t_rec;
+        load_words<kBmax>(packed + rec * rbytes, packed + meta_offset + rec * kMetaBytes, w, v);
+      } else {
 #pragma unroll
-      for (int pass = 0; pass < 2; ++pass) {
-        const int kl = 16 * d + 8 * pass + (lane >> 2);
-        const int k = it * kPK + kl;
+        for (int j = 0; j < 8; ++j) v.p[j] = 0u;
+        v.m = 0u;   // scale 0: the row's weights are +0
+      }
+    };
+    // stage it's words sit in buf[it % kPAhead], loaded kPAhead stages before they
+    // are needed (the loop is unrolled by kPAhead so the buffers stay in registers)
+    PfWords buf[kPAhead];
+#pragma unroll
+    for (int u = 0; u < kPAhead; ++u)
+      if (u < n_k) load_stage(u, buf[u]);
+    for (int i0 = 0; i0 < n_k && ok; i0 += kPAhead) {
+#pragma unroll
+      for (int u = 0; u < kPAhead; ++u) {
+        const int it = i0 + u;
+        if (it >= n_k || !ok) break;
+        const int st = it % kPStages;
+        ok = bar_wait(saddr(&sy.empty[st]), ((uint32_t)(it / kPStages) & 1u) ^ 1u);
+        if (!ok) break;
         uint32_t h[16];
-        if (k < K) {
-          const size_t rec = (size_t)k * n_tiles + t_rec;
-          rebuild_word<kBmax>(packed + rec * rbytes, packed + meta_offset + rec * kMetaBytes, w, h);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) h[j] = 0u;
-        }
-        // element (column c of the lane's 32, row kl): atom (kl / 8, q / 2) at
-        // (2 (kl / 8) + q / 2) KB, row kl % 8 at 128 bytes each, 16-byte chunk
-        // 4 (q % 2) + c / 8 stored at chunk index (chunk ^ (kl % 8))
-        const uint32_t r8 = (uint32_t)(kl & 7);
-        const uint32_t row = a0 + st * kPABytes + (uint32_t)((2 * (kl >> 3) + (q >> 1)) * 1024) + r8 * 128u;
+        rebuild_half2<kBmax>(buf[u], h);
+        if (it + kPAhead < n_k) load_stage(it + kPAhead, buf[u]);
+        const uint32_t row = a0 + st * kPABytes + row_off;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           const uint32_t chunk = ((uint32_t)(4 * (q & 1) + cc)) ^ r8;
@@ -269,11 +308,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
                        "r"(h[4 * cc + 1]), "r"(h[4 * cc + 2]), "r"(h[4 * cc + 3])
                        : "memory");
         }
+        // the tensor core reads the tile through the async proxy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) bar_arrive(saddr(&sy.full_a[st]));
       }
-      // the tensor core reads the tile through the async proxy
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) bar_arrive(saddr(&sy.full_a[st]));
     }
     // ---------------- epilogue ----------------
     // TMEM lane i of quarter (warp % 4) holds output column n0 + 32 (warp % 4) + i;
@@ -283,8 +322,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (ok) {
       const int qq = warp & 3;
       const int n = n0 + 32 * qq + lane;
+      const int c0 = (d >= 4) ? kPN / 64 : 0;   // warps 6..9 take token columns 128..255
 #pragma unroll 1
-      for (int cc = 0; cc < kPN / 32; ++cc) {
+      for (int cc = c0; cc < c0 + kPN / 64; ++cc) {
         if (t0 + 32 * cc >= T) break;
         uint32_t v[32];
         const uint32_t taddr = tmem + ((uint32_t)(32 * qq) << 16) + (uint32_t)(32 * cc);
