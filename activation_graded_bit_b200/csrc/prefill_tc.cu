@@ -10,13 +10,15 @@
 // fp16_rne(s * (q - z)) per (row k, 128-column group), q the b_max-bit code.
 //
 // One CTA computes a tile of 128 output columns (the MMA's M, from W_hat) by 256
-// tokens (the MMA's N, from X) with fp32 accumulators in tensor memory, looping
-// over K in stages of 64 rows held in a 4-deep shared-memory ring:
-//   warp 0      X tiles by TMA (no multicast): 256 tokens x 64 k, K-major,
+// tokens (the MMA's N, from X), or by 512 tokens as two 256-token halves that share
+// each rebuilt weight tile (when the grid of such CTAs takes fewer waves), with fp32
+// accumulators in tensor memory (256 or 512 columns), looping over K in stages of
+// 64 rows held in a 4-deep (256 tokens) or 2-deep (512 tokens) shared-memory ring:
+//   warp 0      X tiles by TMA (no multicast): 256 tokens x 64 k per half, K-major,
 //               128-byte swizzle, one mbarrier transaction per stage;
-//   warp 1      allocates 256 TMEM columns and, from one lane, issues the four
-//               kind::f16 MMAs (K = 16 each) of a stage once both operand tiles
-//               are full, then commits to the stage's "empty" barrier;
+//   warp 1      allocates the TMEM columns and, from one lane, issues the four
+//               kind::f16 MMAs (K = 16 each) of a stage per token half once both
+//               operand tiles are full, then commits to the stage's "empty" barrier;
 //   warps 2..9  rebuild the stage's 64 x 128 weight tile, 8 rows per warp: 4 lanes
 //               per row, each lane the 32 columns of one record word, written as
 //               binary16 in the MN-major 128-byte-swizzled layout the A descriptor
@@ -27,7 +29,7 @@
 //               c - z exactly, and a paired multiply by s rounds s (c - z) once to
 //               binary16, the value grinqh_dequant writes. After the last stage the
 //               same warps read the accumulators (TMEM -> registers -> Y), two warps
-//               per TMEM lane quarter, each half of the 256 token columns.
+//               per TMEM lane quarter, each half of the token columns.
 // Every wait on an mbarrier is bounded by the global timer (about one second);
 // a wait that gives up sets bit 0 of the status word and the CTA skips the rest
 // of its work, frees its tensor memory and returns.
@@ -64,7 +66,15 @@ struct PfSync {
   uint32_t failed;                       // some wait of this CTA gave up
 };
 
-constexpr size_t kPSmem = 1024 + (size_t)kPStages * (kPABytes + kPBBytes) + sizeof(PfSync);
+// Stages and shared memory of a CTA with kHalves token halves of 256.
+template <int kHalves>
+struct PfGeom {
+  static constexpr int kStages = kHalves == 1 ? 4 : 2;
+  static constexpr int kBStage = kHalves * kPBBytes;
+  static constexpr int kTokens = kHalves * kPN;
+  static constexpr size_t kSmem = 1024 + (size_t)kStages * (kPABytes + kBStage) + sizeof(PfSync);
+};
+static_assert(PfGeom<1>::kSmem <= 227 * 1024 && PfGeom<2>::kSmem <= 227 * 1024, "prefill shared memory");
 
 __device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -185,21 +195,23 @@ __device__ __forceinline__ void rebuild_half2(const PfWords& v, uint32_t (&h)[16
   }
 }
 
-template <int kBmax>
+template <int kBmax, int kHalves>
 __global__ void __launch_bounds__(kPThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint8_t* __restrict__ packed, size_t meta_offset,
                       int T, int K, int N, int n_tiles, float* __restrict__ Y, uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) uint8_t pf_smem[];
   const uint32_t raw = saddr(pf_smem);
+  using G = PfGeom<kHalves>;
+  constexpr int kSt = G::kStages;
   const uint32_t a0 = (raw + 1023u) & ~1023u;   // 1 KB-aligned operand ring (swizzle atoms)
-  const uint32_t b0 = a0 + kPStages * kPABytes;
-  PfSync& sy = *reinterpret_cast<PfSync*>(pf_smem + (a0 - raw) + kPStages * (kPABytes + kPBBytes));
+  const uint32_t b0 = a0 + kSt * kPABytes;
+  PfSync& sy = *reinterpret_cast<PfSync*>(pf_smem + (a0 - raw) + kSt * (kPABytes + G::kBStage));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kPM, t0 = blockIdx.y * kPN;
+  const int n0 = blockIdx.x * kPM, t0 = blockIdx.y * G::kTokens;
   const int n_k = (K + kPK - 1) / kPK;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kPStages; ++i) {
+    for (int i = 0; i < kSt; ++i) {
       bar_init(saddr(&sy.full_a[i]), kPRebuildWarps);
       bar_init(saddr(&sy.full_b[i]), 1);
       bar_init(saddr(&sy.empty[i]), 1);
@@ -210,7 +222,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(&sy.tmem)),
-                 "r"(kPN)
+                 "r"(G::kTokens)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -224,23 +236,25 @@ __global__ void __launch_bounds__(kPThreads, 1)
     // ---------------- activations: one TMA per stage ----------------
     int issued = -1;
     for (int it = 0; it < n_k && ok; ++it) {
-      const int st = it % kPStages;
-      ok = bar_wait(saddr(&sy.empty[st]), ((uint32_t)(it / kPStages) & 1u) ^ 1u);
+      const int st = it % kSt;
+      ok = bar_wait(saddr(&sy.empty[st]), ((uint32_t)(it / kSt) & 1u) ^ 1u);
       if (ok && lane == 0) {
-        bar_expect(saddr(&sy.full_b[st]), kPBBytes);
-        tma_x(b0 + st * kPBBytes, &xmap, it * kPK, t0, saddr(&sy.full_b[st]));
+        bar_expect(saddr(&sy.full_b[st]), G::kBStage);
+#pragma unroll
+        for (int hh = 0; hh < kHalves; ++hh)   // token rows past T arrive as zeros
+          tma_x(b0 + st * G::kBStage + hh * kPBBytes, &xmap, it * kPK, t0 + hh * kPN, saddr(&sy.full_b[st]));
       }
       if (ok) issued = it;
       __syncwarp();
     }
     // the CTA's last copies have landed before anything here can end
-    for (int it = (issued - kPStages + 1 > 0 ? issued - kPStages + 1 : 0); it <= issued; ++it)
-      bar_wait(saddr(&sy.full_b[it % kPStages]), (uint32_t)(it / kPStages) & 1u);
+    for (int it = (issued - kSt + 1 > 0 ? issued - kSt + 1 : 0); it <= issued; ++it)
+      bar_wait(saddr(&sy.full_b[it % kSt]), (uint32_t)(it / kSt) & 1u);
   } else if (warp == 1) {
     // ---------------- MMA issue ----------------
     for (int it = 0; it < n_k && ok; ++it) {
-      const int st = it % kPStages;
-      const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
+      const int st = it % kSt;
+      const uint32_t ph = (uint32_t)(it / kSt) & 1u;
       ok = bar_wait(saddr(&sy.full_a[st]), ph) && bar_wait(saddr(&sy.full_b[st]), ph);
       tc_after();
       if (ok && lane == 0) {
@@ -248,9 +262,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
         for (int kk = 0; kk < kPK / 16; ++kk) {
           // A: MN-major; 64-column atoms 1 KB apart along M, 8-row groups 2 KB apart along K
           const uint64_t ad = smem_desc(a0 + st * kPABytes + kk * 4096, 1024, 2048);
-          // B: K-major rows of 128 bytes, 8-row groups 1 KB apart; K = 16 is 32 bytes into the row
-          const uint64_t bd = smem_desc(b0 + st * kPBBytes + kk * 32, 16, 1024);
-          mma_f16(tmem, ad, bd, (it > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int hh = 0; hh < kHalves; ++hh) {
+            // B: K-major rows of 128 bytes, 8-row groups 1 KB apart; K = 16 is 32 bytes into the row
+            const uint64_t bd = smem_desc(b0 + st * G::kBStage + hh * kPBBytes + kk * 32, 16, 1024);
+            mma_f16(tmem + (uint32_t)(hh * kPN), ad, bd, (it > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         mma_commit(saddr(&sy.empty[st]));
       }
@@ -294,8 +311,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
       for (int u = 0; u < kPAhead; ++u) {
         const int it = i0 + u;
         if (it >= n_k || !ok) break;
-        const int st = it % kPStages;
-        ok = bar_wait(saddr(&sy.empty[st]), ((uint32_t)(it / kPStages) & 1u) ^ 1u);
+        const int st = it % kSt;
+        ok = bar_wait(saddr(&sy.empty[st]), ((uint32_t)(it / kSt) & 1u) ^ 1u);
         if (!ok) break;
         uint32_t h[16];
         rebuild_half2<kBmax>(buf[u], h);
@@ -322,9 +339,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (ok) {
       const int qq = warp & 3;
       const int n = n0 + 32 * qq + lane;
-      const int c0 = (d >= 4) ? kPN / 64 : 0;   // warps 6..9 take token columns 128..255
+      constexpr int kChunks = G::kTokens / 64;   // 32-column chunks per warp: half the token columns
+      const int c0 = (d >= 4) ? kChunks : 0;      // warps 6..9 take the second half
 #pragma unroll 1
-      for (int cc = c0; cc < c0 + kPN / 64; ++cc) {
+      for (int cc = c0; cc < c0 + kChunks; ++cc) {
         if (t0 + 32 * cc >= T) break;
         uint32_t v[32];
         const uint32_t taddr = tmem + ((uint32_t)(32 * qq) << 16) + (uint32_t)(32 * cc);
@@ -354,13 +372,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
   if (threadIdx.x == 0 && sy.failed) atomicOr(status, 1u);
   if (warp == 1) {
     tc_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPN) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(G::kTokens) : "memory");
   }
 }
 
 }  // namespace
 
-size_t prefill_tc_smem_bytes() { return kPSmem; }
+size_t prefill_tc_smem_bytes() { return PfGeom<1>::kSmem; }
 
 cudaError_t launch_prefill_tc(const uint16_t* X, const void* packed, int T, int K, int N, int n_tiles, int b_max,
                               float* Y, uint32_t* status, cudaStream_t st) {
@@ -383,14 +401,32 @@ cudaError_t launch_prefill_tc(const uint16_t* X, const void* packed, int T, int 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   const size_t meta_offset = meta_offset_for(K, n_tiles, b_max);
-  const dim3 grid((unsigned)((N + kPM - 1) / kPM), (unsigned)((T + kPN - 1) / kPN));
+  // 512-token CTAs (each weight tile rebuilt once per 512 tokens) where they take
+  // less time than 256-token CTAs: a wide CTA takes about 1.6x a narrow one (its MMA
+  // work doubles, its rebuild does not), so compare waves x per-CTA time on this GPU
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms < 1) sms = 1;
+  const long long cols = (N + kPM - 1) / kPM;
+  const long long waves_n = (cols * ((T + kPN - 1) / kPN) + sms - 1) / sms;
+  const long long waves_w = (cols * ((T + 2 * kPN - 1) / (2 * kPN)) + sms - 1) / sms;
+  const bool wide = T > kPN && 16 * waves_w < 10 * waves_n;
+  const int tokens = wide ? PfGeom<2>::kTokens : PfGeom<1>::kTokens;
+  const dim3 grid((unsigned)((N + kPM - 1) / kPM), (unsigned)((T + tokens - 1) / tokens));
   cudaError_t e;
-#define GRINQH_PF_CASE(B)                                                                                      \
-  case B:                                                                                                      \
-    e = cudaFuncSetAttribute(prefill_tc_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmem); \
-    if (e != cudaSuccess) return e;                                                                            \
-    prefill_tc_kernel<B><<<grid, kPThreads, kPSmem, st>>>(map, (const uint8_t*)packed, meta_offset, T, K, N,   \
-                                                          n_tiles, Y, status);                                 \
+#define GRINQH_PF_LAUNCH(B, H)                                                                                  \
+  e = cudaFuncSetAttribute(prefill_tc_kernel<B, H>, cudaFuncAttributeMaxDynamicSharedMemorySize,                \
+                           (int)PfGeom<H>::kSmem);                                                              \
+  if (e != cudaSuccess) return e;                                                                               \
+  prefill_tc_kernel<B, H><<<grid, kPThreads, PfGeom<H>::kSmem, st>>>(map, (const uint8_t*)packed, meta_offset, T, \
+                                                                       K, N, n_tiles, Y, status);
+#define GRINQH_PF_CASE(B)            \
+  case B:                            \
+    if (wide) {                      \
+      GRINQH_PF_LAUNCH(B, 2)         \
+    } else {                         \
+      GRINQH_PF_LAUNCH(B, 1)         \
+    }                                \
     break;
   switch (b_max) {
     GRINQH_PF_CASE(2)
@@ -400,6 +436,7 @@ cudaError_t launch_prefill_tc(const uint16_t* X, const void* packed, int T, int 
     default: return cudaErrorInvalidValue;
   }
 #undef GRINQH_PF_CASE
+#undef GRINQH_PF_LAUNCH
   return cudaGetLastError();
 }
 

@@ -3,8 +3,9 @@ fp64 oracle ("GRINQH" Section 4: prefill takes every weight at full b_max precis
 and runs a dense product): within |y - y_ref| <= 1e-4 * sum_k |x_k w16_kn| + 1e-6 of
 the fp64 product over the same binary16 operands (w16 = fp16_rne(s (q - z)), the
 operands grinqh_dequant writes). Shapes cover several 64-row stages with a ragged
-last stage, partial 128-column and 256-token tiles, every b_max, and more than one
-CTA along the token axis; the status word stays zero."""
+last stage, partial 128-column and 256-token tiles, every b_max, more than one CTA
+along the token axis, and the 512-token tiles taken from 1024 tokens on; the status
+word stays zero."""
 import numpy as np
 import pytest
 import torch
@@ -55,6 +56,18 @@ def test_prefill_tc_several_token_tiles(g, orc):
     rng = np.random.default_rng(7)
     toks = list(rng.choice(T, 10, replace=False)) + [0, 255, 256, T - 1]
     _run(g, orc, 2048, 2048, T, 8, (112,), tokens=toks)
+
+
+@pytest.mark.parametrize("bmax", (8, 4))
+def test_prefill_tc_512_token_tiles(g, orc, bmax):
+    # a CTA takes 512 tokens as two 256-token halves sharing the rebuilt weight tile
+    # when that grid needs fewer waves: 4096 columns x 1200 tokens is 160 narrow CTAs
+    # (two waves on 148 SMs) or 96 wide ones (one wave). Three wide CTAs along the token
+    # axis, the last with a partial first half and an empty second half; sampled
+    # tokens around the half and tile edges
+    T = 1200
+    toks = [0, 1, 255, 256, 300, 511, 512, 767, 768, 1023, 1024, 1050, 1151, T - 1]
+    _run(g, orc, 136, 4096, T, bmax, (114, bmax), tokens=toks)
 
 
 def test_prefill_tc_agrees_with_dequant_gemm(g, orc):
