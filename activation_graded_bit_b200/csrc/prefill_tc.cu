@@ -195,7 +195,7 @@ __device__ __forceinline__ void rebuild_half2(const PfWords& v, uint32_t (&h)[16
   }
 }
 
-template <int kBmax, int kHalves>
+template <int kBmax, int kHalves, int kSplit>
 __global__ void __launch_bounds__(kPThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap xmap, const uint8_t* __restrict__ packed, size_t meta_offset,
                       int T, int K, int N, int n_tiles, float* __restrict__ Y, uint32_t* __restrict__ status) {
@@ -208,7 +208,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
   PfSync& sy = *reinterpret_cast<PfSync*>(pf_smem + (a0 - raw) + kSt * (kPABytes + G::kBStage));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kPM, t0 = blockIdx.y * G::kTokens;
-  const int n_k = (K + kPK - 1) / kPK;
+  // with kSplit > 1 the CTAs of a cluster (along z) take consecutive ranges of the
+  // K stages and add their accumulators through distributed shared memory
+  const int n_k_all = (K + kPK - 1) / kPK;
+  const int rank = (kSplit > 1) ? (int)blockIdx.z : 0;
+  const int ks0 = (int)(((long long)n_k_all * rank) / kSplit);
+  const int n_k = (int)(((long long)n_k_all * (rank + 1)) / kSplit) - ks0;   // this CTA's stages (>= 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSt; ++i) {
@@ -242,7 +247,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         bar_expect(saddr(&sy.full_b[st]), G::kBStage);
 #pragma unroll
         for (int hh = 0; hh < kHalves; ++hh)   // token rows past T arrive as zeros
-          tma_x(b0 + st * G::kBStage + hh * kPBBytes, &xmap, it * kPK, t0 + hh * kPN, saddr(&sy.full_b[st]));
+          tma_x(b0 + st * G::kBStage + hh * kPBBytes, &xmap, (ks0 + it) * kPK, t0 + hh * kPN, saddr(&sy.full_b[st]));
       }
       if (ok) issued = it;
       __syncwarp();
@@ -290,7 +295,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const uint32_t r8 = (uint32_t)(kl & 7);
     const uint32_t row_off = (uint32_t)((2 * (kl >> 3) + (q >> 1)) * 1024) + r8 * 128u;
     auto load_stage = [&](int it, PfWords& v) {
-      const int k = it * kPK + kl;
+      const int k = (ks0 + it) * kPK + kl;
       if (k < K) {
         const size_t rec = (size_t)k * n_tiles + t_rec;
         load_words<kBmax>(packed + rec * rbytes, packed + meta_offset + rec * kMetaBytes, w, v);
@@ -333,7 +338,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
     // ---------------- epilogue ----------------
     // TMEM lane i of quarter (warp % 4) holds output column n0 + 32 (warp % 4) + i;
-    // TMEM column j holds token t0 + j
+    // TMEM column j holds token t0 + j. Without a K split the warps store Y; with
+    // one they store the accumulators to shared memory as D[token][column] (the
+    // operand ring is free once every MMA has completed) for the cluster sum below.
     if (ok) ok = bar_wait(saddr(&sy.accum), 0u);
     tc_after();
     if (ok) {
@@ -341,9 +348,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const int n = n0 + 32 * qq + lane;
       constexpr int kChunks = G::kTokens / 64;   // 32-column chunks per warp: half the token columns
       const int c0 = (d >= 4) ? kChunks : 0;      // warps 6..9 take the second half
+      float* dump = reinterpret_cast<float*>(pf_smem + (a0 - raw));
 #pragma unroll 1
       for (int cc = c0; cc < c0 + kChunks; ++cc) {
-        if (t0 + 32 * cc >= T) break;
+        if (kSplit == 1 && t0 + 32 * cc >= T) break;
         uint32_t v[32];
         const uint32_t taddr = tmem + ((uint32_t)(32 * qq) << 16) + (uint32_t)(32 * cc);
         asm volatile(
@@ -356,15 +364,44 @@ __global__ void __launch_bounds__(kPThreads, 1)
               "=r"(v[30]), "=r"(v[31])
             : "r"(taddr));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        if (n < N) {
+        if (kSplit == 1) {
+          if (n < N) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int t = t0 + 32 * cc + i;
-            if (t < T) Y[(size_t)t * N + n] = __uint_as_float(v[i]);
+            for (int i = 0; i < 32; ++i) {
+              const int t = t0 + 32 * cc + i;
+              if (t < T) Y[(size_t)t * N + n] = __uint_as_float(v[i]);
+            }
           }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dump[(32 * cc + i) * kPM + 32 * qq + lane] = __uint_as_float(v[i]);
         }
       }
     }
+  }
+  if (kSplit > 1) {
+    // every thread of every CTA of the cluster takes part (no CTA leaves early):
+    // rank r adds tokens [r 256 / kSplit, (r + 1) 256 / kSplit) over the ranks'
+    // dumps in rank order and stores them to Y
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    const uint32_t dump0 = a0;
+    constexpr int kSlice = kPN / kSplit;
+    for (int e = threadIdx.x; e < kSlice * kPM; e += kPThreads) {
+      const int tl = rank * kSlice + e / kPM, c = e % kPM;
+      const uint32_t off = dump0 + (uint32_t)(tl * kPM + c) * 4u;
+      float v = 0.0f;
+#pragma unroll
+      for (int q = 0; q < kSplit; ++q) {
+        uint32_t ra;
+        float f;
+        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(off), "r"((uint32_t)q));
+        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(f) : "r"(ra) : "memory");
+        v += f;
+      }
+      const int t = t0 + tl, n = n0 + c;
+      if (t < T && n < N) Y[(size_t)t * N + n] = v;
+    }
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   }
   if (!ok) sy.failed = 1u;
   tc_before();
@@ -412,21 +449,45 @@ cudaError_t launch_prefill_tc(const uint16_t* X, const void* packed, int T, int 
   const long long waves_w = (cols * ((T + 2 * kPN - 1) / (2 * kPN)) + sms - 1) / sms;
   const bool wide = T > kPN && 16 * waves_w < 10 * waves_n;
   const int tokens = wide ? PfGeom<2>::kTokens : PfGeom<1>::kTokens;
-  const dim3 grid((unsigned)((N + kPM - 1) / kPM), (unsigned)((T + tokens - 1) / tokens));
+  // a K split over a cluster of 2 or 4 CTAs when the grid of 256-token CTAs is small
+  const long long grid_n = cols * ((T + kPN - 1) / kPN);
+  const int n_k_all = (K + kPK - 1) / kPK;
+  int split = 1;
+  if (!wide) {
+    if (4 * grid_n <= sms && n_k_all >= 4) split = 4;
+    else if (2 * grid_n <= sms && n_k_all >= 2) split = 2;
+  }
+  const dim3 grid((unsigned)cols, (unsigned)((T + tokens - 1) / tokens), (unsigned)split);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kPThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = (unsigned)split;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   cudaError_t e;
-#define GRINQH_PF_LAUNCH(B, H)                                                                                  \
-  e = cudaFuncSetAttribute(prefill_tc_kernel<B, H>, cudaFuncAttributeMaxDynamicSharedMemorySize,                \
-                           (int)PfGeom<H>::kSmem);                                                              \
-  if (e != cudaSuccess) return e;                                                                               \
-  prefill_tc_kernel<B, H><<<grid, kPThreads, PfGeom<H>::kSmem, st>>>(map, (const uint8_t*)packed, meta_offset, T, \
-                                                                       K, N, n_tiles, Y, status);
-#define GRINQH_PF_CASE(B)            \
-  case B:                            \
-    if (wide) {                      \
-      GRINQH_PF_LAUNCH(B, 2)         \
-    } else {                         \
-      GRINQH_PF_LAUNCH(B, 1)         \
-    }                                \
+#define GRINQH_PF_LAUNCH(B, H, S)                                                                            \
+  e = cudaFuncSetAttribute(prefill_tc_kernel<B, H, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,          \
+                           (int)PfGeom<H>::kSmem);                                                           \
+  if (e != cudaSuccess) return e;                                                                            \
+  cfg.dynamicSmemBytes = PfGeom<H>::kSmem;                                                                   \
+  e = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<B, H, S>, map, (const uint8_t*)packed, meta_offset, T, K, N, \
+                         n_tiles, Y, status);
+#define GRINQH_PF_CASE(B)                \
+  case B:                                \
+    if (wide) {                          \
+      GRINQH_PF_LAUNCH(B, 2, 1)          \
+    } else if (split == 4) {             \
+      GRINQH_PF_LAUNCH(B, 1, 4)          \
+    } else if (split == 2) {             \
+      GRINQH_PF_LAUNCH(B, 1, 2)          \
+    } else {                             \
+      GRINQH_PF_LAUNCH(B, 1, 1)          \
+    }                                    \
     break;
   switch (b_max) {
     GRINQH_PF_CASE(2)
@@ -437,6 +498,7 @@ cudaError_t launch_prefill_tc(const uint16_t* X, const void* packed, int T, int 
   }
 #undef GRINQH_PF_CASE
 #undef GRINQH_PF_LAUNCH
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

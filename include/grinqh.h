@@ -194,7 +194,8 @@ grinqh_status grinqh_prefill(const grinqh_layout* layout, const void* packed, co
  * accumulation) without writing W_hat to memory: each CTA rebuilds a 128-column
  * slice of W_hat from the bit planes into shared memory, 64 rows at a time, and
  * the 5th-generation tensor cores (tcgen05, sm_100a) multiply it with TMA-loaded
- * tiles of 256 tokens, accumulating in tensor memory. Paper: Section 4,
+ * tiles of 256 or 512 tokens (K split over a cluster of 2 or 4 CTAs when the
+ * grid is small), accumulating in tensor memory. Paper: Section 4,
  * "Prefill vs. Decoding Evaluation" (full b_max precision, dense product) and
  * Section 5 (unpacking fused with the product). Allocates nothing and links no
  * library kernel; the summation order differs from grinqh_prefill's, so the two
