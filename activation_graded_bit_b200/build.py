@@ -12,8 +12,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libgrinqh.so")
-SOURCES = ["api.cu", "pack.cu", "select.cu", "vmm.cu", "calibrate.cu", "prefill.cu", "prefill_tc.cu", "lut_build.cpp"]
-HEADERS = ["common.cuh", "kernels.h", "async.cuh"]
+SOURCES = ["api.cu", "pack.cu", "select.cu", "vmm.cu", "calibrate.cu", "prefill.cu", "prefill_tc.cu", "batch_tc.cu", "lut_build.cpp"]
+HEADERS = ["common.cuh", "kernels.h", "async.cuh", "tc_common.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC,-ffp-contract=off", "-Xptxas", "-v"]

@@ -390,6 +390,22 @@ grinqh_status grinqh_select_vmm_batch(const grinqh_layout* layout, const void* p
   return cuda_status(launch_vmm(a, (cudaStream_t)stream, true));
 }
 
+grinqh_status grinqh_select_vmm_batch_tc(const grinqh_layout* layout, const void* packed, const uint16_t* X,
+                                         int32_t tokens, const float* thresholds, const uint8_t* classes,
+                                         int32_t n_classes, float* Y, uint32_t* status, void* stream) {
+  if (!layout_ok(layout) || !valid_classes(classes, n_classes)) return GRINQH_ERR_INVALID_ARG;
+  if (!classes_fit(classes, n_classes, layout->b_max)) return GRINQH_ERR_INVALID_ARG;
+  if (tokens < 1 || tokens > kMaxTokens) return GRINQH_ERR_INVALID_ARG;
+  if (!packed || !X || !Y || !status || (n_classes > 1 && !thresholds)) return GRINQH_ERR_INVALID_ARG;
+  const grinqh_layout& L = *layout;
+  if (L.K % 8 != 0) return GRINQH_ERR_UNSUPPORTED;   // 16-byte loads of X rows
+  if (!aligned(packed, 16) || !aligned(X, 16) || !aligned(Y, 4) || !aligned(status, 16) ||
+      (thresholds && !aligned(thresholds, 4)))
+    return GRINQH_ERR_ALIGNMENT;
+  return cuda_status(launch_batch_tc(X, tokens, packed, L.K, L.N, L.n_tiles, L.b_max, thresholds,
+                                     table(classes, n_classes), Y, status, (cudaStream_t)stream));
+}
+
 grinqh_status grinqh_pack_codes(const grinqh_layout* layout, const uint8_t* codes, void* packed, void* stream) {
   if (!layout_ok(layout) || !codes || !packed) return GRINQH_ERR_INVALID_ARG;
   if (!aligned(packed, 16)) return GRINQH_ERR_ALIGNMENT;

@@ -41,6 +41,13 @@ struct ClassTable {
   uint8_t width[9];   // bit width of class j
 };
 
+// The batched graded product on the tensor cores (batch_tc.cu): X fp16 [T][K]
+// (K % 8 == 0, 16-byte aligned), Y fp32 [T][N]; *status bit 0: a bounded wait
+// gave up, bit 1: a value outside the binary16 range of the MMA operands.
+cudaError_t launch_batch_tc(const uint16_t* X, int T, const void* packed, int K, int N, int n_tiles, int b_max,
+                            const float* thresholds, const ClassTable& ct, float* Y, uint32_t* status,
+                            cudaStream_t st);
+
 // Largest K of launch_select: each 1024-channel block reads all of x to count
 // the channels ahead of it, K^2 / 512 bytes of L2 reads per call (8 MiB here).
 constexpr int kSelectMaxK = 1 << 16;

@@ -42,6 +42,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace grinqh {
 namespace {
@@ -55,7 +56,6 @@ constexpr int kPBBytes = kPN * kPK * 2;        // 32 KB of binary16 activations 
 constexpr int kPRebuildWarps = 8;           // 8 k rows of a stage each
 constexpr int kPAhead = 3;                  // stages a rebuild lane loads ahead
 constexpr int kPThreads = 32 * (2 + kPRebuildWarps);
-constexpr unsigned long long kPWaitNs = 1000000000ull;   // bound of one wait
 
 struct PfSync {
   unsigned long long full_a[kPStages];   // one arrival per rebuild warp
@@ -76,46 +76,6 @@ struct PfGeom {
 };
 static_assert(PfGeom<1>::kSmem <= 227 * 1024 && PfGeom<2>::kSmem <= 227 * 1024, "prefill shared memory");
 
-__device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ unsigned long long now_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void bar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void bar_expect(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool bar_test(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0u;
-}
-// Wait for the phase of parity `parity` to complete; false after about a second.
-__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
-  if (bar_test(bar, parity)) return true;
-  const unsigned long long t0 = now_ns();
-  for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (bar_test(bar, parity)) return true;
-    if (now_ns() - t0 > kPWaitNs) return false;
-  }
-}
-
 // 2-D tiled TMA load of box {64 k, 256 tokens} at (k0, t0) into shared memory.
 __device__ __forceinline__ void tma_x(uint32_t dst, const CUtensorMap* map, int k0, int t0, uint32_t bar) {
   asm volatile(
@@ -125,29 +85,9 @@ __device__ __forceinline__ void tma_x(uint32_t dst, const CUtensorMap* map, int 
       : "memory");
 }
 
-// Shared-memory matrix descriptor (tcgen05): start address, leading and stride
-// byte offsets in 16-byte units, descriptor version 1, 128-byte swizzle.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
 // Instruction descriptor of kind::f16: D fp32, A and B binary16, A (weights)
 // MN-major, B (activations) K-major, N = 256, M = 128.
 constexpr uint32_t kPIdesc = (1u << 4) | (1u << 15) | ((uint32_t)(kPN >> 3) << 17) | ((uint32_t)(kPM >> 4) << 24);
-
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(kPIdesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
 // One lane's words of one (row, tile) record: its two words of each plane pair
 // and its group's scale | zero word.
@@ -271,7 +211,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
           for (int hh = 0; hh < kHalves; ++hh) {
             // B: K-major rows of 128 bytes, 8-row groups 1 KB apart; K = 16 is 32 bytes into the row
             const uint64_t bd = smem_desc(b0 + st * G::kBStage + hh * kPBBytes + kk * 32, 16, 1024);
-            mma_f16(tmem + (uint32_t)(hh * kPN), ad, bd, (it > 0 || kk > 0) ? 1u : 0u);
+            mma_f16(tmem + (uint32_t)(hh * kPN), ad, bd, kPIdesc, (it > 0 || kk > 0) ? 1u : 0u);
           }
         }
         mma_commit(saddr(&sy.empty[st]));
@@ -383,7 +323,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     // every thread of every CTA of the cluster takes part (no CTA leaves early):
     // rank r adds tokens [r 256 / kSplit, (r + 1) 256 / kSplit) over the ranks'
     // dumps in rank order and stores them to Y
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    cluster_sync_all();
     const uint32_t dump0 = a0;
     constexpr int kSlice = kPN / kSplit;
     for (int e = threadIdx.x; e < kSlice * kPM; e += kPThreads) {
@@ -391,17 +331,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const uint32_t off = dump0 + (uint32_t)(tl * kPM + c) * 4u;
       float v = 0.0f;
 #pragma unroll
-      for (int q = 0; q < kSplit; ++q) {
-        uint32_t ra;
-        float f;
-        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(off), "r"((uint32_t)q));
-        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(f) : "r"(ra) : "memory");
-        v += f;
-      }
+      for (int q = 0; q < kSplit; ++q) v += ld_dsmem_f32(off, (uint32_t)q);
       const int t = t0 + tl, n = n0 + c;
       if (t < T && n < N) Y[(size_t)t * N + n] = v;
     }
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    cluster_sync_all();
   }
   if (!ok) sy.failed = 1u;
   tc_before();

@@ -72,6 +72,7 @@ _select_vmm_batch = _sig("grinqh_select_vmm_batch", [_LP, _P, _P, _I, _P, _P, _I
 _dequant = _sig("grinqh_dequant", [_LP, _P, _P, _P])
 _prefill = _sig("grinqh_prefill", [_LP, _P, _P, _I, _P, _P, _P])
 _prefill_tc = _sig("grinqh_prefill_tc", [_LP, _P, _P, _I, _P, _P, _P])
+_select_vmm_batch_tc = _sig("grinqh_select_vmm_batch_tc", [_LP, _P, _P, _I, _P, _P, _I, _P, _P, _P])
 _pack_codes = _sig("grinqh_pack_codes", [_LP, _P, _P, _P])
 _lut_build = _sig("grinqh_lut_build", [_P, _I, _I, _I, _P, _P])
 _lut_bytes = _sig("grinqh_lut_bytes", [_LP, ctypes.POINTER(ctypes.c_size_t)])
@@ -82,7 +83,7 @@ EXPORTS = ("grinqh_version", "grinqh_status_string", "grinqh_layout_init", "grin
            "grinqh_unpack_codes", "grinqh_maxent_distribution", "grinqh_calibrate_workspace_bytes",
            "grinqh_calibrate", "grinqh_select", "grinqh_vmm_workspace_bytes", "grinqh_vmm",
            "grinqh_vmm_noalloc", "grinqh_select_vmm", "grinqh_vmm_batch_workspace_bytes",
-           "grinqh_select_vmm_batch", "grinqh_dequant", "grinqh_prefill", "grinqh_prefill_tc", "grinqh_pack_codes",
+           "grinqh_select_vmm_batch", "grinqh_dequant", "grinqh_prefill", "grinqh_prefill_tc", "grinqh_select_vmm_batch_tc", "grinqh_pack_codes",
            "grinqh_lut_bytes", "grinqh_vmm_lut", "grinqh_lut_build")
 
 
@@ -327,6 +328,26 @@ def select_vmm_batch(p: PackedLayer, X: torch.Tensor, thresholds: Optional[torch
                              ctypes.addressof(cb), n, _ptr(Y), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)),
            "grinqh_select_vmm_batch")
+    return Y
+
+
+def select_vmm_batch_tc(p: PackedLayer, X: torch.Tensor, thresholds: Optional[torch.Tensor],
+                        classes: Sequence[int], status: torch.Tensor, Y: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """grinqh_select_vmm_batch_tc: the batched graded product on the tensor cores; X is a
+    contiguous [T, K] CUDA tensor of fp16 (or its bit view), status a zero-filled
+    16-byte CUDA tensor; returns Y fp32 [T, N]."""
+    assert X.is_cuda and X.dim() == 2 and X.is_contiguous() and X.element_size() == 2 and X.shape[1] == p.K
+    T = X.shape[0]
+    if Y is None:
+        Y = torch.empty((T, p.N), dtype=torch.float32, device=X.device)
+    cb, n = _classes_buf(classes)
+    _need(Y, T * p.N, 4, "grinqh_select_vmm_batch_tc Y")
+    _need(thresholds, n - 1, 4, "grinqh_select_vmm_batch_tc thresholds")
+    _need(status, 4, 4, "grinqh_select_vmm_batch_tc status")
+    _check(_select_vmm_batch_tc(ctypes.byref(p.layout), _ptr(p.packed), _ptr(X), T, _ptr(thresholds),
+                                ctypes.addressof(cb), n, _ptr(Y), _ptr(status), _stream(stream)),
+           "grinqh_select_vmm_batch_tc")
     return Y
 
 

@@ -832,10 +832,12 @@ def run_stack(args):
                                         "gpu_launches_per_token": len(grp) + sum(1 for d in grp if d["ws"].numel() > 16)}}))
 
 def run_batch(args):
-    """Batch > 1 through grinqh_select_vmm_batch on the Llama3-8B step (21
-    (linear, width) pairs, two packed copies rotated): for T tokens per call,
-    microseconds per call and per token, graph-replayed; the T activation
-    vectors of a pair are drawn like the batch-1 ones."""
+    """Batch > 1 on the Llama3-8B step (21 (linear, width) pairs, two packed copies
+    rotated): for T tokens per call, microseconds per call and per token,
+    graph-replayed, through grinqh_select_vmm_batch (every token graded and rebuilt
+    as at batch one) and through grinqh_select_vmm_batch_tc (rows rebuilt once for
+    all tokens, width classes as tensor-core MMAs); the T activation vectors of a
+    pair are drawn like the batch-1 ones."""
     import torch
     from activation_graded_bit_b200 import grinqh as g
     from activation_graded_bit_b200 import workloads as wl
@@ -847,18 +849,10 @@ def run_batch(args):
         groups.setdefault(pr["copy"], []).append(pr)
     copies = sorted(groups)
     stream = torch.cuda.Stream(device=dev)
+    status = torch.zeros(4, dtype=torch.int32, device=dev)
     out = []
-    for T in (1, 2, 4, 8, 16):
-        for pr in pairs:
-            X = wl.activations_outlier(pr["K"], T, key=(7, pr["copy"], T, pr["K"], pr["N"], int(pr["target"])),
-                                       chan_key=(1, 0, 0))
-            pr["X"] = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).to(dev)
-            pr["Y"] = torch.empty((T, pr["N"]), dtype=torch.float32, device=dev)
-            pr["wsT"] = g.vmm_batch_workspace(pr["packed"].layout, T, dev)
 
-        def step(c):
-            for pr in groups[c]:
-                g.select_vmm_batch(pr["packed"], pr["X"], pr["th"], CLASSES, pr["wsT"], Y=pr["Y"], stream=stream)
+    def timed(step):
         graphs = {}
         with torch.cuda.stream(stream):
             for c in copies:
@@ -880,13 +874,35 @@ def run_batch(args):
                 graphs[copies[i % len(copies)]].replay()
             e1.record(stream)
         stream.synchronize()
-        us_call = e0.elapsed_time(e1) * 1e3 / (steps * len(groups[copies[0]]))
-        out.append({"tokens": T, "us_per_call": round(us_call, 3), "us_per_token": round(us_call / T, 3)})
         del graphs
+        return e0.elapsed_time(e1) * 1e3 / (steps * len(groups[copies[0]]))
+
+    for T in (1, 2, 4, 8, 16, 32, 64):
+        for pr in pairs:
+            X = wl.activations_outlier(pr["K"], T, key=(7, pr["copy"], T, pr["K"], pr["N"], int(pr["target"])),
+                                       chan_key=(1, 0, 0))
+            pr["X"] = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).to(dev)
+            pr["Y"] = torch.empty((T, pr["N"]), dtype=torch.float32, device=dev)
+            pr["wsT"] = g.vmm_batch_workspace(pr["packed"].layout, T, dev)
+
+        def step(c):
+            for pr in groups[c]:
+                g.select_vmm_batch(pr["packed"], pr["X"], pr["th"], CLASSES, pr["wsT"], Y=pr["Y"], stream=stream)
+
+        def step_tc(c):
+            for pr in groups[c]:
+                g.select_vmm_batch_tc(pr["packed"], pr["X"], pr["th"], CLASSES, status, Y=pr["Y"], stream=stream)
+        us_call = timed(step)
+        us_tc = timed(step_tc)
+        torch.cuda.synchronize()
+        assert int(status.count_nonzero()) == 0, "the tensor-core batch reported a status"
+        out.append({"tokens": T, "us_per_call": round(us_call, 3), "us_per_token": round(us_call / T, 3),
+                    "tc_us_per_call": round(us_tc, 3), "tc_us_per_token": round(us_tc / T, 3)})
         assert all(bool(torch.isfinite(pr["Y"]).all()) for pr in groups[copies[0]])
-    print(json.dumps({"metric": "grinqh_select_vmm_batch: us per (linear, width) call and per token vs batch size",
+    print(json.dumps({"metric": "batched graded VMM: us per (linear, width) call and per token vs batch size "
+                                "(per-token kernel and tensor-core kernel)",
                       "unit": "µs", "higher_is_better": False, "data": "synthetic",
-                      "config": {"workload": WORKLOAD.replace("batch 1", "batch 1..16"), "classes": list(CLASSES),
+                      "config": {"workload": WORKLOAD.replace("batch 1", "batch 1..64"), "classes": list(CLASSES),
                                  "b_max": BMAX, "l2": "two packed copies of the layer set rotate"},
                       "points": out}))
 

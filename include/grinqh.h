@@ -21,6 +21,7 @@
  * and, for the same packed layer:
  *   grinqh_select_vmm        grading and the graded product in one launch
  *   grinqh_select_vmm_batch  the same for T tokens in one launch
+ *   grinqh_select_vmm_batch_tc  the same on the tensor cores, one rebuild per row
  *   grinqh_vmm_noalloc       grinqh_vmm on the library's own static scratch
  *   grinqh_dequant / grinqh_prefill   full-width weights and the dense prefill
  *                            product for many tokens
@@ -422,6 +423,35 @@ grinqh_status grinqh_select_vmm_batch(const grinqh_layout* layout, const void* p
                                       int32_t tokens, const float* thresholds, const uint8_t* classes,
                                       int32_t n_classes, float* Y, void* workspace, size_t workspace_bytes,
                                       void* stream);
+
+/*
+ * The batched graded product on the 5th-generation tensor cores: Y[t] = the graded
+ * product of X[t] (every token graded from its own |x| and every row rebuilt at
+ * that token's width, as grinqh_select_vmm does), with each row's planes read
+ * and merged once for all tokens. Paper: Section 3.1 (per-token grading), Section
+ * 3.3 (nested codes and bin midpoints) and Section 6 (the method targets batch
+ * size one; this library keeps every token's grading). Per 128-column group the
+ * product is split by width class into tcgen05 MMAs (sm_100a): the codes masked
+ * to the class's width times a power of two (exact in binary16) against x times
+ * the scale's significand split into two binary16 parts, fp32 accumulation; the
+ * bin midpoint and zero point enter as a per-token constant in fp32. Results
+ * agree with grinqh_select_vmm_batch within the VMM tolerance, not bitwise.
+ * Deterministic: the same inputs give the same bits. Allocates nothing.
+ *   X        device fp16 [tokens][K] row-major, 16-byte aligned; K a multiple of 8.
+ *   tokens   1..65535; CTAs take 64 tokens each.
+ *   thresholds, classes, n_classes: as grinqh_select_vmm.
+ *   Y        device fp32 [tokens][N], output (overwritten), 4-byte aligned.
+ *   status   device, 16 bytes, 16-byte aligned, zero-filled before first use;
+ *            bit 0 of its first word: a wait inside the kernel gave up after about
+ *            a second; bit 1: a value outside the binary16 range of the operands
+ *            (|x| times the scale's significand of 32768 or more, or a scale of
+ *            2^(14 - b_max) or more). Either bit means Y is not valid; no call
+ *            clears them.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (K not a multiple of 8), CUDA.
+ */
+grinqh_status grinqh_select_vmm_batch_tc(const grinqh_layout* layout, const void* packed, const uint16_t* X,
+                                         int32_t tokens, const float* thresholds, const uint8_t* classes,
+                                         int32_t n_classes, float* Y, uint32_t* status, void* stream);
 
 /*
  * grinqh_vmm without a caller-provided workspace. The paper has no counterpart:
