@@ -15,18 +15,20 @@
 // The first term is an MMA per class: A = the codes masked to the class width
 // times a power of two, exact in binary16; B = x m in two binary16 parts (hi =
 // fp16(v), lo = fp16(v - hi), about 22 significant bits together, near |x| in
-// magnitude), zero where the token's class differs; fp32 accumulation in tensor
-// memory. The second term is a per-token constant of the group, added in fp32 at
+// magnitude), zero where the token's class differs, the hi parts of the tokens in
+// B's first Tp rows and the lo parts in the next Tp, so that one MMA of N = 2 Tp
+// fetches the A tile once for both; fp32 accumulation in tensor memory, the two
+// halves added in the epilogue. The second term is a per-token constant of the group, added in fp32 at
 // the end. A binary16 overflow (|x m| >= 32768, or a scale of 2^(14 - b_max) or
 // more) sets bit 1 of the status word: the launch's Y is then not valid.
 //
 // One CTA computes one 128-column group (the MMA's M) for up to 32 tokens (the
-// MMA's N, padded to 16), looping over K in stages of 64 rows; a step is one
-// stage with up to four active classes (more classes take more steps per stage)
-// and owns one slot of a 2-deep shared-memory ring (per class 16 KB of codes and
-// 2 x 4 KB of activations), so the roles meet once per stage:
+// MMA's N is twice that, padded to 16 tokens), looping over K in stages of 64
+// rows; a step is one stage with up to four active classes (more classes take
+// more steps per stage) and owns one slot of a 2-deep shared-memory ring (per
+// class 16 KB of codes and 8 KB of activations), so the roles meet once per stage:
 //   warp 0      allocates the TMEM columns and, from one lane, issues per step and
-//               class four K = 16 MMAs for the hi part and four for the lo part;
+//               class four K = 16 MMAs;
 //   warps 1..8  read a stage's plane words (two stages ahead), merge each row's
 //               codes once, and per class write the masked codes as binary16
 //               (the row's exponent byte over c, minus 2^pe 1024: exact) in the
@@ -58,8 +60,9 @@ constexpr int kQMaxTok = 32;                     // tokens per CTA (MMA N, padde
 constexpr int kQRing = 2;                        // ring slots, one per step
 constexpr int kQCls = 4;                         // classes per step
 constexpr int kQABytes = kQM * kQK * 2;          // 16 KB: one class's codes
-constexpr int kQBBytes = kQMaxTok * kQK * 2;     // 4 KB: one class's hi (or lo) activations
-constexpr int kQSlot = kQCls * (kQABytes + 2 * kQBBytes);   // 96 KB: codes of 4 classes, then activations
+constexpr int kQBBytes = 2 * kQMaxTok * kQK * 2; // 8 KB: one class's hi and lo activations
+constexpr int kQSlot = kQCls * (kQABytes + kQBBytes);   // 96 KB: codes of 4 classes, then activations
+constexpr int kQTmemCols = 2 * kQMaxTok;         // accumulator: hi products, then lo products
 constexpr int kQRebuildWarps = 8, kQBuildWarps = 8;
 constexpr int kQBuildThreads = 32 * kQBuildWarps;
 static_assert(kQBuildThreads >= 8 * kQMaxTok, "one 8-row chunk per grading thread");
@@ -147,7 +150,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   if (threadIdx.x < kQMaxTok) sy.corr[threadIdx.x] = 0.0f;
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(&sy.tmem)),
-                 "r"(kQMaxTok)
+                 "r"(kQTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -163,27 +166,27 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
   if (warp == 0) {
     // ---------------- MMA issue ----------------
-    // kind::f16, D fp32, A (codes) MN-major, B (activations) K-major, M = 128, N = Tp
-    const uint32_t idesc = (1u << 4) | (1u << 15) | ((uint32_t)(Tp >> 3) << 17) | ((uint32_t)(kQM >> 4) << 24);
+    // kind::f16, D fp32, A (codes) MN-major, B (activations) K-major, M = 128, N = 2 Tp
+    const uint32_t idesc = (1u << 4) | (1u << 15) | ((uint32_t)(2 * Tp >> 3) << 17) | ((uint32_t)(kQM >> 4) << 24);
+    // descriptors of slot 0, class 0, K step 0; the others differ in the start
+    // address field only (bits 0..13, address / 16; no carry out of it: the ring
+    // ends below 256 KB)
+    const uint64_t ad0 = smem_desc(a0, 1024, 2048);
+    const uint64_t bd0 = smem_desc(a0 + kQCls * kQABytes, 16, 1024);
     for (int u = 0; u < steps && ok; ++u) {
       const int slot = u % kQRing;
       const uint32_t ph = (uint32_t)(u / kQRing) & 1u;
       ok = bar_wait(saddr(&sy.full_a[slot]), ph) && bar_wait(saddr(&sy.full_b[slot]), ph);
       tc_after();
       if (ok && lane == 0) {
-        const uint32_t sa = a0 + slot * kQSlot;
         const int ncl = min(kQCls, n_act - (u % n_grp) * kQCls);   // classes of this step
         for (int ci = 0; ci < ncl; ++ci) {
-          const uint32_t aa = sa + ci * kQABytes;
-          const uint32_t bb = sa + kQCls * kQABytes + ci * 2 * kQBBytes;
+          const uint32_t oa = (uint32_t)(slot * kQSlot + ci * kQABytes) >> 4;
+          const uint32_t ob = (uint32_t)(slot * kQSlot + ci * kQBBytes) >> 4;
 #pragma unroll
-          for (int kk = 0; kk < kQK / 16; ++kk) {
-            const uint64_t ad = smem_desc(aa + kk * 4096, 1024, 2048);
-            const uint64_t bh = smem_desc(bb + kk * 32, 16, 1024);
-            const uint64_t bl = smem_desc(bb + kQBBytes + kk * 32, 16, 1024);
-            mma_f16(tmem, ad, bh, idesc, (u > 0 || ci > 0 || kk > 0) ? 1u : 0u);
-            mma_f16(tmem, ad, bl, idesc, 1u);
-          }
+          for (int kk = 0; kk < kQK / 16; ++kk)
+            mma_f16(tmem, ad0 + oa + kk * (4096 >> 4), bd0 + ob + kk * (32 >> 4), idesc,
+                    (u > 0 || ci > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(saddr(&sy.empty[slot]));
       }
@@ -295,6 +298,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
         for (int e = 0; e < 8; ++e) mw[e] = 0u;
       }
     };
+    float th[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) th[i] = (i < nth) ? sy.th[i] : __int_as_float(0x7fc00000);   // NaN: no |x| reaches it
     uint4 xn;
     uint32_t mn[8];
     load_chunk(0, xn, mn);
@@ -315,7 +321,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const float ax = fabsf(x);
         int j = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) j += (i < nth && ax >= sy.th[i]) ? 1 : 0;   // NaN reaches none
+        for (int i = 0; i < 8; ++i) j += (ax >= th[i]) ? 1 : 0;   // NaN reaches none
         const int b = sy.width[j];
         const float xs = x * s;                       // exact: two 11-bit significands
         // m: the scale's significand in [1, 2) (s 2^14 for a subnormal scale)
@@ -343,12 +349,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
         if (!ok) break;
         const int ncl = min(kQCls, n_act - gi * kQCls);
         if (id < nch) {
-          // row t of the K-major tile: 8-row groups 1 KB apart, 128 bytes per row,
-          // 16-byte chunk kc stored at chunk index kc ^ (t % 8)
+          // row t (hi) and row Tp + t (lo) of the K-major tile: 8-row groups 1 KB
+          // apart, 128 bytes per row, 16-byte chunk kc stored at chunk index kc ^ (row
+          // % 8); Tp is a multiple of 16, so row Tp + t sits Tp * 128 bytes after row t
           const uint32_t off = (uint32_t)((t >> 3) * 1024 + (t & 7) * 128) + ((uint32_t)(kc ^ (t & 7)) << 4);
+          const uint32_t lo_off = (uint32_t)Tp * 128u;
           for (int ci = 0; ci < ncl; ++ci) {
             const uint32_t jc = (uint32_t)sy.act[gi * kQCls + ci];
-            const uint32_t sb = a0 + slot * kQSlot + kQCls * kQABytes + ci * 2 * kQBBytes;
+            const uint32_t sb = a0 + slot * kQSlot + kQCls * kQABytes + ci * kQBBytes;
             uint32_t mh[4], ml[4];
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
@@ -360,7 +368,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sb + off), "r"(mh[0]), "r"(mh[1]),
                          "r"(mh[2]), "r"(mh[3])
                          : "memory");
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sb + kQBBytes + off), "r"(ml[0]),
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sb + lo_off + off), "r"(ml[0]),
                          "r"(ml[1]), "r"(ml[2]), "r"(ml[3])
                          : "memory");
           }
@@ -386,7 +394,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
   // ---------------- epilogue ----------------
   // warps 1..4 read TMEM lane quarter (warp % 4): lane i = column n0 + 32 (warp % 4) + i,
-  // TMEM column t = token t; y = D + the token's constant
+  // TMEM column t = token t's hi product, column Tp + t its lo product; y = both +
+  // the token's constant
   float* dump = reinterpret_cast<float*>(q_smem + (a0 - raw));   // [token][column] for the cluster sum
   if (warp >= 1 && warp <= 4) {
     const bool acc_ok = (sy.failed & 1u) == 0u && bar_wait(saddr(&sy.accum), 0u);
@@ -394,23 +403,30 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int qq = warp & 3;
     const int n = n0 + 32 * qq + lane;
     for (int c16 = 0; c16 < Tp; c16 += 16) {
-      uint32_t v[16];
+      uint32_t v[16], w[16];
       if (n_act > 0 && n_k > 0) {
+        const uint32_t ta = tmem + ((uint32_t)(32 * qq) << 16) + (uint32_t)c16;
         asm volatile(
             "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
             "%14, %15}, [%16];"
             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
               "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-            : "r"(tmem + ((uint32_t)(32 * qq) << 16) + (uint32_t)c16));
+            : "r"(ta));
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+            "%14, %15}, [%16];"
+            : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7]),
+              "=r"(w[8]), "=r"(w[9]), "=r"(w[10]), "=r"(w[11]), "=r"(w[12]), "=r"(w[13]), "=r"(w[14]), "=r"(w[15])
+            : "r"(ta + (uint32_t)Tp));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = 0u;   // no class of nonzero width: only the constant
+        for (int i = 0; i < 16; ++i) v[i] = w[i] = 0u;   // no class of nonzero width: only the constant
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int t = c16 + i;
-        const float yv = __uint_as_float(v[i]) + sy.corr[t < kQMaxTok ? t : 0];
+        const float yv = (__uint_as_float(v[i]) + __uint_as_float(w[i])) + sy.corr[t < kQMaxTok ? t : 0];
         if (kSplit == 1) {
           if (t < Tc && n < N && acc_ok) Y[(size_t)t * N + n] = yv;
         } else {
@@ -442,7 +458,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   if (threadIdx.x == 0 && sy.failed != 0u) atomicOr(status, sy.failed);
   if (warp == 0) {
     tc_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kQMaxTok) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kQTmemCols) : "memory");
   }
 }
 

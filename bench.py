@@ -581,6 +581,9 @@ def run_profile_case(args):
     ws = g.vmm_workspace(p.layout, dev)
     y = torch.empty(N, dtype=torch.float32, device=dev)
     sel = g.empty_selection(K, wl.CLASSES, dev)
+    if args.prefill or args.batch:
+        _profile_tc(args, g, wl, p, th, K, N, li, dev)
+        return
     if args.lut:
         # nested table codes on the same layer: synthetic codes and tables
         codes = torch.randint(0, 256, (K, N), generator=gen, device=dev, dtype=torch.uint8)
@@ -605,6 +608,31 @@ def run_profile_case(args):
           % (args.profile, args.bits, args.iters, "vmm_lut" if args.lut else "vmm", active,
              active * p.layout.n_tiles, int(alg)))
 
+
+def _profile_tc(args, g, wl, p, th, K, N, li, dev):
+    """The tensor-core kernels' small case: `--iters` eager grinqh_prefill_tc calls
+    (with --prefill) or grinqh_select_vmm_batch_tc calls (with --batch) on one
+    linear at `--tokens` tokens, and the flop and algorithmic byte counts a
+    capture is divided by."""
+    import torch
+    T = args.tokens if args.tokens else (2048 if args.prefill else 16)
+    X = wl.activations_outlier(K, T, key=(1, 1, li, T), chan_key=(1, 0, li))
+    X_d = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).to(dev)
+    Y = torch.empty((T, N), dtype=torch.float32, device=dev)
+    status = torch.zeros(4, dtype=torch.int32, device=dev)
+    for _ in range(args.iters):
+        if args.prefill:
+            g.prefill_tc(p, X_d, status, Y=Y)
+        else:
+            g.select_vmm_batch_tc(p, X_d, th, wl.CLASSES, status, Y=Y)
+    torch.cuda.synchronize()
+    assert int(status.count_nonzero()) == 0 and bool(torch.isfinite(Y).all())
+    # prefill: every row at b_max, 2 T K N flops; planes + scale/zero words read
+    # once, X read, Y written. batch: the rows some token grades nonzero, read once.
+    alg = p.packed.numel() + 2.0 * K * T + 4.0 * N * T
+    print("profile case %s %s: %d calls at %d tokens; %.4g flops per call (2 T K N), %d algorithmic bytes"
+          % (args.profile, "prefill_tc" if args.prefill else "select_vmm_batch_tc @ %g bits" % args.bits,
+             args.iters, T, 2.0 * T * K * N, int(alg)))
 
 
 # ---------------------------------------------------------------------------
@@ -1149,6 +1177,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", default=None, help="linear name: run one small case for ncu and exit")
     ap.add_argument("--bits", type=float, default=4.0)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="with --profile and --prefill or --batch: tokens per call (default 2048 or 16)")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--sweep", action="store_true", help="average-bit sweep on a 14336x4096 layer (one JSON line)")
     ap.add_argument("--stack", action="store_true", help="32-layer linear stack tokens/s (one JSON line)")
@@ -1175,6 +1205,9 @@ def main():
         WORKLOAD = WORKLOAD + ", b_max %d codes, classes %s" % (BMAX, "/".join(map(str, CLASSES)))
     if args.warmup < 3:
         args.warmup = 3
+    if args.profile:
+        run_profile_case(args)
+        return
     if args.sweep:
         run_sweep(args)
         return
@@ -1187,15 +1220,13 @@ def main():
     if args.prefill:
         run_prefill(args)
         return
-    if args.lut and not args.profile:
+    if args.lut:
         run_lut(args)
         return
     if args.cold:
         run_cold(args)
         return
-    if args.profile:
-        run_profile_case(args)
-    elif args.impl == "reference":
+    if args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)
