@@ -18,9 +18,12 @@
 // magnitude), zero where the token's class differs, the hi parts of the tokens in
 // B's first Tp rows and the lo parts in the next Tp, so that one MMA of N = 2 Tp
 // fetches the A tile once for both; fp32 accumulation in tensor memory, the two
-// halves added in the epilogue. The second term is a per-token constant of the group, added in fp32 at
-// the end. A binary16 overflow (|x m| >= 32768, or a scale of 2^(14 - b_max) or
-// more) sets bit 1 of the status word: the launch's Y is then not valid.
+// halves added in the epilogue. The four K = 16 MMAs of a stage and class go to
+// four accumulators (summed at the end), so that no MMA waits for the result of
+// the one issued just before it. The second term is a per-token constant of the
+// group, added in fp32 at the end. A binary16 overflow (|x m| rounded to binary16
+// >= 32768, or a scale of 2^(14 - b_max) or more) sets bit 1 of the status word:
+// the launch's Y is then not valid.
 //
 // One CTA computes one 128-column group (the MMA's M) for up to 32 tokens (the
 // MMA's N is twice that, padded to 16 tokens), looping over K in stages of 64
@@ -37,7 +40,7 @@
 //   warps 9..16 grade the stage's (token, row) pairs against the thresholds,
 //               form the hi/lo parts once, and per class write the masked parts in
 //               the K-major 128-byte-swizzled layout of the B descriptor; they also
-//               accumulate the per-token constant.
+//               accumulate the per-token constant (Tp / 4 of them: 8 rows a thread).
 // Small grids split K over a cluster of 2, 4 or 8 CTAs that add their
 // accumulators through distributed shared memory in rank order (deterministic).
 // Every mbarrier wait is bounded by the global timer; one that gives up sets bit
@@ -62,7 +65,9 @@ constexpr int kQCls = 4;                         // classes per step
 constexpr int kQABytes = kQM * kQK * 2;          // 16 KB: one class's codes
 constexpr int kQBBytes = 2 * kQMaxTok * kQK * 2; // 8 KB: one class's hi and lo activations
 constexpr int kQSlot = kQCls * (kQABytes + kQBBytes);   // 96 KB: codes of 4 classes, then activations
-constexpr int kQTmemCols = 2 * kQMaxTok;         // accumulator: hi products, then lo products
+constexpr int kQAcc = 4;                         // accumulators, one per K = 16 step of a stage
+constexpr int kQAccCols = 2 * kQMaxTok;          // one accumulator: hi products, then lo products
+constexpr int kQTmemCols = kQAcc * kQAccCols;
 constexpr int kQRebuildWarps = 8, kQBuildWarps = 8;
 constexpr int kQBuildThreads = 32 * kQBuildWarps;
 static_assert(kQBuildThreads >= 8 * kQMaxTok, "one 8-row chunk per grading thread");
@@ -79,13 +84,25 @@ struct QSync {
   int n_act;                           // classes of nonzero width
   int act[9];                          // their class indices
   int width[9];                        // width of every class
-  float th[8];                         // the thresholds
+  float mid[9];                        // bin midpoint of every class of nonzero width
+  uint32_t actmask;                    // bit j: class j has nonzero width
+  int n_th;                            // thresholds
+  unsigned short thh[8];               // the thresholds rounded up to binary16 (NaN past the last)
   float corr[kQMaxTok];                // per token: sum of x s (mid - z) over this CTA's rows
 };
 
 constexpr size_t kQSmem = 1024 + (size_t)kQRing * kQSlot + sizeof(QSync);
 static_assert(kQSmem <= 227 * 1024, "batch kernel shared memory");
 static_assert(kQMaxTok * kQM * 4 <= kQRing * kQSlot, "the split's accumulator copy fits the ring");
+
+// prmt.b32 in its generic mode: a selector nibble with its top bit set fills the
+// result byte with the top bit of the source byte it names (the CUDA intrinsic
+// __byte_perm uses only the low three bits of each nibble)
+__device__ __forceinline__ uint32_t prmt_sign(uint32_t a, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(0u), "r"(sel));
+  return r;
+}
 
 struct QWords {
   uint32_t p[8];
@@ -133,20 +150,31 @@ __global__ void __launch_bounds__(kQThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kQRing; ++i) {
       bar_init(saddr(&sy.full_a[i]), kQRebuildWarps);
-      bar_init(saddr(&sy.full_b[i]), kQBuildWarps);
+      bar_init(saddr(&sy.full_b[i]), Tp / 4);   // the grading warps with tokens (8 rows a thread)
       bar_init(saddr(&sy.empty[i]), 1);
     }
     bar_init(saddr(&sy.accum), 1);
     sy.failed = 0u;
     int na = 0;
-    for (int j = 0; j < ct.n; ++j) {
-      sy.width[j] = ct.width[j];
-      if (ct.width[j] > 0) sy.act[na++] = j;
+    uint32_t am = 0u;
+    for (int j = 0; j < 9; ++j) {
+      const int b = (j < ct.n) ? ct.width[j] : 0;
+      sy.width[j] = b;
+      sy.mid[j] = (b <= 0 || b >= kBmax) ? 0.0f : (float)(1u << (kBmax - b - 1));
+      if (b > 0) {
+        sy.act[na++] = j;
+        am |= 1u << j;
+      }
     }
     sy.n_act = na;
+    sy.actmask = am;
+    sy.n_th = ct.n - 1;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (threadIdx.x < 8) sy.th[threadIdx.x] = (threadIdx.x < ct.n - 1) ? __ldg(thresholds + threadIdx.x) : 0.0f;
+  if (threadIdx.x < 8)
+    sy.thh[threadIdx.x] = (threadIdx.x < ct.n - 1)
+                              ? __half_as_ushort(__float2half_ru(__ldg(thresholds + threadIdx.x)))
+                              : (unsigned short)0x7E00u;
   if (threadIdx.x < kQMaxTok) sy.corr[threadIdx.x] = 0.0f;
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(&sy.tmem)),
@@ -185,8 +213,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
           const uint32_t ob = (uint32_t)(slot * kQSlot + ci * kQBBytes) >> 4;
 #pragma unroll
           for (int kk = 0; kk < kQK / 16; ++kk)
-            mma_f16(tmem, ad0 + oa + kk * (4096 >> 4), bd0 + ob + kk * (32 >> 4), idesc,
-                    (u > 0 || ci > 0 || kk > 0) ? 1u : 0u);
+            mma_f16(tmem + (uint32_t)(kk * kQAccCols), ad0 + oa + kk * (4096 >> 4), bd0 + ob + kk * (32 >> 4),
+                    idesc, (u > 0 || ci > 0) ? 1u : 0u);
         }
         mma_commit(saddr(&sy.empty[slot]));
       }
@@ -237,6 +265,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
         const uint32_t cw = ((uint32_t)(pe + 25) & 31u) << 10;   // 2^pe 1024
         const uint32_t cw2 = cw * 0x10001u;
         const __half2 c2 = *reinterpret_cast<const __half2*>(&cw2);
+        // F[2j], F[2j+1]: the binary16 pairs {2^pe (1024 + c0), 2^pe (1024 + c1)} and
+        // {2^pe (1024 + c2), 2^pe (1024 + c3)} of the four codes in R[j]
+        uint32_t F[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          F[2 * j] = __byte_perm(R[j], ebx4, 0x5140u);
+          F[2 * j + 1] = __byte_perm(R[j], ebx4, 0x7362u);
+        }
         if (it + kQAhead < n_k) load_stage(it + kQAhead, buf[i]);
         for (int gi = 0; gi < n_grp && ok; ++gi) {
           const int u = it * n_grp + gi;
@@ -246,18 +282,15 @@ __global__ void __launch_bounds__(kQThreads, 1)
           const int ncl = min(kQCls, n_act - gi * kQCls);
           for (int ci = 0; ci < ncl; ++ci) {
           const uint32_t b = (uint32_t)sy.width[sy.act[gi * kQCls + ci]];
-          const uint32_t top = ((0xFFu << (8u - b)) & 0xFFu) * 0x01010101u;
+          // keep the exponent bytes and the top b bits of every code byte
+          const uint32_t top = 0xFF00FF00u | (((0xFFu << (8u - b)) & 0xFFu) * 0x00010001u);
           const uint32_t row = a0 + slot * kQSlot + ci * kQABytes + row_off;
           uint32_t h[16];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t v = R[j] & top;
-            const uint32_t lo = __byte_perm(v, ebx4, 0x5140u);   // {2^pe (1024 + c0), 2^pe (1024 + c1)}
-            const uint32_t hi = __byte_perm(v, ebx4, 0x7362u);   // {2^pe (1024 + c2), 2^pe (1024 + c3)}
-            const __half2 e0 = __hsub2(*reinterpret_cast<const __half2*>(&lo), c2);
-            const __half2 e1 = __hsub2(*reinterpret_cast<const __half2*>(&hi), c2);
-            h[2 * j] = *reinterpret_cast<const uint32_t*>(&e0);
-            h[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&e1);
+          for (int j = 0; j < 16; ++j) {
+            const uint32_t v = F[j] & top;
+            const __half2 e = __hsub2(*reinterpret_cast<const __half2*>(&v), c2);
+            h[j] = *reinterpret_cast<const uint32_t*>(&e);
           }
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
@@ -276,114 +309,132 @@ __global__ void __launch_bounds__(kQThreads, 1)
   } else {
     // ---------------- activations: grade once per stage, mask per class ----------------
     // thread i takes the 8-row chunk i of a stage: chunk id = 8 t + kc is rows
-    // 8 kc .. 8 kc + 7 of token t (at most 32 tokens: one chunk per thread); its x
-    // and scale/zero words are loaded one stage ahead
+    // 8 kc .. 8 kc + 7 of token t (at most 32 tokens: one chunk per thread, Tp / 4
+    // warps; the others have nothing to do); its x and scale/zero words are loaded
+    // one stage ahead. Rows are taken in pairs, as binary16 pairs:
+    //   class: the number of thresholds |x| reaches, counted as 1024 + j in
+    //     binary16 (HSET2 results added); a binary16 |x| reaches the threshold th
+    //     exactly when it reaches th rounded up to binary16;
+    //   hi = fp16(x m) and lo = fp16(x m - hi) (one fused multiply-add: x m - hi
+    //     is exact in binary32, so it is rounded once, as in two steps);
+    //   the per-token constant x s (mid - z) in fp32 (x s exact).
     const int id = threadIdx.x - 32 * (1 + kQRebuildWarps);
-    const int nch = Tp * 8;
-    const int nth = ct.n - 1;   // thresholds
-    const int t = id >> 3, kc = id & 7;
-    const bool mine = id < nch && t < Tc;   // padding tokens stay zero
-    float corr = 0.0f;
-    auto load_chunk = [&](int it, uint4& xv, uint32_t (&mw)[8]) {
-      const int k0 = (ks0 + it) * kQK + 8 * kc;
-      if (mine && k0 < K) {
-        xv = __ldg(reinterpret_cast<const uint4*>(X + (size_t)t * K + k0));
+    const int nch = Tp * 8;   // a multiple of 32: whole warps
+    if (id < nch) {
+      const int t = id >> 3, kc = id & 7;
+      const bool mine = t < Tc;   // padding tokens stay zero
+      float corr = 0.0f;
+      auto load_chunk = [&](int it, uint4& xv, uint32_t (&mw)[8]) {
+        const int k0 = (ks0 + it) * kQK + 8 * kc;
+        if (mine && k0 < K) {
+          xv = __ldg(reinterpret_cast<const uint4*>(X + (size_t)t * K + k0));
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          mw[e] = __ldg(reinterpret_cast<const uint32_t*>(packed + meta_offset +
-                                                           ((size_t)(k0 + e) * n_tiles + t_rec) * kMetaBytes + 4 * sl));
-      } else {
-        xv = make_uint4(0u, 0u, 0u, 0u);   // rows past K, padding tokens: x = 0 (class 0, no term)
+          for (int e = 0; e < 8; ++e)
+            mw[e] = __ldg(reinterpret_cast<const uint32_t*>(packed + meta_offset +
+                                                             ((size_t)(k0 + e) * n_tiles + t_rec) * kMetaBytes + 4 * sl));
+        } else {
+          xv = make_uint4(0u, 0u, 0u, 0u);   // rows past K, padding tokens: x = 0 (class 0, no term)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mw[e] = 0u;
-      }
-    };
-    float th[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) th[i] = (i < nth) ? sy.th[i] : __int_as_float(0x7fc00000);   // NaN: no |x| reaches it
-    uint4 xn;
-    uint32_t mn[8];
-    load_chunk(0, xn, mn);
-    for (int it = 0; it < n_k && ok; ++it) {
-      const uint4 xv = xn;
-      uint32_t mw[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mw[e] = mn[e];
-      if (it + 1 < n_k) load_chunk(it + 1, xn, mn);
-      // hi and lo parts of x m as 4 + 4 half pairs, and the 8 classes, one nibble each
-      uint32_t hw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u}, cls = 0u;
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint32_t m = mw[e];
-        const float s = half_bits_to_float(m), z = half_bits_to_float(m >> 16);
-        const float x = half_bits_to_float((e & 1) ? (xw[e >> 1] >> 16) : xw[e >> 1]);
-        const float ax = fabsf(x);
-        int j = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) j += (ax >= th[i]) ? 1 : 0;   // NaN reaches none
-        const int b = sy.width[j];
-        const float xs = x * s;                       // exact: two 11-bit significands
-        // m: the scale's significand in [1, 2) (s 2^14 for a subnormal scale)
-        const uint32_t sbits = m & 0xFFFFu;
-        const float mm = (((sbits >> 10) & 31u) != 0u)
-                             ? __half2float(__ushort_as_half((unsigned short)((sbits & 0x3FFu) | 0x3C00u)))
-                             : s * 16384.0f;
-        const float v = x * mm;                       // exact
-        if (fabsf(v) >= 32768.0f) bad = true;
-        const __half vh = __float2half_rn(v);
-        const __half vl = __float2half_rn(v - __half2float(vh));
-        const uint32_t hb = __half_as_ushort(vh), lb = __half_as_ushort(vl);
-        hw[e >> 1] |= (e & 1) ? (hb << 16) : hb;
-        lw[e >> 1] |= (e & 1) ? (lb << 16) : lb;
-        cls |= (uint32_t)j << (4 * e);
-        if (b > 0) {
-          const float mid = (b >= kBmax) ? 0.0f : (float)(1u << (kBmax - b - 1));
-          corr = fmaf(xs, mid - z, corr);
+          for (int e = 0; e < 8; ++e) mw[e] = 0u;
         }
-      }
-      for (int gi = 0; gi < n_grp && ok; ++gi) {
-        const int u = it * n_grp + gi;
-        const int slot = u % kQRing;
-        ok = bar_wait(saddr(&sy.empty[slot]), ((uint32_t)(u / kQRing) & 1u) ^ 1u);
-        if (!ok) break;
-        const int ncl = min(kQCls, n_act - gi * kQCls);
-        if (id < nch) {
+      };
+      __half2 th2[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) th2[i] = __half2half2(__ushort_as_half(sy.thh[i]));
+      const bool few = sy.n_th <= 4;
+      const uint32_t actmask = sy.actmask;
+      __half2 amax = __float2half2_rn(0.0f);
+      uint4 xn;
+      uint32_t mn[8];
+      load_chunk(0, xn, mn);
+      for (int it = 0; it < n_k && ok; ++it) {
+        const uint4 xv = xn;
+        uint32_t mw[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mw[e] = mn[e];
+        if (it + 1 < n_k) load_chunk(it + 1, xn, mn);
+        uint32_t hw[4], lw[4], cnt[4];
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const uint32_t x2b = xw[p];
+          const uint32_t s2b = __byte_perm(mw[2 * p], mw[2 * p + 1], 0x5410u);   // scales of rows 2p, 2p+1
+          const uint32_t z2b = __byte_perm(mw[2 * p], mw[2 * p + 1], 0x7632u);   // zero points
+          const __half2 x2 = *reinterpret_cast<const __half2*>(&x2b);
+          const __half2 s2 = *reinterpret_cast<const __half2*>(&s2b);
+          const __half2 ax2 = __habs2(x2);
+          __half2 c2 = __float2half2_rn(1024.0f);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) c2 = __hadd2(c2, __hge2(ax2, th2[i]));   // NaN reaches none
+          if (!few) {
+#pragma unroll
+            for (int i = 4; i < 8; ++i) c2 = __hadd2(c2, __hge2(ax2, th2[i]));
+          }
+          cnt[p] = *reinterpret_cast<const uint32_t*>(&c2);   // low byte of each half: the class
+          // m: the scale's significand in [1, 2); s 2^14 (exact) for a subnormal scale
+          const uint32_t norm = (s2b & 0x03FF03FFu) | 0x3C003C00u;
+          const __half2 sub = __hmul2(s2, __float2half2_rn(16384.0f));
+          const uint32_t isn = ((s2b & 0x7C007C00u) + 0x7FFF7FFFu) & 0x80008000u;   // bit 15 of a half: normal
+          const uint32_t sel = prmt_sign(isn, 0xBB99u);                        // 0xFFFF where normal
+          const uint32_t m2b = (norm & sel) | (*reinterpret_cast<const uint32_t*>(&sub) & ~sel);
+          const __half2 m2 = *reinterpret_cast<const __half2*>(&m2b);
+          const __half2 hi = __hmul2(x2, m2);
+          const __half2 lo = __hfma2(x2, m2, __hneg2(hi));
+          amax = __hmax2(amax, __habs2(hi));   // NaN (x NaN, or inf times 0) is passed over
+          hw[p] = *reinterpret_cast<const uint32_t*>(&hi);
+          lw[p] = *reinterpret_cast<const uint32_t*>(&lo);
+#pragma unroll
+          for (int l = 0; l < 2; ++l) {
+            const uint32_t j = (cnt[p] >> (16 * l)) & 0xFu;
+            const float x = half_bits_to_float(x2b >> (16 * l));
+            const float sv = half_bits_to_float(s2b >> (16 * l));
+            const float z = half_bits_to_float(z2b >> (16 * l));
+            if ((actmask >> j) & 1u) corr = fmaf(x * sv, sy.mid[j] - z, corr);   // x s exact: two 11-bit significands
+          }
+        }
+        // the class of rows 0..3 and 4..7, one byte each
+        const uint32_t cb0 = __byte_perm(cnt[0], cnt[1], 0x6420u), cb1 = __byte_perm(cnt[2], cnt[3], 0x6420u);
+        for (int gi = 0; gi < n_grp && ok; ++gi) {
+          const int u = it * n_grp + gi;
+          const int slot = u % kQRing;
+          ok = bar_wait(saddr(&sy.empty[slot]), ((uint32_t)(u / kQRing) & 1u) ^ 1u);
+          if (!ok) break;
+          const int ncl = min(kQCls, n_act - gi * kQCls);
           // row t (hi) and row Tp + t (lo) of the K-major tile: 8-row groups 1 KB
           // apart, 128 bytes per row, 16-byte chunk kc stored at chunk index kc ^ (row
           // % 8); Tp is a multiple of 16, so row Tp + t sits Tp * 128 bytes after row t
           const uint32_t off = (uint32_t)((t >> 3) * 1024 + (t & 7) * 128) + ((uint32_t)(kc ^ (t & 7)) << 4);
           const uint32_t lo_off = (uint32_t)Tp * 128u;
           for (int ci = 0; ci < ncl; ++ci) {
-            const uint32_t jc = (uint32_t)sy.act[gi * kQCls + ci];
+            const uint32_t jx = (uint32_t)sy.act[gi * kQCls + ci] * 0x01010101u;
             const uint32_t sb = a0 + slot * kQSlot + kQCls * kQABytes + ci * kQBBytes;
-            uint32_t mh[4], ml[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const uint32_t m0 = (((cls >> (8 * p)) & 0xFu) == jc) ? 0x0000FFFFu : 0u;
-              const uint32_t m1 = (((cls >> (8 * p + 4)) & 0xFu) == jc) ? 0xFFFF0000u : 0u;
-              mh[p] = hw[p] & (m0 | m1);
-              ml[p] = lw[p] & (m0 | m1);
-            }
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sb + off), "r"(mh[0]), "r"(mh[1]),
-                         "r"(mh[2]), "r"(mh[3])
+            // bit 7 of a byte: that row's class differs (bytes are at most 15, so
+            // adding 0x7F carries into no other byte)
+            const uint32_t d0 = ((cb0 ^ jx) + 0x7F7F7F7Fu) & 0x80808080u;
+            const uint32_t d1 = ((cb1 ^ jx) + 0x7F7F7F7Fu) & 0x80808080u;
+            // per half: 0xFFFF where the row's class differs (the byte's top bit replicated)
+            const uint32_t k0m = prmt_sign(d0, 0x9988u), k1m = prmt_sign(d0, 0xBBAAu);
+            const uint32_t k2m = prmt_sign(d1, 0x9988u), k3m = prmt_sign(d1, 0xBBAAu);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sb + off), "r"(hw[0] & ~k0m),
+                         "r"(hw[1] & ~k1m), "r"(hw[2] & ~k2m), "r"(hw[3] & ~k3m)
                          : "memory");
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sb + lo_off + off), "r"(ml[0]),
-                         "r"(ml[1]), "r"(ml[2]), "r"(ml[3])
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sb + lo_off + off), "r"(lw[0] & ~k0m),
+                         "r"(lw[1] & ~k1m), "r"(lw[2] & ~k2m), "r"(lw[3] & ~k3m)
                          : "memory");
           }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) bar_arrive(saddr(&sy.full_b[slot]));
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) bar_arrive(saddr(&sy.full_b[slot]));
       }
+      if (__hge(__hmax(__low2half(amax), __high2half(amax)), __float2half_rn(32768.0f))) bad = true;
+      // per-token constant: the 8 threads of a token are 8 consecutive lanes
+      float v = corr;
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      if (kc == 0) sy.corr[t] = v;
     }
-    // per-token constant: the 8 threads of a token are 8 consecutive lanes
-    float v = corr;
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    if (kc == 0 && id < nch) sy.corr[t] = v;
   }
   if (!ok) atomicOr(&sy.failed, 1u);
   if (bad) atomicOr(&sy.failed, 2u);
@@ -393,9 +444,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
   ok = ok && (sy.failed & 1u) == 0u;
 
   // ---------------- epilogue ----------------
-  // warps 1..4 read TMEM lane quarter (warp % 4): lane i = column n0 + 32 (warp % 4) + i,
-  // TMEM column t = token t's hi product, column Tp + t its lo product; y = both +
-  // the token's constant
+  // warps 1..4 read TMEM lane quarter (warp % 4): lane i = column n0 + 32 (warp % 4) + i;
+  // in accumulator a (columns 64 a ..), column t holds token t's hi product and
+  // column Tp + t its lo product; y = the sum of all eight + the token's constant
   float* dump = reinterpret_cast<float*>(q_smem + (a0 - raw));   // [token][column] for the cluster sum
   if (warp >= 1 && warp <= 4) {
     const bool acc_ok = (sy.failed & 1u) == 0u && bar_wait(saddr(&sy.accum), 0u);
@@ -403,30 +454,30 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int qq = warp & 3;
     const int n = n0 + 32 * qq + lane;
     for (int c16 = 0; c16 < Tp; c16 += 16) {
-      uint32_t v[16], w[16];
-      if (n_act > 0 && n_k > 0) {
-        const uint32_t ta = tmem + ((uint32_t)(32 * qq) << 16) + (uint32_t)c16;
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-            "%14, %15}, [%16];"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-            : "r"(ta));
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-            "%14, %15}, [%16];"
-            : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7]),
-              "=r"(w[8]), "=r"(w[9]), "=r"(w[10]), "=r"(w[11]), "=r"(w[12]), "=r"(w[13]), "=r"(w[14]), "=r"(w[15])
-            : "r"(ta + (uint32_t)Tp));
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-      } else {
+      float acc[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = w[i] = 0u;   // no class of nonzero width: only the constant
-      }
+      for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+      if (n_act > 0 && n_k > 0) {
+#pragma unroll
+        for (int part = 0; part < 2 * kQAcc; ++part) {   // accumulator part / 2, hi (even) or lo (odd) half
+          uint32_t v[16];
+          const uint32_t ta = tmem + ((uint32_t)(32 * qq) << 16) + (uint32_t)((part >> 1) * kQAccCols) +
+                              (uint32_t)((part & 1) * Tp + c16);
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+              "%14, %15}, [%16];"
+              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+              : "r"(ta));
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
+        }
+      }   // else no class of nonzero width: only the constant
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int t = c16 + i;
-        const float yv = (__uint_as_float(v[i]) + __uint_as_float(w[i])) + sy.corr[t < kQMaxTok ? t : 0];
+        const float yv = acc[i] + sy.corr[t < kQMaxTok ? t : 0];
         if (kSplit == 1) {
           if (t < Tc && n < N && acc_ok) Y[(size_t)t * N + n] = yv;
         } else {

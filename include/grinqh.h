@@ -438,15 +438,15 @@ grinqh_status grinqh_select_vmm_batch(const grinqh_layout* layout, const void* p
  * agree with grinqh_select_vmm_batch within the VMM tolerance, not bitwise.
  * Deterministic: the same inputs give the same bits. Allocates nothing.
  *   X        device fp16 [tokens][K] row-major, 16-byte aligned; K a multiple of 8.
- *   tokens   1..65535; CTAs take 64 tokens each.
+ *   tokens   1..65535; CTAs take 32 tokens each.
  *   thresholds, classes, n_classes: as grinqh_select_vmm.
  *   Y        device fp32 [tokens][N], output (overwritten), 4-byte aligned.
  *   status   device, 16 bytes, 16-byte aligned, zero-filled before first use;
  *            bit 0 of its first word: a wait inside the kernel gave up after about
  *            a second; bit 1: a value outside the binary16 range of the operands
- *            (|x| times the scale's significand of 32768 or more, or a scale of
- *            2^(14 - b_max) or more). Either bit means Y is not valid; no call
- *            clears them.
+ *            (|x| times the scale's significand, rounded to binary16, of 32768 or
+ *            more, or a scale of 2^(14 - b_max) or more). Either bit means Y is
+ *            not valid; no call clears them.
  * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (K not a multiple of 8), CUDA.
  */
 grinqh_status grinqh_select_vmm_batch_tc(const grinqh_layout* layout, const void* packed, const uint16_t* X,

@@ -118,3 +118,53 @@ def test_batch_tc_refuses_k_not_multiple_of_8(g):
     with pytest.raises(g.GrinqhError) as e:
         g.select_vmm_batch_tc(p, X, th, CL, status)
     assert e.value.code == 3
+
+
+def test_batch_tc_threshold_ties_and_unrepresentable_thresholds(g, orc):
+    """Section 3.1: a channel's class is the number of thresholds its |x| reaches.
+    Thresholds equal to some |x| (a tie reaches it), one fp32 step above and below
+    a binary16 value, zero, unsorted and above every |x|: the kernel (which
+    compares binary16 |x| with the thresholds rounded up to binary16) takes the
+    oracle's fp32 decisions, so y agrees within the VMM tolerance for every token."""
+    K, N, T = 512, 256, 8
+    key = (141,)
+    W = wl.weights_rowstd_loguniform(K, N, key=key + (0,))
+    X = wl.activations_outlier(K, T, key=key + (2,), chan_key=key)
+    ax = np.abs(X.view(np.float16).astype(np.float32))
+    a, b, c = float(ax[0, 5]), float(ax[1, 7]), float(ax[2, 9])
+    cases = [np.array([a, np.nextafter(np.float32(b), np.float32(np.inf)), np.nextafter(np.float32(c), np.float32(0)),
+                       float(ax.max()) * 2.0], np.float32),
+             np.array([float(ax.max()) * 2.0, a, 0.0, b], np.float32)]   # unsorted, with zero
+    p = g.pack(torch.from_numpy(W).cuda())
+    Xd = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).cuda()
+    q, s, z = orc.rtn_quantize(W, 8)
+    cl = np.array(CL, np.uint8)
+    for th_ref in cases:
+        status = torch.zeros(4, dtype=torch.int32, device="cuda")
+        Y = g.select_vmm_batch_tc(p, Xd, torch.from_numpy(th_ref).cuda(), CL, status)
+        torch.cuda.synchronize()
+        assert int(status.count_nonzero()) == 0
+        Yb = Y.cpu().numpy()
+        for t in range(T):
+            bits, _, _ = orc.select(X[t], th_ref, cl)
+            yr, bound = orc.vmm(X[t], q, s, z, bits)
+            assert_close(Yb[t], yr, bound, "thresholds %s token %d" % (th_ref, t))
+
+
+def test_batch_tc_flags_values_outside_binary16_range(g):
+    """|x| times the scale's significand at 32768 or more (after rounding to
+    binary16) has no binary16 operand: the kernel sets bit 1 of the status word;
+    below it (|x| <= 16000, significand < 2) the word stays zero."""
+    K, N, T = 256, 256, 4
+    p = g.pack(torch.randn(K, N, device="cuda") * 0.02)
+    th = torch.tensor([0.5, 1.0, 1.5, 2.0], dtype=torch.float32, device="cuda")
+    X = torch.zeros((T, K), dtype=torch.float16, device="cuda")
+    X[:, ::3] = 16000.0
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    g.select_vmm_batch_tc(p, X.view(torch.int16), th, CL, status)
+    torch.cuda.synchronize()
+    assert int(status.count_nonzero()) == 0
+    X[2, 77] = 40000.0
+    g.select_vmm_batch_tc(p, X.view(torch.int16), th, CL, status)
+    torch.cuda.synchronize()
+    assert int(status[0].item()) == 2, status.cpu().numpy()
