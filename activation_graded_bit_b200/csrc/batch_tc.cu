@@ -224,11 +224,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
     __syncwarp();
   } else if (warp <= kQRebuildWarps) {
     // ---------------- codes: rebuild once per row, mask per class ----------------
-    // warp d rebuilds k rows 8 d .. 8 d + 7 of a stage (lane = 4 row + q); lane
-    // quarter q owns columns 32 q .. 32 q + 31 of the group, record word 4 sl + q
-    const int d = warp - 1, q = lane & 3;
+    // warp d rebuilds k rows 8 d .. 8 d + 7 of a stage (lane = row + 8 q); lane
+    // quarter q owns columns 32 q .. 32 q + 31 of the group, record word 4 sl + q.
+    // The 8 lanes of one 128-byte store phase then hold the 8 rows of one swizzle
+    // atom at the same column chunk, which the swizzle spreads over all 32 banks.
+    const int d = warp - 1, q = lane >> 3;
     const int w = 4 * sl + q;
-    const int kl = 8 * d + (lane >> 2);
+    const int kl = 8 * d + (lane & 7);
     const size_t rbytes = (size_t)record_bytes_for(kBmax);
     const uint32_t r8 = (uint32_t)(kl & 7);
     const uint32_t row_off = (uint32_t)((2 * (kl >> 3) + (q >> 1)) * 1024) + r8 * 128u;
