@@ -1102,6 +1102,7 @@ def run_prefill(args):
     except Exception:
         pass
     tflops_peak = float(peaks.get("bf16_tflops", 1590.0))
+    tflops_sust = float(peaks.get("bf16_tflops_sustained", 1400.0))
     hbm_peak, hbm_kind = _peaks()
     lin = []
     for li, (name, K, N) in enumerate(wl.LLAMA3_8B):
@@ -1150,6 +1151,7 @@ def run_prefill(args):
             out.append({"linear": d["name"], "K": K, "N": N, "tokens": T,
                         "prefill_tc_us": round(us_tc, 2), "tc_tflops": round(flops / (us_tc * 1e-6) / 1e12, 1),
                         "tc_frac": round(flops / (us_tc * 1e-6) / 1e12 / tflops_peak, 4),
+                        "tc_frac_sustained": round(flops / (us_tc * 1e-6) / 1e12 / tflops_sust, 4),
                         "dequant_gemm_us": round(us_all, 2),
                         "dequant_us": round(us_deq, 2), "tflops": round(flops / (us_all * 1e-6) / 1e12, 1),
                         "tflops_frac": round(flops / (us_all * 1e-6) / 1e12 / tflops_peak, 4),
@@ -1160,7 +1162,8 @@ def run_prefill(args):
     print(json.dumps({"metric": "prefill: us per linear and TFLOP/s of the fused tensor-core product "
                                 "(grinqh_prefill_tc) and of dequant + library fp16 GEMM (grinqh_prefill)",
                       "unit": "µs", "higher_is_better": False, "data": "synthetic",
-                      "peak_tflops": tflops_peak, "peak_gbs": hbm_peak, "peak_kind": hbm_kind,
+                      "peak_tflops": tflops_peak, "peak_tflops_sustained": tflops_sust, "peak_gbs": hbm_peak,
+                      "peak_kind": hbm_kind,
                       "config": {"workload": "llama3-8b linears, prefill of 512 and 2048 tokens, b_max 8 codes, "
                                              "two packed copies rotated"},
                       "points": out}))
