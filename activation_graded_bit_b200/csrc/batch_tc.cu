@@ -32,7 +32,7 @@
 // class 16 KB of codes and 8 KB of activations), so the roles meet once per stage:
 //   warp 0      allocates the TMEM columns and, from one lane, issues per step and
 //               class four K = 16 MMAs;
-//   warps 1..8  read a stage's plane words (two stages ahead), merge each row's
+//   warps 1..8  read a stage's plane words (three stages ahead), merge each row's
 //               codes once, and per class write the masked codes as binary16
 //               (the row's exponent byte over c, minus 2^pe 1024: exact) in the
 //               MN-major 128-byte-swizzled layout of the A descriptor; then the
@@ -72,7 +72,7 @@ constexpr int kQRebuildWarps = 8, kQBuildWarps = 8;
 constexpr int kQBuildThreads = 32 * kQBuildWarps;
 static_assert(kQBuildThreads >= 8 * kQMaxTok, "one 8-row chunk per grading thread");
 constexpr int kQThreads = 32 * (1 + kQRebuildWarps + kQBuildWarps);
-constexpr int kQAhead = 2;                       // stages a rebuild lane loads ahead
+constexpr int kQAhead = 3;                       // stages a rebuild lane loads ahead
 
 struct QSync {
   unsigned long long full_a[kQRing];   // one arrival per rebuild warp
@@ -245,6 +245,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
         v.m = 0u;
       }
     };
+    // the masks of the first kQCls active classes (every class when at most four are
+    // active) in registers: keep the exponent bytes and the top b bits of every code byte
+    uint32_t topc[kQCls];
+#pragma unroll
+    for (int ci = 0; ci < kQCls; ++ci) {
+      const uint32_t b = (ci < n_act) ? (uint32_t)sy.width[sy.act[ci]] : 8u;
+      topc[ci] = 0xFF00FF00u | (((0xFFu << (8u - b)) & 0xFFu) * 0x00010001u);
+    }
     QWords buf[kQAhead];
 #pragma unroll
     for (int i = 0; i < kQAhead; ++i)
@@ -282,10 +290,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
           ok = bar_wait(saddr(&sy.empty[slot]), ((uint32_t)(u / kQRing) & 1u) ^ 1u);
           if (!ok) break;
           const int ncl = min(kQCls, n_act - gi * kQCls);
-          for (int ci = 0; ci < ncl; ++ci) {
-          const uint32_t b = (uint32_t)sy.width[sy.act[gi * kQCls + ci]];
-          // keep the exponent bytes and the top b bits of every code byte
-          const uint32_t top = 0xFF00FF00u | (((0xFFu << (8u - b)) & 0xFFu) * 0x00010001u);
+#pragma unroll
+          for (int ci = 0; ci < kQCls; ++ci) {
+          if (ci >= ncl) break;
+          uint32_t top = topc[ci];
+          if (gi > 0) {
+            const uint32_t b = (uint32_t)sy.width[sy.act[gi * kQCls + ci]];
+            top = 0xFF00FF00u | (((0xFFu << (8u - b)) & 0xFFu) * 0x00010001u);
+          }
           const uint32_t row = a0 + slot * kQSlot + ci * kQABytes + row_off;
           uint32_t h[16];
 #pragma unroll
@@ -345,6 +357,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
       for (int i = 0; i < 8; ++i) th2[i] = __half2half2(__ushort_as_half(sy.thh[i]));
       const bool few = sy.n_th <= 4;
       const uint32_t actmask = sy.actmask;
+      uint32_t jxc[kQCls];   // the first kQCls active classes, one per byte
+#pragma unroll
+      for (int ci = 0; ci < kQCls; ++ci) jxc[ci] = (ci < n_act) ? (uint32_t)sy.act[ci] * 0x01010101u : 0u;
       __half2 amax = __float2half2_rn(0.0f);
       uint4 xn;
       uint32_t mn[8];
@@ -407,8 +422,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
           // % 8); Tp is a multiple of 16, so row Tp + t sits Tp * 128 bytes after row t
           const uint32_t off = (uint32_t)((t >> 3) * 1024 + (t & 7) * 128) + ((uint32_t)(kc ^ (t & 7)) << 4);
           const uint32_t lo_off = (uint32_t)Tp * 128u;
-          for (int ci = 0; ci < ncl; ++ci) {
-            const uint32_t jx = (uint32_t)sy.act[gi * kQCls + ci] * 0x01010101u;
+#pragma unroll
+          for (int ci = 0; ci < kQCls; ++ci) {
+            if (ci >= ncl) break;
+            const uint32_t jx = (gi == 0) ? jxc[ci] : (uint32_t)sy.act[gi * kQCls + ci] * 0x01010101u;
             const uint32_t sb = a0 + slot * kQSlot + kQCls * kQABytes + ci * kQBBytes;
             // bit 7 of a byte: that row's class differs (bytes are at most 15, so
             // adding 0x7F carries into no other byte)
